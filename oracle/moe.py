@@ -1,0 +1,134 @@
+"""Oracle: routing permutation and the MoE layer forward (test infrastructure only).
+
+Definitions followed
+--------------------
+* Routing ("grouped-nf4-gemm" README intro: one launch covers all active
+  experts; the decode glue's router epilogue and combine): the layer receives
+  top-k expert ids [T, k] and gate weights [T, k]. Slots ``s = t*k + j`` are
+  ordered expert by expert; within an expert, slots keep increasing ``s``
+  (a stable order). ``counts[e]`` = slots routed to e, ``offsets`` = the
+  exclusive prefix sum (E+1 entries, int64), ``perm[p]`` = the slot at
+  expert-ordered position p, ``inv_perm[s]`` = the position of slot s.
+* Layer (bitsandbytes PR #1984 Design: per-expert dequantise loop with a gated
+  SiLU activation; "experts4bit-qlora" README: fused ``gate_up_proj
+  [E, 2I, H]`` and ``down_proj [E, H, I]``; "grouped-nf4-gemm" README: the
+  fused kernel computes what dequantise-then-matmul computes):
+
+      [G | U]  = X_e . D(W_gu[e])^T      gate = rows 0..I-1, up = rows I..2I-1
+      h        = bf16_rne(silu(G) * U)
+      O        = h . D(W_d[e])^T
+      y[t]     = bf16_rne( sum_j gates[t, j] * O[slot t*k + j] )   (slot order)
+
+  where D is the parity-contract decode (``dequant_ref`` for NF4,
+  ``dequant_mxfp4`` for MXFP4) and everything else is fp64. The oracle rounds h
+  to bf16 because the fused layer stores h as bf16 between its two GEMMs.
+
+Parity pins (tests): routing invariants and a brute-force loop; the E=1, k=1,
+gate=1 case reduces to a dense SwiGLU MLP checked against torch on CPU; a
+pure-Python loop agrees with this module on tiny shapes.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .formats import (
+    bf16_round,
+    dequant_ref,
+    dequant_ref_exact,
+    dequant_mxfp4,
+)
+
+
+def route_ref(ids, E: int):
+    """Stable expert-contiguous order of the T*k routing slots.
+
+    ids: int [T, k] with values in [0, E). Returns (counts int32 [E],
+    offsets int64 [E+1], perm int32 [T*k], inv_perm int32 [T*k]).
+    """
+    flat = np.asarray(ids).reshape(-1).astype(np.int64)
+    if flat.size and (flat.min() < 0 or flat.max() >= E):
+        raise ValueError("expert id out of range")
+    counts = np.bincount(flat, minlength=E).astype(np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.argsort(flat, kind="stable").astype(np.int32)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=np.int32)
+    return counts, offsets, perm, inv
+
+
+def swiglu_ref(G, U):
+    """silu(G) * U in fp64."""
+    G = np.asarray(G, np.float64)
+    return G / (1.0 + np.exp(-G)) * np.asarray(U, np.float64)
+
+
+def _decode(fmt, codes, scales, N, K, exact=False):
+    if fmt == "nf4":
+        if exact:
+            return dequant_ref_exact(codes, scales, N, K)
+        return dequant_ref(codes, scales, N, K).astype(np.float64)
+    if fmt == "mxfp4":
+        return dequant_mxfp4(codes, scales).reshape(N, K).astype(np.float64)
+    raise ValueError(fmt)
+
+
+def expert_tokens(ids, tokens=None):
+    """For each expert, the (slot, token) pairs routed to it, in slot order,
+    restricted to ``tokens`` when given."""
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    sel = np.arange(T) if tokens is None else np.asarray(tokens)
+    out = {}
+    for t in sel:
+        for j in range(k):
+            out.setdefault(int(ids[t, j]), []).append((int(t) * k + j, int(t)))
+    for e in out:
+        out[e].sort()
+    return out
+
+
+def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales,
+                    E, H, I, tokens=None, exact_decode=False, return_h=False):
+    """The MoE layer forward (per-expert dequantise-then-matmul loop).
+
+    x: bf16 values as any float array [T, H]; ids int [T, k]; gates fp32
+    [T, k]. Weights per expert: NF4 codes [E, 2I, H/2] + absmax [E, 2I, H/64]
+    and [E, H, I/2] + [E, H, I/64]; MXFP4 blocks [E, 2I, H/32, 16] + scales
+    [E, 2I, H/32] and [E, H, I/32, 16] + [E, H, I/32].
+
+    tokens: optional subset of token indices; only their outputs are computed
+    (an expert's weights are decoded only if a selected token uses it).
+    Returns y as fp64 holding bf16 values, [len(tokens) or T, H]; with
+    return_h, also {slot: h row (fp64 holding bf16 values)}.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ids = np.asarray(ids)
+    gates = np.asarray(gates, dtype=np.float32)
+    T, k = ids.shape
+    sel = np.arange(T) if tokens is None else np.asarray(tokens)
+    row_of = {int(t): i for i, t in enumerate(sel)}
+    acc = np.zeros((len(sel), H), dtype=np.float64)
+    # O for every selected slot, kept so the combine can run in slot order
+    O_slot = {}
+    h_slot = {}
+    for e, pairs in sorted(expert_tokens(ids, sel).items()):
+        Wgu = _decode(fmt, gu_codes[e], gu_scales[e], 2 * I, H, exact_decode)
+        Wd = _decode(fmt, dn_codes[e], dn_scales[e], H, I, exact_decode)
+        X = x[[t for _, t in pairs]]
+        GU = X @ Wgu.T
+        h = bf16_round(swiglu_ref(GU[:, :I], GU[:, I:]))
+        O = h @ Wd.T
+        for r, (s, _) in enumerate(pairs):
+            O_slot[s] = O[r]
+            h_slot[s] = h[r]
+        del Wgu, Wd
+    for t in sel:
+        for j in range(k):
+            s = int(t) * k + j
+            acc[row_of[int(t)]] += np.float64(gates[t, j]) * O_slot[s]
+    y = bf16_round(acc)
+    if return_h:
+        return y, h_slot
+    return y
