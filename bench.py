@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the packed-4-bit MoE layer forward on B200.
+
+Default workload: the small-M decode layer, NF4, E=8 experts, H=4096,
+I=14336, top-2, T=16 tokens (weights N(0, 0.02) fp32 drawn on the GPU and
+packed by the library's quantiser; x N(0, 1) in bf16; N(0, 1) router logits,
+top-2 and a softmax over the chosen two). One step = one layer forward:
+routing pass, gate_up grouped GEMM with SwiGLU, down grouped GEMM with the
+weighted combine, bf16 output.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl e4b|reference]
+                    [--workload NAME] [--T T] [--sweep]
+
+Prints one JSON line (rank 0). Under torchrun (N > 1) every rank runs its own
+batch of T tokens on its own GPU with replicated weights and no collective on
+the data path (weak scaling); the timed region is bracketed by barriers and
+the max over ranks is reported. --impl reference times the CPU oracle on the
+host cores instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and packed-weight HBM GB/s (% roofline) on 1 B200"
+DEFAULT_WORKLOAD = "decode_nf4_E8_H4096_I14336_top2"
+DEFAULT_T = 16
+L2_BYTES = 126 * 2 ** 20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["e4b", "reference"], default="e4b")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--sweep", action="store_true",
+                    help="print one line per workload and token count (no cpu baseline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_grouped_moe_e4b_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(key: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        rec = d[key][kernel]
+        if rec.get("source_hash") != _source_hash():
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def build_layer(wl, device):
+    import torch
+    from bit_grouped_moe_e4b_b200 import e4b, synth
+
+    packed = []
+    for which in ("gate_up", "down"):
+        w = synth.layer_weights(wl, which, device)
+        packed += list(e4b.quantize(wl.fmt, w))
+        del w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return e4b.PackedLayer(wl.fmt, wl.E, wl.H, wl.I, *packed)
+
+
+def kernel_bytes(wl, T, ids):
+    """Algorithmic bytes per launch of each kernel."""
+    # storage per weight: 4-bit code + fp32 absmax per 64 (NF4) or one e8m0 byte per 32 (MXFP4)
+    bpw = 0.5 + (4.0 / 64 if wl.fmt == "nf4" else 1.0 / 32)
+    active = len(np.unique(ids))
+    R = ids.size
+    gu = active * 2 * wl.I * wl.H * bpw + 2 * T * wl.H + 4 * R
+    dn = active * wl.H * wl.I * bpw + 2 * T * wl.H + 4 * R
+    return {"gate_up": gu, "down": dn, "active_experts": active,
+            "packed_bytes": active * 3 * wl.H * wl.I * bpw,
+            "layer": active * 3 * wl.H * wl.I * bpw + 4 * T * wl.H + 8 * R}
+
+
+def run_gpu(wl, T, steps, warmup, rank, world, dist):
+    import torch
+    from bit_grouped_moe_e4b_b200 import e4b, synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layer = build_layer(wl, dev)
+    x_h = synth.tokens_bf16(wl, T)
+    ids_h, gates_h = synth.routing(wl, T)
+    x = x_h.to(dev)
+    ids = torch.from_numpy(ids_h).to(dev)
+    gates = torch.from_numpy(gates_h).to(dev)
+    ws = e4b.workspace(layer, T, wl.top_k, dev)
+    y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(warmup):
+        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws)
+    torch.cuda.synchronize()
+    status = e4b.e4b_read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    path = e4b.e4b_last_path()
+    launches_per_step = e4b.e4b_last_launch_count()
+
+    # timed region: inputs resident in HBM
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for row in ev:  # torch creates the CUDA event on first record
+        for e_ in row:
+            e_.record(stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for i in range(steps):
+        e4b.e4b_set_timing_events(ev[i])
+        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e4b.e4b_set_timing_events(None)
+    clk = clocks.stop()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    phases = {name: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(steps)]))
+              for name, a, b in (("route", 0, 1), ("gate_up", 1, 2), ("down", 2, 3), ("finalize", 3, 4))}
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end-to-end through the C ABI with host buffers (pinned), copies inside
+    x_pin = x_h.pin_memory()
+    ids_pin = torch.from_numpy(ids_h).pin_memory()
+    g_pin = torch.from_numpy(gates_h).pin_memory()
+    y_pin = torch.empty((T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+    ids_d = torch.empty_like(ids)
+    g_d = torch.empty_like(gates)
+    for _ in range(warmup):
+        x_d.copy_(x_pin, non_blocking=True)
+        e4b.e4b_moe_forward(layer, x_d, ids_d.copy_(ids_pin, non_blocking=True),
+                            g_d.copy_(g_pin, non_blocking=True), y, ws)
+        y_pin.copy_(y, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        x_d.copy_(x_pin, non_blocking=True)
+        ids_d.copy_(ids_pin, non_blocking=True)
+        g_d.copy_(g_pin, non_blocking=True)
+        e4b.e4b_moe_forward(layer, x_d, ids_d, g_d, y, ws)
+        y_pin.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if e4b.e4b_read_device_status(ws) != 0:
+        raise RuntimeError("device status set during the timed loops")
+    return {
+        "ms": ms, "phases": phases, "clocks": clk, "path": path,
+        "launches": launches_per_step * steps, "e2e_ms": e2e_ms,
+        "h2d": x_h.numel() * 2 + ids_h.nbytes + gates_h.nbytes, "d2h": T * wl.H * 2,
+        "ids": ids_h, "layer": layer, "x": x_h, "gates": gates_h,
+    }
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample(wl, T, ids, gates, x_h, slots):
+    """Times the CPU oracle on routed slots of the same workload: per slot,
+    the expert's decode + fp64 matmuls + bf16(h) (oracle.fast.expert_term).
+    The experts are packed by the oracle before timing. Returns seconds."""
+    import torch
+    from oracle import fast
+    from bit_grouped_moe_e4b_b200 import synth
+
+    fast.build()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    need = sorted({int(ids.reshape(-1)[s]) for s in slots})
+    packed = {}
+    for e in need:
+        for which in ("gate_up", "down"):
+            packed[(which, e)] = fast.quantize(wl.fmt, synth.expert_weight(wl, which, e, dev).cpu().numpy())
+    x = x_h.float().numpy().astype(np.float64)
+    t = time.perf_counter()
+    for s in slots:
+        e = int(ids.reshape(-1)[s])
+        fast.expert_term(wl.fmt, x[s // wl.top_k][None], packed[("gate_up", e)], packed[("down", e)],
+                         wl.H, wl.I)
+    return time.perf_counter() - t
+
+
+def run_reference(args, wl, T):
+    from bit_grouped_moe_e4b_b200 import synth
+
+    x_h = synth.tokens_bf16(wl, T)
+    ids, gates = synth.routing(wl, T)
+    R = ids.size
+    # one routed slot per step (a bounded sample: one expert term of one token)
+    if args.warmup:
+        oracle_sample(wl, T, ids, gates, x_h, [i % R for i in range(min(args.warmup, 2))])
+    slots = [(args.warmup + i) % R for i in range(args.steps)]
+    secs = oracle_sample(wl, T, ids, gates, x_h, slots)
+    tokens = len(slots) / wl.top_k
+    value = tokens / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": T, "format": wl.fmt, "E": wl.E, "H": wl.H, "I": wl.I,
+                   "top_k": wl.top_k},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} routed slots (one expert term of one token each: "
+                                   "decode gate_up and down, fp64 matmuls, bf16 h), weights packed "
+                                   "before timing"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from bit_grouped_moe_e4b_b200.configs import WORKLOADS
+
+    wl = WORKLOADS[args.workload]
+    T = args.T or (DEFAULT_T if args.workload == DEFAULT_WORKLOAD else wl.T[-1])
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl, T)
+        return
+
+    import torch
+    from bit_grouped_moe_e4b_b200 import build as builder
+
+    builder.build()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    hbm, bf16, bf16_sus, peak_src = _peaks()
+
+    cases = [(wl, T)]
+    if args.sweep:
+        cases = [(w, t) for w in WORKLOADS.values() for t in w.T]
+    for wl_i, T_i in cases:
+        r = run_gpu(wl_i, T_i, args.steps, args.warmup, rank, world, dist)
+        kb = kernel_bytes(wl_i, T_i, r["ids"])
+        dominant = max(("gate_up", "down"), key=lambda k: r["phases"][k])
+        dur_s = r["phases"][dominant] * 1e-3
+        achieved = kb[dominant] / dur_s / 1e9
+        step_s = r["ms"] * 1e-3 / args.steps
+        tokens_s = world * T_i / step_s
+        flops = 2.0 * r["ids"].size * 3 * wl_i.H * wl_i.I
+        key = f"{wl_i.name}_T{T_i}"
+        line = {
+            "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl_i.name, "T": T_i, "format": wl_i.fmt, "E": wl_i.E,
+                       "H": wl_i.H, "I": wl_i.I, "top_k": wl_i.top_k,
+                       "active_experts": kb["active_experts"], "path": ["none", "gemv", "tcgen05"][r["path"]],
+                       "weights": "N(0,0.02) fp32 packed on the GPU by e4b_quantize_*",
+                       "l2": "no flush: packed weights of the active experts "
+                             f"({kb['packed_bytes'] / 2 ** 20:.0f} MiB) exceed the 126 MB L2",
+                       "parallelism": f"replicas x{world}, token batches per GPU"},
+            "packed_gbs": kb["packed_bytes"] / step_s / 1e9,
+            "layer_frac_of_hbm": (kb["layer"] / step_s / 1e9) / hbm,
+            "tflops": flops / step_s / 1e12,
+            "phases_ms": r["phases"],
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_src,
+                         "traffic": _traffic(key, dominant),
+                         "algorithmic_bytes": kb[dominant]},
+            "clocks": r["clocks"],
+            "e2e": {"value": world * T_i / (r["e2e_ms"] * 1e-3 / args.steps), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": r["launches"],
+        }
+        if (not args.sweep and rank == 0 and world == 1 and not args.no_cpu_baseline):
+            slots = list(range(wl_i.top_k))  # one token: both of its slots
+            secs = oracle_sample(wl_i, T_i, r["ids"], r["gates"], r["x"], slots)
+            line["cpu_baseline"] = {
+                "value": 1.0 / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"token 0 of the batch ({wl_i.top_k} routed slots: decode gate_up and "
+                          "down of each expert, fp64 matmuls, bf16 h); single-threaded C core"}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        del r
+        torch.cuda.empty_cache()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

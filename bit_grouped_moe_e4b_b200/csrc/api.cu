@@ -1,0 +1,335 @@
+// The C ABI of libe4b: argument checks, workspace layout, path choice and
+// launch order. Every entry point is declared and documented in include/e4b.h.
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+using namespace e4b;
+
+thread_local int32_t g_last_path = E4B_PATH_NONE;
+thread_local int32_t g_last_launches = 0;
+thread_local cudaEvent_t g_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+thread_local bool g_timing = false;
+
+void mark(int i, cudaStream_t s) {
+  if (g_timing) cudaEventRecord(g_events[i], s);
+}
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace of the layer forward.
+struct MoeWs {
+  size_t status, counts, offsets, perm, inv, h, acc, total;
+};
+
+MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
+  MoeWs w;
+  const int64_t R = T * top_k;
+  size_t o = 0;
+  w.status = o;  o += kStatusBytes;
+  w.counts = o;  o = align_up(o + size_t(E) * 4, 256);
+  w.offsets = o; o = align_up(o + size_t(E + 1) * 8, 256);
+  w.perm = o;    o = align_up(o + size_t(R) * 4, 256);
+  w.inv = o;     o = align_up(o + size_t(R) * 4, 256);
+  w.h = o;       o = align_up(o + size_t(R) * size_t(I) * 2, 256);
+  w.acc = o;     o = align_up(o + size_t(T) * size_t(H) * 4, 256);
+  w.total = o;
+  return w;
+}
+
+e4b_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return E4B_OK;
+  return E4B_ERR_CUDA;
+}
+
+// Shape rules shared by both kernel families.
+e4b_status check_projection(int fmt, int64_t N, int64_t K, bool swiglu) {
+  if (fmt != E4B_FMT_NF4 && fmt != E4B_FMT_MXFP4) return E4B_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return E4B_ERR_INVALID_ARG;
+  if (N % (swiglu ? 32 : 16)) return E4B_ERR_UNSUPPORTED;
+  if (fmt == E4B_FMT_NF4 && K % E4B_NF4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (fmt == E4B_FMT_MXFP4 && K % E4B_MXFP4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  return E4B_OK;
+}
+
+// Small-M when an expert sees few rows on average; the tcgen05 kernel needs
+// E <= 256 for its on-chip expert table.
+bool choose_gemv(int64_t R, int64_t E, uint32_t flags) {
+  if (flags & E4B_FLAG_FORCE_GEMV) return true;
+  if (flags & E4B_FLAG_FORCE_TCGEN05) return false;
+  if (E > 256) return true;
+  return R <= 32 * E;
+}
+
+e4b_status run_projection(const GemmProblem& p, bool gemv, cudaStream_t st) {
+  const int sms = sm_count();
+  cudaError_t e = gemv ? launch_gemv(p, st, sms) : launch_tc_gemm(p, st, sms);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* e4b_version(void) { return "e4b 0.1.0 sm_100a"; }
+
+const char* e4b_status_string(int32_t s) {
+  switch (s) {
+    case E4B_OK: return "ok";
+    case E4B_ERR_INVALID_ARG: return "invalid argument";
+    case E4B_ERR_UNSUPPORTED: return "unsupported shape";
+    case E4B_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case E4B_ERR_CUDA: return "CUDA error";
+    case E4B_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case E4B_ERR_BAD_EXPERT_ID: return "expert id out of range";
+    case E4B_ERR_MISALIGNED: return "misaligned pointer or stride";
+    default: return "unknown status";
+  }
+}
+
+int32_t e4b_last_path(void) { return g_last_path; }
+
+e4b_status e4b_set_timing_events(void* const* events, int32_t n) {
+  if (n == 0) {
+    g_timing = false;
+    return E4B_OK;
+  }
+  if (n != 5 || !events) return E4B_ERR_INVALID_ARG;
+  for (int i = 0; i < 5; ++i) {
+    if (!events[i]) return E4B_ERR_INVALID_ARG;
+    g_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  g_timing = true;
+  return E4B_OK;
+}
+int32_t e4b_last_launch_count(void) { return g_last_launches; }
+
+e4b_status e4b_nf4_codebook(float* out_host) {
+  if (!out_host) return E4B_ERR_INVALID_ARG;
+  host_nf4_levels(out_host);
+  return E4B_OK;
+}
+
+e4b_status e4b_quantize_nf4(const float* w, int64_t E, int64_t N, int64_t K, int32_t blocksize,
+                            uint8_t* codes, float* absmax, void* stream) {
+  if (!w || !codes || !absmax || E <= 0 || N <= 0 || K <= 0) return E4B_ERR_INVALID_ARG;
+  if (blocksize != E4B_NF4_BLOCK || K % E4B_NF4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (!aligned16(w) || (reinterpret_cast<uintptr_t>(codes) & 3u) ||
+      (reinterpret_cast<uintptr_t>(absmax) & 3u))
+    return E4B_ERR_MISALIGNED;
+  const int64_t nblocks = E * N * (K / E4B_NF4_BLOCK);
+  return cuda_status(launch_quantize_nf4(w, nblocks, codes, absmax,
+                                         static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_quantize_mxfp4(const float* w, int64_t E, int64_t N, int64_t K, uint8_t* blocks,
+                              uint8_t* scales, void* stream) {
+  if (!w || !blocks || !scales || E <= 0 || N <= 0 || K <= 0) return E4B_ERR_INVALID_ARG;
+  if (K % E4B_MXFP4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (!aligned16(w) || (reinterpret_cast<uintptr_t>(blocks) & 3u)) return E4B_ERR_MISALIGNED;
+  const int64_t nblocks = E * N * (K / E4B_MXFP4_BLOCK);
+  return cuda_status(launch_quantize_mxfp4(w, nblocks, blocks, scales,
+                                           static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_dequantize(int32_t fmt, const uint8_t* codes, const void* scales, int64_t E,
+                          int64_t N, int64_t K, uint16_t* out, void* stream) {
+  if (!codes || !scales || !out || E <= 0 || N <= 0 || K <= 0) return E4B_ERR_INVALID_ARG;
+  if (fmt != E4B_FMT_NF4 && fmt != E4B_FMT_MXFP4) return E4B_ERR_INVALID_ARG;
+  if (fmt == E4B_FMT_NF4 && K % E4B_NF4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (fmt == E4B_FMT_MXFP4 && K % E4B_MXFP4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(codes) & 3u) || !aligned16(out)) return E4B_ERR_MISALIGNED;
+  if (fmt == E4B_FMT_NF4 && (reinterpret_cast<uintptr_t>(scales) & 3u)) return E4B_ERR_MISALIGNED;
+  return cuda_status(launch_dequantize(fmt, codes, scales, E * N * K, out,
+                                       static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_route_workspace_size(int64_t T, int32_t top_k, int32_t E, size_t* bytes) {
+  if (!bytes || T < 0 || top_k <= 0 || E <= 0) return E4B_ERR_INVALID_ARG;
+  *bytes = kStatusBytes;
+  return E4B_OK;
+}
+
+e4b_status e4b_route(const int32_t* ids, int64_t T, int32_t top_k, int32_t E, int32_t* counts,
+                     int64_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (T < 0 || top_k <= 0 || E <= 0) return E4B_ERR_INVALID_ARG;
+  if (!counts || !offsets || !ws || (T > 0 && (!ids || !perm || !inv_perm)))
+    return E4B_ERR_INVALID_ARG;
+  if (E > 1024 || T * int64_t(top_k) >= (int64_t(1) << 31)) return E4B_ERR_UNSUPPORTED;
+  if (ws_bytes < size_t(kStatusBytes)) return E4B_ERR_WORKSPACE_TOO_SMALL;
+  g_last_launches = 1;
+  return cuda_status(launch_route(ids, int32_t(T * top_k), E, counts, offsets, perm, inv_perm,
+                                  nullptr, static_cast<int32_t*>(ws),
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+e4b_status e4b_grouped_gemm(const e4b_gemm_args* a, uint32_t flags, void* stream) {
+  if (!a) return E4B_ERR_INVALID_ARG;
+  if (a->E <= 0 || a->top_k <= 0 || a->R_max < 0) return E4B_ERR_INVALID_ARG;
+  if (a->epilogue < E4B_EPI_STORE || a->epilogue > E4B_EPI_COMBINE) return E4B_ERR_INVALID_ARG;
+  e4b_status st = check_projection(a->fmt, a->N, a->K, a->epilogue == E4B_EPI_SWIGLU);
+  if (st != E4B_OK) return st;
+  if (!a->codes || !a->scales || !a->a || !a->offsets || !a->out) return E4B_ERR_INVALID_ARG;
+  if (a->epilogue == E4B_EPI_COMBINE && !a->gates) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(a->codes) || !aligned16(a->a) || !aligned16(a->out) || a->lda % 8 || a->ldo % 8)
+    return E4B_ERR_MISALIGNED;
+  if (a->lda < a->K) return E4B_ERR_INVALID_ARG;
+  if (a->R_max == 0) return E4B_OK;
+  const bool gemv = choose_gemv(a->R_max, a->E, flags);
+  if (!gemv && a->E > 256) return E4B_ERR_UNSUPPORTED;
+  GemmProblem p{};
+  p.fmt = a->fmt;
+  p.epilogue = a->epilogue;
+  p.E = a->E;
+  p.top_k = a->top_k;
+  p.N = a->N;
+  p.K = a->K;
+  p.R_max = a->R_max;
+  p.codes = a->codes;
+  p.scales = a->scales;
+  p.a = a->a;
+  p.lda = a->lda;
+  p.row_slot = a->a_row_slot;
+  p.out_slot = a->out_row_slot;
+  p.offsets = a->offsets;
+  p.gates = a->gates;
+  p.out = a->out;
+  p.ldo = a->ldo;
+  p.flags = flags;
+  g_last_path = gemv ? E4B_PATH_GEMV : E4B_PATH_TCGEN05;
+  g_last_launches = 1;
+  return run_projection(p, gemv, static_cast<cudaStream_t>(stream));
+}
+
+e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
+                                  size_t* bytes) {
+  if (!w || !bytes || T < 0 || top_k <= 0 || w->E <= 0 || w->H <= 0 || w->I <= 0)
+    return E4B_ERR_INVALID_ARG;
+  *bytes = moe_ws_layout(w->E, w->H, w->I, T, top_k).total;
+  return E4B_OK;
+}
+
+e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
+                           const int32_t* ids, const float* gates, uint16_t* y, void* ws,
+                           size_t ws_bytes, uint32_t flags, void* stream) {
+  if (!w || T < 0 || top_k <= 0) return E4B_ERR_INVALID_ARG;
+  const int64_t E = w->E, H = w->H, I = w->I;
+  if (E <= 0 || H <= 0 || I <= 0 || top_k > E) return E4B_ERR_INVALID_ARG;
+  e4b_status st = check_projection(w->fmt, 2 * I, H, true);
+  if (st != E4B_OK) return st;
+  st = check_projection(w->fmt, H, I, false);
+  if (st != E4B_OK) return st;
+  if (H % 8) return E4B_ERR_UNSUPPORTED;
+  if (E > 1024 || T * int64_t(top_k) >= (int64_t(1) << 31)) return E4B_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (T == 0) return E4B_OK;
+  if (!x || !ids || !gates || !y || !ws || !w->gate_up_codes || !w->gate_up_scales ||
+      !w->down_codes || !w->down_scales)
+    return E4B_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || !aligned16(w->gate_up_codes) ||
+      !aligned16(w->down_codes) || !aligned16(w->gate_up_scales) || !aligned16(w->down_scales))
+    return E4B_ERR_MISALIGNED;
+  const MoeWs L = moe_ws_layout(E, H, I, T, top_k);
+  if (ws_bytes < L.total) return E4B_ERR_WORKSPACE_TOO_SMALL;
+
+  const int64_t R = T * top_k;
+  const bool gemv = choose_gemv(R, E, flags);
+  if (!gemv && E > 256) return E4B_ERR_UNSUPPORTED;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(base + L.status);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + L.counts);
+  int64_t* offsets = reinterpret_cast<int64_t*>(base + L.offsets);
+  int32_t* perm = reinterpret_cast<int32_t*>(base + L.perm);
+  int32_t* inv = reinterpret_cast<int32_t*>(base + L.inv);
+  uint16_t* h = reinterpret_cast<uint16_t*>(base + L.h);
+  float* acc = reinterpret_cast<float*>(base + L.acc);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  mark(0, s);
+  cudaError_t ce = launch_route(ids, int32_t(R), int32_t(E), counts, offsets, perm, inv, nullptr,
+                                status, s);
+  if (ce != cudaSuccess) return E4B_ERR_CUDA;
+
+  GemmProblem g{};
+  g.fmt = w->fmt;
+  g.epilogue = E4B_EPI_SWIGLU;
+  g.E = int(E);
+  g.top_k = top_k;
+  g.N = 2 * I;
+  g.K = H;
+  g.R_max = R;
+  g.codes = w->gate_up_codes;
+  g.scales = w->gate_up_scales;
+  g.a = x;
+  g.lda = H;
+  g.row_slot = perm;
+  g.out_slot = perm;
+  g.offsets = offsets;
+  g.out = h;
+  g.ldo = I;
+  g.zero_buf = acc;
+  g.zero_count = T * H;
+  g.status = status;
+  g.flags = flags;
+  mark(1, s);
+  st = run_projection(g, gemv, s);
+  if (st != E4B_OK) return st;
+
+  GemmProblem d = g;
+  d.epilogue = E4B_EPI_COMBINE;
+  d.N = H;
+  d.K = I;
+  d.codes = w->down_codes;
+  d.scales = w->down_scales;
+  d.a = h;
+  d.lda = I;
+  d.row_slot = nullptr;
+  d.out_slot = perm;
+  d.gates = gates;
+  d.out = acc;
+  d.ldo = H;
+  d.zero_buf = nullptr;
+  d.zero_count = 0;
+  mark(2, s);
+  st = run_projection(d, gemv, s);
+  if (st != E4B_OK) return st;
+
+  mark(3, s);
+  ce = launch_finalize(acc, T * H, y, s, sm_count());
+  if (ce != cudaSuccess) return E4B_ERR_CUDA;
+  mark(4, s);
+  g_last_path = gemv ? E4B_PATH_GEMV : E4B_PATH_TCGEN05;
+  g_last_launches = 4;
+  return E4B_OK;
+}
+
+e4b_status e4b_read_device_status(void* ws, int32_t* status_host, void* stream) {
+  if (!ws || !status_host) return E4B_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return E4B_ERR_CUDA;
+  int32_t v[2] = {0, 0};
+  if (cudaMemcpy(v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return E4B_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(v)) != cudaSuccess) return E4B_ERR_CUDA;
+  *status_host = v[0];
+  return E4B_OK;
+}
+
+}  // extern "C"

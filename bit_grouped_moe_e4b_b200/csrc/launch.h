@@ -1,0 +1,53 @@
+// Internal host-side launchers shared by the C-ABI layer (api.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "e4b.h"
+
+namespace e4b {
+
+cudaError_t launch_quantize_nf4(const float* w, int64_t nblocks, uint8_t* codes, float* absmax,
+                                cudaStream_t st, int sms);
+cudaError_t launch_quantize_mxfp4(const float* w, int64_t nblocks, uint8_t* blocks, uint8_t* scales,
+                                  cudaStream_t st, int sms);
+cudaError_t launch_dequantize(int fmt, const uint8_t* codes, const void* scales, int64_t nweights,
+                              uint16_t* out, cudaStream_t st, int sms);
+void host_nf4_levels(float* out);
+
+size_t route_smem_bytes(int32_t E);
+cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* counts, int64_t* offsets,
+                         int32_t* perm, int32_t* inv, int32_t* active, int32_t* status,
+                         cudaStream_t st);
+
+// Description of one grouped projection as the kernels see it.
+struct GemmProblem {
+  int fmt;          // e4b_format
+  int epilogue;     // e4b_epilogue
+  int E;
+  int top_k;
+  int64_t N, K;     // weight rows (both halves for SWIGLU), inner dim
+  int64_t R_max;    // bound on offsets[E]
+  const uint8_t* codes;
+  const void* scales;
+  const uint16_t* a;
+  int64_t lda;
+  const int32_t* row_slot;  // may be null: row p reads a[p]; else a[row_slot[p] / top_k]
+  const int32_t* out_slot;  // COMBINE: slot of row p (p when null)
+  const int64_t* offsets;   // [E+1]
+  const float* gates;       // COMBINE
+  void* out;
+  int64_t ldo;
+  float* zero_buf;          // optional buffer the kernel clears first (fp32 accumulator)
+  int64_t zero_count;       // floats in zero_buf
+  int32_t* status;          // device status word or null
+  uint32_t flags;
+};
+
+cudaError_t launch_gemv(const GemmProblem& p, cudaStream_t st, int sms);
+cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms);
+cudaError_t launch_finalize(const float* acc, int64_t n, uint16_t* y, cudaStream_t st, int sms);
+
+}  // namespace e4b

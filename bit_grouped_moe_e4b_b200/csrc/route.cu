@@ -1,0 +1,147 @@
+// Routing pass: per-expert histogram, prefix scan, and a stable scatter of the
+// T*top_k routing slots into expert-contiguous order, in one CTA.
+//
+// "grouped-nf4-gemm" README, intro: one launch covers all active experts of a
+// projection, which needs the routed rows grouped by expert; the decode glue
+// lists a router epilogue in front of the grouped GEMM.
+//
+// The 32 warps of the CTA own consecutive ranges of slots and walk them in
+// 32-slot pieces. __match_any_sync groups the lanes of a piece that share an
+// expert, so ranks inside a piece come from a popcount and the order of slots
+// within an expert is the slot order (stable), as the layer's combine and the
+// oracle both assume.
+#include "common.cuh"
+#include "launch.h"
+
+namespace e4b {
+
+constexpr int kRouteThreads = 1024;
+constexpr int kRouteWarps = kRouteThreads / 32;
+
+__global__ void __launch_bounds__(kRouteThreads, 1)
+route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __restrict__ counts,
+             int64_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+             int32_t* __restrict__ active, int32_t* __restrict__ status) {
+  extern __shared__ int32_t smem[];
+  int32_t* wcnt = smem;                        // [kRouteWarps][E] counts, then bases
+  int32_t* scan = smem + kRouteWarps * E;      // [kRouteThreads] scan scratch
+  __shared__ int32_t s_bad;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) wcnt[i] = 0;
+  if (tid == 0) {
+    s_bad = 0;
+    // The status word describes the most recent call: route runs first.
+    if (status) {
+      status[0] = 0;
+      status[1] = 0;
+    }
+  }
+  __syncthreads();
+
+  const int32_t chunk = (R + kRouteWarps - 1) / kRouteWarps;
+  const int32_t beg = min(R, warp * chunk);
+  const int32_t end = min(R, beg + chunk);
+  int32_t* my = wcnt + warp * E;
+
+  // pass 1: per-warp histogram
+  for (int32_t s0 = beg; s0 < end; s0 += 32) {
+    const int32_t s = s0 + lane;
+    const bool in = s < end;
+    int32_t e = in ? ids[s] : -1;
+    const bool ok = in && e >= 0 && e < E;
+    if (in && !ok) atomicAdd(&s_bad, 1);
+    if (!ok) e = -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    if (ok && lane == leader) my[e] += __popc(peers);
+  }
+  __syncthreads();
+
+  // per expert: totals and per-warp exclusive bases
+  int32_t total = 0;
+  if (tid < E) {
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int32_t c = wcnt[w * E + tid];
+      wcnt[w * E + tid] = total;
+      total += c;
+    }
+  }
+  // block-wide exclusive scan of totals over experts (E <= 1024)
+  scan[tid] = (tid < E) ? total : 0;
+  __syncthreads();
+  for (int d = 1; d < kRouteThreads; d <<= 1) {
+    const int32_t v = tid >= d ? scan[tid - d] : 0;
+    __syncthreads();
+    scan[tid] += v;
+    __syncthreads();
+  }
+  const int32_t incl = scan[tid];
+  const int32_t excl = incl - ((tid < E) ? total : 0);
+  if (tid < E) {
+    counts[tid] = total;
+    offsets[tid] = excl;
+    for (int w = 0; w < kRouteWarps; ++w) wcnt[w * E + tid] += excl;
+  }
+  if (tid == E - 1) offsets[E] = incl;
+  __syncthreads();
+
+  // active-expert list for the small-M kernels: active[0] = count, then ids
+  if (active) {
+    scan[tid] = (tid < E && total > 0) ? 1 : 0;
+    __syncthreads();
+    for (int d = 1; d < kRouteThreads; d <<= 1) {
+      const int32_t v = tid >= d ? scan[tid - d] : 0;
+      __syncthreads();
+      scan[tid] += v;
+      __syncthreads();
+    }
+    if (tid < E && total > 0) active[scan[tid]] = tid;  // 1-based slot
+    if (tid == kRouteThreads - 1) active[0] = scan[tid];
+  }
+
+  // pass 2: stable scatter
+  for (int32_t s0 = beg; s0 < end; s0 += 32) {
+    const int32_t s = s0 + lane;
+    const bool in = s < end;
+    int32_t e = in ? ids[s] : -1;
+    const bool ok = in && e >= 0 && e < E;
+    if (!ok) e = -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    int32_t pos = -1;
+    if (ok) {
+      pos = my[e] + __popc(peers & ((1u << lane) - 1u));
+      perm[pos] = s;
+    }
+    if (in) inv[s] = pos;
+    __syncwarp();
+    if (ok && lane == leader) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  if (tid == 0 && s_bad) {
+    record_status(status, E4B_ERR_BAD_EXPERT_ID);
+    atomicAdd(status + 1, s_bad);
+  }
+}
+
+size_t route_smem_bytes(int32_t E) { return size_t(kRouteWarps) * E * 4 + kRouteThreads * 4; }
+
+cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* counts, int64_t* offsets,
+                         int32_t* perm, int32_t* inv, int32_t* active, int32_t* status,
+                         cudaStream_t st) {
+  const size_t smem = route_smem_bytes(E);
+  static bool configured = false;  // the attribute is per function, set once
+  if (!configured) {
+    cudaError_t err = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(route_smem_bytes(1024)));
+    if (err != cudaSuccess) return err;
+    configured = true;
+  }
+  route_kernel<<<1, kRouteThreads, smem, st>>>(ids, R, E, counts, offsets, perm, inv, active, status);
+  return cudaGetLastError();
+}
+
+}  // namespace e4b

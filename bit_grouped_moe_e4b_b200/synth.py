@@ -2,10 +2,10 @@
 
 This module draws random numbers and nothing else: it holds none of the
 layer's arithmetic (no quantisation, decode, routing permutation, GEMM or
-activation). Every stream is a numpy PCG64 generator keyed by
-SeedSequence([seed, T, stream]) for token-side data and
-SeedSequence([hash(layer), stream, expert]) for weights, so one expert's
-weights can be regenerated on their own.
+activation). Token-side streams are numpy PCG64 generators keyed by
+SeedSequence([seed, T, stream]); weights come from torch's generator seeded
+from SeedSequence([hash(layer), stream, expert]), so one expert's weights can
+be regenerated on their own, on the device that uses them.
 
 Streams: 0 = x, 1 = router logits, 2 = per-expert logit bias, 3 = gate_up
 weights, 4 = down weights.
@@ -36,16 +36,33 @@ def _layer_key(layer: str) -> int:
     return zlib.crc32(layer.encode())
 
 
-def expert_weight(wl: Workload, which: str, e: int) -> np.ndarray:
-    """fp32 weights of expert e: "gate_up" [2I, H] or "down" [H, I], N(0, std)."""
+def _weight_seed(wl: Workload, stream: int, e: int) -> int:
+    ss = np.random.SeedSequence([_layer_key(wl.layer), stream, e])
+    return int(ss.generate_state(1, np.uint64)[0] & np.uint64(0x7FFFFFFFFFFFFFFF))
+
+
+def expert_weight(wl: Workload, which: str, e: int, device="cpu") -> torch.Tensor:
+    """fp32 weights of expert e: "gate_up" [2I, H] or "down" [H, I], N(0, std).
+
+    Drawn by torch's seeded generator on `device` (Philox on a GPU), so
+    full-size stacks are generated where they are used; a test hands the
+    oracle a host copy of the very same tensor. The values depend on the
+    device's generator, not only on the seed."""
     if which == "gate_up":
         shape, stream = (2 * wl.I, wl.H), GATE_UP_STREAM
     elif which == "down":
         shape, stream = (wl.H, wl.I), DOWN_STREAM
     else:
         raise ValueError(which)
-    g = _rng(_layer_key(wl.layer), stream, e)
-    return g.standard_normal(shape, dtype=np.float32) * np.float32(wl.weight_std)
+    g = torch.Generator(device=device)
+    g.manual_seed(_weight_seed(wl, stream, e))
+    w = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return w * wl.weight_std
+
+
+def layer_weights(wl: Workload, which: str, device="cpu") -> torch.Tensor:
+    """The stacked fp32 weights [E, ...] of one projection."""
+    return torch.stack([expert_weight(wl, which, e, device) for e in range(wl.E)])
 
 
 def tokens_bf16(wl: Workload, T: int) -> torch.Tensor:

@@ -1,0 +1,267 @@
+/*
+ * e4b.h -- packed-4-bit Mixture-of-Experts layer for B200 (sm_100a), C ABI.
+ *
+ * One MoE layer run directly on 4-bit-packed fused expert stacks:
+ * gate_up_proj [E, 2I, H] and down_proj [E, H, I] stored as NF4 (16-level
+ * NormalFloat codebook, two codes per byte, fp32 absmax per 64 weights along
+ * the input dimension, every expert quantised on its own) or as MXFP4 (OCP
+ * e2m1 codes, one e8m0 scale per 32 weights). One launch covers all active
+ * experts of a projection; weights are decoded on the fly through a 16-entry
+ * per-block table; products accumulate in fp32; no bf16 copy of a weight
+ * stack is ever written to memory.
+ *
+ * Sources (page titles; sections):
+ *   [G]  "grouped-nf4-gemm" README: intro (one launch for all active experts,
+ *        LUT decode, blockwise scaling, fp32 accumulation, bf16 epilogue; NF4
+ *        on the bitsandbytes gemm_4bit layout; MXFP4 as OCP e2m1 + e8m0);
+ *        "Try it on CPU right now" blocks 1-2 (quantize_pack_nf4 -> packed
+ *        [N, K/2] u8 + absmax [N, K/64] f32; quantize_pack_mxfp4 -> blocks
+ *        [N, K/32, 16] u8 + scales [N, K/32] u8); "Which entry point?" table.
+ *   [P]  bitsandbytes PR #1984 "Experts4bit": Summary and Design (per-expert
+ *        quantisation with per-expert absmax, per-expert dequantise loop,
+ *        gated SiLU / SwiGLU activation).
+ *   [Q]  "experts4bit-qlora" README: fused gate_up_proj / down_proj stacks
+ *        (transformers v5 layout).
+ *
+ * Conventions for every entry point
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *     its comment says "host". The library allocates and frees nothing and
+ *     keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every
+ *     call only enqueues work on that stream and returns without waiting,
+ *     except the few marked "synchronises".
+ *   - Argument errors are returned before anything is enqueued. Errors the
+ *     GPU detects (an expert id outside [0, E), a bounded wait that gave up)
+ *     are recorded in the workspace's status word; read it with
+ *     e4b_read_device_status.
+ *   - Element counts and offsets are 64-bit. bf16 values are passed as their
+ *     16-bit patterns (uint16_t).
+ *   - There is no fallback: a shape the kernels do not support returns
+ *     E4B_ERR_UNSUPPORTED.
+ */
+#ifndef E4B_H_
+#define E4B_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  E4B_OK = 0,
+  E4B_ERR_INVALID_ARG = 1,         /* null pointer, negative size, k > E ... */
+  E4B_ERR_UNSUPPORTED = 2,         /* shape outside what the kernels handle */
+  E4B_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size query */
+  E4B_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  E4B_ERR_DEVICE_TIMEOUT = 5,      /* (device) a bounded wait gave up */
+  E4B_ERR_BAD_EXPERT_ID = 6,       /* (device) an id outside [0, E); the slot is dropped */
+  E4B_ERR_MISALIGNED = 7           /* a pointer or row stride breaks 16-byte alignment */
+} e4b_status;
+
+typedef enum { E4B_FMT_NF4 = 0, E4B_FMT_MXFP4 = 1 } e4b_format;
+
+/* Which kernel family ran last (e4b_last_path). */
+typedef enum {
+  E4B_PATH_NONE = 0,
+  E4B_PATH_GEMV = 1,   /* small-M: register-fed mma.sync streaming the packed bytes */
+  E4B_PATH_TCGEN05 = 2 /* large-M: TMA + on-the-fly decode + tcgen05 MMA into TMEM */
+} e4b_path;
+
+/* Flags for e4b_moe_forward / e4b_grouped_gemm. */
+#define E4B_FLAG_FORCE_GEMV 0x1u     /* use the small-M path whatever the shape */
+#define E4B_FLAG_FORCE_TCGEN05 0x2u  /* use the tcgen05 path whatever the shape */
+#define E4B_FLAG_TEST_TIMEOUT 0x4u   /* bounded waits give up at once (tests the error path) */
+
+/* NF4 block size (weights per absmax) and MXFP4 block size (weights per scale). */
+#define E4B_NF4_BLOCK 64
+#define E4B_MXFP4_BLOCK 32
+
+/*
+ * A layer's packed expert stacks [Q, G].
+ *   NF4:   gate_up_codes  uint8 [E, 2I, H/2]  (two codes per byte, the earlier
+ *                                              weight in the high nibble)
+ *          gate_up_scales float [E, 2I, H/64] (absmax per 64 weights)
+ *          down_codes     uint8 [E, H, I/2]
+ *          down_scales    float [E, H, I/64]
+ *   MXFP4: gate_up_codes  uint8 [E, 2I, H/32, 16] (the earlier weight in the low nibble)
+ *          gate_up_scales uint8 [E, 2I, H/32]     (e8m0: value 2^(byte-127))
+ *          down_codes     uint8 [E, H, I/32, 16]
+ *          down_scales    uint8 [E, H, I/32]
+ * Rows 0..I-1 of gate_up are the gate projection, rows I..2I-1 the up
+ * projection. All four arrays must be 16-byte aligned.
+ */
+typedef struct {
+  int32_t fmt; /* e4b_format */
+  int32_t E, H, I;
+  const uint8_t* gate_up_codes;
+  const void* gate_up_scales;
+  const uint8_t* down_codes;
+  const void* down_scales;
+} e4b_moe_weights;
+
+/* ---------------------------------------------------------------- formats */
+
+/*
+ * e4b_quantize_nf4 -- [G] CPU block 1 (quantize_pack_nf4), [P] Summary.
+ * w: float [E, N, K] row-major. For each expert, row and block of
+ * `blocksize` weights along K: absmax = max|w|; every weight gets the index of
+ * the NF4 level nearest to fp32(w / absmax) (ties to the lower index; an
+ * all-zero block gets the zero level, index 7). Writes codes uint8
+ * [E, N, K/2] (earlier weight in the high nibble) and absmax float
+ * [E, N, K/blocksize]. blocksize must be 64; K % 64 == 0.
+ */
+e4b_status e4b_quantize_nf4(const float* w, int64_t E, int64_t N, int64_t K, int32_t blocksize,
+                            uint8_t* codes, float* absmax, void* stream);
+
+/*
+ * e4b_quantize_mxfp4 -- [G] intro and CPU block 2 (quantize_pack_mxfp4),
+ * OCP Microscaling v1.0. w: float [E, N, K], K % 32 == 0. Per 32-weight
+ * block: scale exponent e = floor(log2 max|w|) - 2 clamped to [-127, 127]
+ * (byte e + 127; an all-zero block gets byte 0 and zero codes); each weight
+ * w / 2^e rounds to the nearest e2m1 value (ties to even, saturating at 6),
+ * sign bit copied from w. Writes blocks uint8 [E, N, K/32, 16] (earlier
+ * weight in the low nibble) and scales uint8 [E, N, K/32].
+ */
+e4b_status e4b_quantize_mxfp4(const float* w, int64_t E, int64_t N, int64_t K,
+                              uint8_t* blocks, uint8_t* scales, void* stream);
+
+/*
+ * e4b_dequantize -- [G] CPU block 1 (dequant_ref) / block 2 (dequant_mxfp4).
+ * Decodes a packed stack [E, N, K] to bf16 out [E, N, K] with exactly the
+ * per-block table the GEMM kernels use: NF4 weight = bf16_rne(fp32(level) *
+ * absmax), MXFP4 weight = sign * e2m1 * 2^(scale-127) (exact in bf16). For
+ * tests of the decode; the layer never calls it.
+ */
+e4b_status e4b_dequantize(int32_t fmt, const uint8_t* codes, const void* scales, int64_t E,
+                          int64_t N, int64_t K, uint16_t* out, void* stream);
+
+/* Host: copies the library's 16 NF4 levels (fp32, ascending) into out[16]. */
+e4b_status e4b_nf4_codebook(float* out_host);
+
+/* ---------------------------------------------------------------- routing */
+
+/* Host: bytes of workspace e4b_route needs for these sizes (always > 0). */
+e4b_status e4b_route_workspace_size(int64_t T, int32_t top_k, int32_t E, size_t* bytes);
+
+/*
+ * e4b_route -- [G] intro (one launch over all active experts needs the
+ * routed rows grouped by expert). ids: int32 [T, top_k] expert per slot
+ * (slot s = t*top_k + j). Writes counts int32 [E] (slots per expert),
+ * offsets int64 [E+1] (exclusive prefix sum), perm int32 [T*top_k] (perm[p]
+ * = the slot at expert-ordered position p; within an expert slots keep
+ * increasing order) and inv_perm int32 [T*top_k] (position of each slot).
+ * An id outside [0, E) sets E4B_ERR_BAD_EXPERT_ID in ws's status word and
+ * its slot is left out (offsets[E] then counts the valid slots; inv_perm of a
+ * dropped slot is -1). ws: device scratch of e4b_route_workspace_size bytes.
+ * Requires E <= 1024 and T*top_k < 2^31.
+ */
+e4b_status e4b_route(const int32_t* ids, int64_t T, int32_t top_k, int32_t E, int32_t* counts,
+                     int64_t* offsets, int32_t* perm, int32_t* inv_perm, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ grouped GEMM */
+
+typedef enum {
+  E4B_EPI_STORE = 0,   /* out bf16 [R, N]: row p = A_p . W_e^T */
+  E4B_EPI_SWIGLU = 1,  /* out bf16 [R, N/2]: silu(gate) * up, gate = rows [0, N/2) */
+  E4B_EPI_COMBINE = 2  /* out fp32 [T, N] += gates[s] * (A_p . W_e^T), s = row_slot[p],
+                          t = s / top_k; the caller zeroes out beforehand */
+} e4b_epilogue;
+
+/*
+ * One projection of all experts in one launch ([G] intro: the grouped GEMM
+ * over all active experts on packed weights, fp32 accumulation, bf16
+ * epilogue). Rows of expert e are [offsets[e], offsets[e+1]); row p multiplies
+ * the bf16 activation row a[(a_row_slot ? a_row_slot[p] / top_k : p) * lda ..
+ * + K) with the decoded weight stack W [E, N, K] (codes / scales laid out as
+ * in e4b_moe_weights). R = offsets[E] rows are produced.
+ *   STORE:   out bf16, row p at out + p*ldo, N values.
+ *   SWIGLU:  out bf16, row p at out + p*ldo, N/2 values silu(g)*u with g the
+ *            row's first N/2 outputs (weight rows 0..N/2-1), u the rest.
+ *   COMBINE: out fp32 [T, ldo]; with s = out_row_slot[p] (p if NULL) and
+ *            t = s / top_k: out[t, n] += gates[s] * (row p output n). The
+ *            caller zeroes out first; the sum order over slots is not fixed.
+ * N must be a multiple of 16 (32 for SWIGLU), K of 64 (NF4) or 32 (MXFP4),
+ * lda and ldo multiples of 8; a, codes and out 16-byte aligned.
+ */
+typedef struct {
+  int32_t fmt;      /* e4b_format */
+  int32_t epilogue; /* e4b_epilogue */
+  int32_t E;
+  int32_t top_k;    /* slots per token (1 when rows are not routing slots) */
+  int64_t N, K;     /* weight rows and inner dimension */
+  int64_t R_max;    /* upper bound on offsets[E], i.e. rows of the row buffers */
+  const uint8_t* codes;        /* [E, N, K/2] */
+  const void* scales;          /* NF4 float [E, N, K/64]; MXFP4 uint8 [E, N, K/32] */
+  const uint16_t* a;           /* bf16 activations */
+  int64_t lda;                 /* elements between activation rows */
+  const int32_t* a_row_slot;   /* optional [R_max]: gather map for activation rows */
+  const int32_t* out_row_slot; /* COMBINE, optional [R_max]: routing slot of each row */
+  const int64_t* offsets;      /* [E+1] */
+  const float* gates;          /* COMBINE: [T*top_k] weight of each slot */
+  void* out;
+  int64_t ldo;                 /* elements between output rows */
+} e4b_gemm_args;
+
+e4b_status e4b_grouped_gemm(const e4b_gemm_args* args, uint32_t flags, void* stream);
+
+/* ---------------------------------------------------------- whole layer */
+
+/* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots. */
+e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
+                                  size_t* bytes);
+
+/*
+ * e4b_moe_forward -- the MoE layer ([P] Design: per-expert gate_up GEMM,
+ * gated SiLU, down GEMM, weighted sum over the chosen experts; [G] intro: one
+ * launch per projection over all active experts on the packed bytes).
+ *   x     bf16 [T, H] (16-byte aligned rows: H % 8 == 0)
+ *   ids   int32 [T, top_k] expert of each slot (duplicates allowed)
+ *   gates float [T, top_k] weight of each slot
+ *   y     bf16 [T, H] output: y[t] = bf16( sum_j gates[t,j] * down_e(
+ *         bf16(silu(gate_e(x[t])) * up_e(x[t])) ) ), e = ids[t,j]
+ *   ws    device scratch of e4b_moe_workspace_size bytes (routing, the bf16
+ *         intermediate h [T*top_k, I], an fp32 accumulator [T, H], status)
+ *   flags E4B_FLAG_* (0 = choose the path from the shape)
+ * The path is chosen on the host from T*top_k/E with no device sync, so the
+ * call is graph-capturable. T == 0 is a no-op.
+ */
+e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
+                           const int32_t* ids, const float* gates, uint16_t* y, void* ws,
+                           size_t ws_bytes, uint32_t flags, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word that
+ * e4b_route / e4b_moe_forward keep at the start of ws. *status_host receives
+ * an e4b_status (E4B_OK if the GPU reported nothing). */
+e4b_status e4b_read_device_status(void* ws, int32_t* status_host, void* stream);
+
+/*
+ * Host: instrumentation for benchmarks. With n == 5, every later
+ * e4b_moe_forward call on this thread records events[0..4] (cudaEvent_t,
+ * created by the caller) on its stream before the routing kernel, before the
+ * gate_up kernel, before the down kernel, before the output conversion and
+ * after it. n == 0 switches recording off. The library does not own the events.
+ */
+e4b_status e4b_set_timing_events(void* const* events, int32_t n);
+
+/* Host: the path the most recent e4b_moe_forward / e4b_grouped_gemm call on
+ * this thread enqueued (an e4b_path). */
+int32_t e4b_last_path(void);
+
+/* Host: number of kernels the most recent e4b_moe_forward call on this thread
+ * enqueued. */
+int32_t e4b_last_launch_count(void);
+
+/* Host: a static string naming the status. */
+const char* e4b_status_string(int32_t status);
+
+/* Host: library version, e.g. "e4b 0.1.0 sm_100a". */
+const char* e4b_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E4B_H_ */

@@ -1,0 +1,147 @@
+"""Oracle: the plain-C core (oracle_core.c) and the sampled full-size layer
+(test infrastructure only).
+
+The C functions restate the numpy definitions in ``formats`` as loops; the
+CPU tests check them against the numpy oracle bit for bit before they are
+used. ``moe_forward_sampled`` is ``moe.moe_forward_ref`` for a few tokens of
+a full-size layer: the same per-expert quantise -> decode -> fp64 matmul ->
+bf16(h) -> fp64 matmul -> weighted sum, with the heavy loops in C. It
+quantises from the fp32 weights itself; nothing comes from the CUDA library.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+from .formats import bf16_round, nf4_codebook
+from .moe import expert_tokens, swiglu_ref
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "oracle_core.c")
+LIB = os.path.join(_HERE, "_oracle_core.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """gcc -O2 without fast-math or FMA contraction (IEEE fp32/fp64 steps)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + ".tmp"
+        subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+                        "-o", tmp, SRC, "-lm"], check=True)
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def _core():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        vp, i64 = ctypes.c_void_p, ctypes.c_int64
+        L.e4bref_nf4_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.e4bref_nf4_decode.argtypes = [vp, vp, i64, i64, vp, vp]
+        L.e4bref_mxfp4_quantize.argtypes = [vp, i64, i64, vp, vp]
+        L.e4bref_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
+        L.e4bref_matvec_f64.argtypes = [vp, i64, i64, vp, i64, vp]
+        for f in ("e4bref_nf4_quantize", "e4bref_nf4_decode", "e4bref_mxfp4_quantize",
+                  "e4bref_mxfp4_decode", "e4bref_matvec_f64"):
+            getattr(L, f).restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags.c_contiguous
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def quantize(fmt: str, w: np.ndarray):
+    """fp32 [N, K] -> (codes, scales) in the layouts of formats.quantize_pack_*."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    if fmt == "nf4":
+        cb = nf4_codebook()
+        codes = np.empty((N, K // 2), np.uint8)
+        scales = np.empty((N, K // 64), np.float32)
+        _core().e4bref_nf4_quantize(_p(w), N, K, _p(cb), _p(codes), _p(scales))
+        return codes, scales
+    codes = np.empty((N, K // 32, 16), np.uint8)
+    scales = np.empty((N, K // 32), np.uint8)
+    _core().e4bref_mxfp4_quantize(_p(w), N, K, _p(codes), _p(scales))
+    return codes, scales
+
+
+def decode(fmt: str, codes, scales, N: int, K: int) -> np.ndarray:
+    """Parity-contract decode to fp32 [N, K] (bf16 values)."""
+    out = np.empty((N, K), np.float32)
+    codes = np.ascontiguousarray(codes)
+    scales = np.ascontiguousarray(scales)
+    if fmt == "nf4":
+        cb = nf4_codebook()
+        _core().e4bref_nf4_decode(_p(codes), _p(scales), N, K, _p(cb), _p(out))
+    else:
+        _core().e4bref_mxfp4_decode(_p(codes), _p(scales), N, K, _p(out))
+    return out
+
+
+def matvec(W: np.ndarray, X: np.ndarray) -> np.ndarray:
+    """fp64 X @ W^T for W fp32 [rows, K], X fp64 [n, K]."""
+    W = np.ascontiguousarray(W, np.float32)
+    X = np.ascontiguousarray(X, np.float64)
+    rows, K = W.shape
+    n = X.shape[0]
+    Y = np.empty((n, rows), np.float64)
+    _core().e4bref_matvec_f64(_p(W), rows, K, _p(X), n, _p(Y))
+    return Y
+
+
+def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None):
+    """One expert's contribution for the rows X (bf16 values, [n, H]):
+    decode gate_up -> fp64 matmul -> bf16(silu(gate) * up) -> decode down ->
+    fp64 matmul. Returns (O fp64 [n, len(cols)], h)."""
+    Wgu = decode(fmt, *packed_gu, 2 * I, H)
+    GU = matvec(Wgu, np.asarray(X, np.float64))
+    del Wgu
+    h = bf16_round(swiglu_ref(GU[:, :I], GU[:, I:]))
+    Wd = decode(fmt, *packed_dn, H, I)
+    if cols is not None:
+        Wd = np.ascontiguousarray(Wd[cols])
+    return matvec(Wd, h), h
+
+
+def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_rows=None,
+                        packed_fn=None):
+    """Outputs y[t, n] for the given tokens (and optionally only the given
+    output columns n) of the layer whose fp32 expert weights weight_fn(which,
+    e) returns ("gate_up" [2I, H], "down" [H, I]); with packed_fn(which, e)
+    given instead, the experts arrive already packed (codes, scales).
+
+    Returns (y fp64 holding bf16 values [len(tokens), len(cols)], cols,
+    packed) where packed[(which, e)] = (codes, scales) this function used.
+    """
+    x = np.asarray(x, np.float64)
+    ids = np.asarray(ids)
+    gates = np.asarray(gates, np.float32)
+    T, k = ids.shape
+    cols = np.arange(H) if down_rows is None else np.asarray(down_rows)
+    O_slot = {}
+    packed = {}
+    for e, pairs in sorted(expert_tokens(ids, tokens).items()):
+        for which in ("gate_up", "down"):
+            if packed_fn is not None:
+                packed[(which, e)] = packed_fn(which, e)
+            else:
+                packed[(which, e)] = quantize(fmt, weight_fn(which, e))
+        X = x[[t for _, t in pairs]]
+        O, _ = expert_term(fmt, X, packed[("gate_up", e)], packed[("down", e)], H, I,
+                           None if down_rows is None else cols)
+        for r, (slot, _) in enumerate(pairs):
+            O_slot[slot] = O[r]
+    y = np.zeros((len(tokens), len(cols)), np.float64)
+    for i, t in enumerate(tokens):
+        for j in range(k):
+            y[i] += np.float64(gates[t, j]) * O_slot[int(t) * k + j]
+    return bf16_round(y), cols, packed

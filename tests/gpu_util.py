@@ -1,0 +1,63 @@
+"""Helpers for the GPU parity tests: build packed layers on both sides and
+compare with the tolerance of the layer's fp outputs."""
+
+import numpy as np
+import torch
+
+import oracle
+from bit_grouped_moe_e4b_b200 import e4b
+
+# max |y - y_ref| <= TOL * (1 + |y_ref|), elementwise (fp32 accumulation on
+# the GPU, fp64 in the oracle, both with the same bf16 decode and bf16 h).
+TOL = 1e-2
+
+
+def scaled_err(y, y_ref) -> float:
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    return float(np.max(np.abs(y - y_ref) / (1.0 + np.abs(y_ref)))) if y.size else 0.0
+
+
+def assert_close(y, y_ref, what=""):
+    err = scaled_err(y, y_ref)
+    assert np.all(np.isfinite(y)), what
+    assert err <= TOL, f"{what}: max scaled error {err:.4g} > {TOL}"
+    return err
+
+
+def oracle_quantize(fmt, w: np.ndarray):
+    if fmt == "nf4":
+        return oracle.quantize_pack_nf4(w)
+    return oracle.quantize_pack_mxfp4(w)
+
+
+def small_layer(fmt, E, H, I, seed, std=0.02):
+    """Random layer quantised by the GPU and by the oracle; checks the codes
+    agree bit for bit. Returns (PackedLayer, oracle tuple (gc, gs, dc, ds))."""
+    rng = np.random.default_rng(seed)
+    wgu = (rng.standard_normal((E, 2 * I, H)) * std).astype(np.float32)
+    wd = (rng.standard_normal((E, H, I)) * std).astype(np.float32)
+    gc_d, gs_d = e4b.quantize(fmt, torch.from_numpy(wgu).cuda())
+    dc_d, ds_d = e4b.quantize(fmt, torch.from_numpy(wd).cuda())
+    gc, gs = oracle_quantize(fmt, wgu)
+    dc, ds = oracle_quantize(fmt, wd)
+    for got, want in ((gc_d, gc), (gs_d, gs), (dc_d, dc), (ds_d, ds)):
+        assert np.array_equal(got.cpu().numpy(), want)
+    layer = e4b.PackedLayer(fmt, E, H, I, gc_d, gs_d, dc_d, ds_d)
+    return layer, (gc, gs, dc, ds)
+
+
+def run_layer(layer, x_bf16: torch.Tensor, ids: np.ndarray, gates: np.ndarray, flags=0):
+    ids_d = torch.from_numpy(np.ascontiguousarray(ids, np.int32)).cuda()
+    g_d = torch.from_numpy(np.ascontiguousarray(gates, np.float32)).cuda()
+    x_d = x_bf16.cuda()
+    ws = e4b.workspace(layer, ids.shape[0], ids.shape[1])
+    y = e4b.moe_forward(layer, x_d, ids_d, g_d, ws=ws, flags=flags)
+    status = e4b.e4b_read_device_status(ws)
+    return y.float().cpu().numpy(), status, ws
+
+
+def oracle_layer(fmt, x_bf16: torch.Tensor, ids, gates, ref, E, H, I, tokens=None):
+    gc, gs, dc, ds = ref
+    return oracle.moe_forward_ref(fmt, x_bf16.float().numpy(), ids, gates, gc, gs, dc, ds, E, H, I,
+                                  tokens=tokens)

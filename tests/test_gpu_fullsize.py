@@ -1,0 +1,69 @@
+"""The five workloads at full size, in the launch configuration the bench
+times (path chosen from the shape), plus the other kernel path: sampled
+tokens checked against the oracle, which quantises the experts those tokens
+use from the same fp32 weights and compares its codes with the GPU's bit for
+bit."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import fast
+from bit_grouped_moe_e4b_b200 import e4b, synth
+from bit_grouped_moe_e4b_b200.configs import WORKLOADS
+from gpu_util import assert_close
+
+pytestmark = pytest.mark.gpu
+
+_layers = {}
+
+
+def _layer(wl):
+    if wl.layer not in _layers:
+        _layers.clear()
+        torch.cuda.empty_cache()
+        packed = []
+        for which in ("gate_up", "down"):
+            w = synth.layer_weights(wl, which, "cuda")
+            packed += list(e4b.quantize(wl.fmt, w))
+            del w
+        _layers[wl.layer] = e4b.PackedLayer(wl.fmt, wl.E, wl.H, wl.I, *packed)
+    return _layers[wl.layer]
+
+
+CASES = [(name, T) for name, wl in WORKLOADS.items() for T in wl.T]
+
+
+@pytest.mark.parametrize("name,T", CASES)
+def test_workload_sampled_tokens(name, T):
+    fast.build()
+    wl = WORKLOADS[name]
+    layer = _layer(wl)
+    x = synth.tokens_bf16(wl, T)
+    ids, gates = synth.routing(wl, T)
+    ids_d = torch.from_numpy(ids).cuda()
+    g_d = torch.from_numpy(gates).cuda()
+    x_d = x.cuda()
+    ws = e4b.workspace(layer, T, wl.top_k)
+    y_auto = e4b.moe_forward(layer, x_d, ids_d, g_d, ws=ws)
+    assert e4b.e4b_read_device_status(ws) == 0
+    auto_path = e4b.e4b_last_path()
+    other = e4b.FLAG_FORCE_TCGEN05 if auto_path == e4b.E4B_PATH_GEMV else e4b.FLAG_FORCE_GEMV
+    y_other = e4b.moe_forward(layer, x_d, ids_d, g_d, ws=ws, flags=other)
+    assert e4b.e4b_read_device_status(ws) == 0
+
+    tokens = sorted({0, T // 2, T - 1})
+    weight_fn = lambda which, e: synth.expert_weight(wl, which, e, "cuda").cpu().numpy()
+    y_ref, cols, packed = fast.moe_forward_sampled(wl.fmt, x.float().numpy(), ids, gates, weight_fn,
+                                                  wl.E, wl.H, wl.I, tokens)
+    for (which, e), (c, s) in packed.items():
+        gc = layer.gate_up_codes if which == "gate_up" else layer.down_codes
+        gs = layer.gate_up_scales if which == "gate_up" else layer.down_scales
+        assert np.array_equal(gc[e].cpu().numpy(), c), (which, e)
+        assert np.array_equal(gs[e].cpu().numpy().view(np.uint8), s.view(np.uint8)), (which, e)
+    for y, what in ((y_auto, "auto"), (y_other, "other path")):
+        got = y.float().cpu().numpy()[tokens]
+        assert_close(got, y_ref, f"{name} T={T} {what}")
+    # rows not sampled: finite and equal across the two kernel paths within tolerance
+    assert torch.isfinite(y_auto.float()).all()
+    assert_close(y_other.float().cpu().numpy(), y_auto.float().cpu().numpy(), f"{name} T={T} paths")

@@ -1,0 +1,145 @@
+"""The whole layer on the GPU against the oracle, at sizes the oracle finishes
+in seconds: several tiles with ragged tails, both kernel paths, both formats,
+and the degenerate routings."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_grouped_moe_e4b_b200 import e4b, synth
+from bit_grouped_moe_e4b_b200.configs import TINY
+from gpu_util import assert_close, oracle_layer, run_layer, small_layer
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"gemv": e4b.FLAG_FORCE_GEMV, "tcgen05": e4b.FLAG_FORCE_TCGEN05}
+
+
+def _x(T, H, seed):
+    rng = np.random.default_rng(seed)
+    return torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("path", ["auto", "gemv", "tcgen05"])
+def test_tiny_workload(path):
+    wl = TINY
+    T = wl.T[0]
+    wgu = synth.layer_weights(wl, "gate_up", "cuda")
+    wd = synth.layer_weights(wl, "down", "cuda")
+    gc_d, gs_d = e4b.quantize("nf4", wgu)
+    dc_d, ds_d = e4b.quantize("nf4", wd)
+    gc, gs = oracle.quantize_pack_nf4(wgu.cpu().numpy())
+    dc, ds = oracle.quantize_pack_nf4(wd.cpu().numpy())
+    assert np.array_equal(gc_d.cpu().numpy(), gc) and np.array_equal(gs_d.cpu().numpy(), gs)
+    assert np.array_equal(dc_d.cpu().numpy(), dc) and np.array_equal(ds_d.cpu().numpy(), ds)
+    layer = e4b.PackedLayer("nf4", wl.E, wl.H, wl.I, gc_d, gs_d, dc_d, ds_d)
+    x = synth.tokens_bf16(wl, T)
+    ids, gates = synth.routing(wl, T)
+    y, status, _ = run_layer(layer, x, ids, gates, 0 if path == "auto" else PATHS[path])
+    assert status == 0
+    y_ref = oracle_layer("nf4", x, ids, gates, (gc, gs, dc, ds), wl.E, wl.H, wl.I)
+    assert_close(y, y_ref, f"tiny workload, {path}")
+    if path != "auto":
+        assert e4b.e4b_last_path() == (e4b.E4B_PATH_GEMV if path == "gemv" else e4b.E4B_PATH_TCGEN05)
+    assert e4b.e4b_last_launch_count() == 4
+
+
+# shapes that span several tiles of both kernels and leave ragged tails:
+# tcgen05 tiles are 128 weight rows x 256 routed rows x 64 K; the small-M
+# kernel walks 16 rows x 256 K per warp step.
+SHAPES = [
+    ("nf4", 3, 256, 320, 300, 2),     # I tail (320 = 2.5 x 128), ~200 rows / expert
+    ("nf4", 5, 384, 192, 97, 3),      # odd T, k=3
+    ("mxfp4", 4, 96, 160, 70, 2),     # K % 64 == 32 on gate_up
+    ("mxfp4", 2, 224, 288, 600, 1),   # > 256 rows on an expert
+]
+
+
+@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("fmt,E,H,I,T,k", SHAPES)
+def test_ragged_shapes(fmt, E, H, I, T, k, path):
+    layer, ref = small_layer(fmt, E, H, I, seed=E * 100 + H)
+    x = _x(T, H, seed=T)
+    rng = np.random.default_rng(T + k)
+    ids, gates = synth.random_ids(rng, T, k, E)
+    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    assert status == 0
+    assert_close(y, oracle_layer(fmt, x, ids, gates, ref, E, H, I), f"{fmt} {E}x{H}x{I} T={T} {path}")
+
+
+EDGE = {
+    "single_slot": (1, 1, lambda T, k, E: np.zeros((1, 1), np.int32)),
+    "all_on_one_expert": (300, 2, lambda T, k, E: np.full((T, k), 3, np.int32)),
+    "duplicate_slots": (40, 2, lambda T, k, E: np.repeat(np.arange(T, dtype=np.int32)[:, None] % E, k, 1)),
+    "k_equals_E": (25, 4, lambda T, k, E: np.tile(np.arange(E, dtype=np.int32), (T, 1))),
+    "mostly_empty": (5, 1, lambda T, k, E: np.array([[1], [1], [2], [1], [2]], np.int32)),
+}
+
+
+@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("case", list(EDGE))
+def test_degenerate_routing(case, path):
+    E, H, I = 4, 128, 256
+    if case == "mostly_empty":
+        E = 16
+    T, k, make = EDGE[case]
+    layer, ref = small_layer("nf4", E, H, I, seed=7)
+    x = _x(T, H, seed=3)
+    ids = make(T, k, E)
+    gates = np.random.default_rng(1).random((T, k)).astype(np.float32)
+    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    assert status == 0
+    assert_close(y, oracle_layer("nf4", x, ids, gates, ref, E, H, I), f"{case} {path}")
+
+
+def test_bad_expert_ids_drop_only_their_slots():
+    E, H, I, T = 4, 128, 128, 6
+    layer, ref = small_layer("nf4", E, H, I, seed=11)
+    x = _x(T, H, seed=5)
+    ids = np.array([[0, 1], [9, 2], [3, -4], [1, 1], [2, 0], [3, 3]], np.int32)
+    gates = np.random.default_rng(2).random((T, 2)).astype(np.float32)
+    y, status, _ = run_layer(layer, x, ids, gates)
+    assert status == 6
+    g2 = gates.copy()
+    ids2 = ids.copy()
+    bad = (ids < 0) | (ids >= E)
+    g2[bad] = 0.0
+    ids2[bad] = 0
+    assert_close(y, oracle_layer("nf4", x, ids2, g2, ref, E, H, I), "bad ids")
+
+
+def test_bounded_wait_reports_timeout_and_returns():
+    E, H, I, T = 2, 128, 128, 40
+    layer, _ = small_layer("nf4", E, H, I, seed=12)
+    x = _x(T, H, seed=6)
+    ids = np.zeros((T, 1), np.int32)
+    gates = np.ones((T, 1), np.float32)
+    _, status, ws = run_layer(layer, x, ids, gates, e4b.FLAG_FORCE_TCGEN05 | e4b.FLAG_TEST_TIMEOUT)
+    assert status == 5
+    # the context is still usable: a normal call right after succeeds
+    y, status, _ = run_layer(layer, x, ids, gates, e4b.FLAG_FORCE_TCGEN05)
+    assert status == 0 and np.all(np.isfinite(y))
+
+
+def test_grouped_gemm_store_epilogue():
+    # the standalone projection entry point, plain bf16 output
+    fmt, E, N, K = "mxfp4", 3, 272, 320
+    rng = np.random.default_rng(3)
+    w = (rng.standard_normal((E, N, K)) * 0.05).astype(np.float32)
+    codes, scales = e4b.quantize(fmt, torch.from_numpy(w).cuda())
+    rc, rs = oracle.quantize_pack_mxfp4(w)
+    counts = np.array([5, 0, 300])
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    R = int(offsets[-1])
+    a = torch.from_numpy(rng.standard_normal((R, K)).astype(np.float32)).to(torch.bfloat16)
+    wdec = oracle.dequant_mxfp4(rc, rs).astype(np.float64)
+    want = np.concatenate([a[offsets[e]:offsets[e + 1]].double().numpy() @ wdec[e].T for e in range(E)])
+    want = oracle.bf16_round(want)
+    for flags in (e4b.FLAG_FORCE_GEMV, e4b.FLAG_FORCE_TCGEN05):
+        out = torch.empty((R, N), dtype=torch.bfloat16, device="cuda")
+        e4b.e4b_grouped_gemm(fmt, e4b.E4B_EPI_STORE, codes, scales, a.cuda(),
+                             torch.from_numpy(offsets).cuda(), out, E=E, N=N, K=K, R_max=R,
+                             flags=flags)
+        torch.cuda.synchronize()
+        assert_close(out.float().cpu().numpy(), want, f"store flags={flags}")

@@ -1,0 +1,90 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/e4b.h declares, and rejects bad arguments on the host before any
+launch."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+from golden_io import read_floats
+from bit_grouped_moe_e4b_b200 import e4b
+
+HEADER = os.path.join(ROOT, "include", "e4b.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(e4b_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = e4b.lib()
+    names = declared_symbols()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(e4b.EXPORTED) == names
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in e4b.e4b_version()
+    assert e4b.e4b_status_string(0) == "ok"
+    assert "expert id" in e4b.e4b_status_string(6)
+
+
+def test_library_codebook_is_the_published_table():
+    pub = np.array(read_floats("nf4_codebook_qlora.txt"), dtype=np.float32)
+    assert np.array_equal(e4b.e4b_nf4_codebook().view(np.uint32), pub.view(np.uint32))
+
+
+def _w(fmt=0, E=8, H=256, I=512, ptr=4096):
+    return e4b.MoeWeights(fmt, E, H, I, ptr, ptr, ptr, ptr)
+
+
+def test_host_argument_checks_return_before_launch():
+    L = e4b.lib()
+    n = ctypes.c_size_t(0)
+    w = _w()
+    assert L.e4b_moe_workspace_size(ctypes.byref(w), 64, 2, ctypes.byref(n)) == 0
+    need = n.value
+    assert need > 64 * 2 * 512 * 2  # holds at least h
+    fwd = L.e4b_moe_forward
+    p = ctypes.c_void_p(4096)
+    # T == 0 is a no-op
+    assert fwd(ctypes.byref(w), None, 0, 2, None, None, None, None, 0, 0, None) == 0
+    # null pointers
+    assert fwd(ctypes.byref(w), None, 4, 2, p, p, p, p, need, 0, None) == 1
+    # top_k > E
+    assert fwd(ctypes.byref(_w(E=2)), p, 4, 3, p, p, p, p, need, 0, None) == 1
+    # unsupported shapes: NF4 needs H, I multiples of 64
+    assert fwd(ctypes.byref(_w(H=96)), p, 4, 2, p, p, p, p, need, 0, None) == 2
+    # misaligned
+    assert fwd(ctypes.byref(w), ctypes.c_void_p(4098), 4, 2, p, p, p, p, need, 0, None) == 7
+    # workspace too small
+    assert fwd(ctypes.byref(w), p, 64, 2, p, p, p, p, need - 1, 0, None) == 3
+    # bad format
+    assert fwd(ctypes.byref(_w(fmt=5)), p, 4, 2, p, p, p, p, need, 0, None) == 1
+    # (every call above and below fails validation, so nothing is launched
+    # even when a GPU is present: the pointers are not real allocations)
+    # quantiser checks
+    assert L.e4b_quantize_nf4(p, 1, 4, 96, 64, p, p, None) == 2
+    assert L.e4b_quantize_nf4(p, 1, 4, 128, 32, p, p, None) == 2
+    assert L.e4b_quantize_nf4(None, 1, 4, 128, 64, p, p, None) == 1
+    assert L.e4b_quantize_mxfp4(p, 1, 4, 48, p, p, None) == 2
+    # routing checks
+    assert L.e4b_route(p, 4, 2, 2000, p, p, p, p, p, 256, None) == 2
+    assert L.e4b_route(p, 4, 2, 8, p, p, p, p, p, 16, None) == 3
+    ga = e4b.GemmArgs(0, 5, 8, 1, 256, 256, 64, 4096, 4096, 4096, 256, None, None, 4096, None, 4096, 256)
+    assert L.e4b_grouped_gemm(ctypes.byref(ga), 0, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        e4b.e4b_quantize_nf4(torch.zeros(1, 4, 64), torch.zeros(1, 4, 32, dtype=torch.uint8),
+                             torch.zeros(1, 4, 1))
