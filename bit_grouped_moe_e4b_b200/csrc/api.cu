@@ -100,6 +100,7 @@ const char* e4b_status_string(int32_t s) {
     case E4B_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case E4B_ERR_BAD_EXPERT_ID: return "expert id out of range";
     case E4B_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case E4B_ERR_EXCEEDS_STATIC_SCRATCH: return "needs more than the 16 MiB static scratch";
     default: return "unknown status";
   }
 }

@@ -28,7 +28,7 @@ FLAG_TEST_TIMEOUT = 0x4
 STATUS_NAMES = {
     0: "E4B_OK", 1: "E4B_ERR_INVALID_ARG", 2: "E4B_ERR_UNSUPPORTED",
     3: "E4B_ERR_WORKSPACE_TOO_SMALL", 4: "E4B_ERR_CUDA", 5: "E4B_ERR_DEVICE_TIMEOUT",
-    6: "E4B_ERR_BAD_EXPERT_ID", 7: "E4B_ERR_MISALIGNED",
+    6: "E4B_ERR_BAD_EXPERT_ID", 7: "E4B_ERR_MISALIGNED", 8: "E4B_ERR_EXCEEDS_STATIC_SCRATCH",
 }
 FMT = {"nf4": E4B_FMT_NF4, "mxfp4": E4B_FMT_MXFP4}
 
@@ -36,7 +36,7 @@ FMT = {"nf4": E4B_FMT_NF4, "mxfp4": E4B_FMT_MXFP4}
 EXPORTED = [
     "e4b_quantize_nf4", "e4b_quantize_mxfp4", "e4b_dequantize", "e4b_nf4_codebook",
     "e4b_route_workspace_size", "e4b_route", "e4b_grouped_gemm", "e4b_moe_workspace_size",
-    "e4b_moe_forward", "e4b_read_device_status", "e4b_set_timing_events", "e4b_last_path",
+    "e4b_moe_forward", "e4b_moe_forward_noalloc", "e4b_read_device_status", "e4b_set_timing_events", "e4b_last_path",
     "e4b_last_launch_count",
     "e4b_status_string", "e4b_version",
 ]
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         "e4b_moe_workspace_size": [ctypes.POINTER(MoeWeights), i64, i32, ctypes.POINTER(sz)],
         "e4b_moe_forward": [ctypes.POINTER(MoeWeights), vp, i64, i32, vp, vp, vp, vp, sz,
                             ctypes.c_uint32, vp],
+        "e4b_moe_forward_noalloc": [ctypes.POINTER(MoeWeights), vp, i64, i32, vp, vp, vp,
+                                    ctypes.c_uint32, vp],
         "e4b_read_device_status": [vp, ctypes.POINTER(i32), vp],
         "e4b_set_timing_events": [ctypes.POINTER(vp), i32],
         "e4b_last_path": [],
@@ -255,6 +257,17 @@ def e4b_moe_forward(layer: PackedLayer, x, ids, gates, y, ws, flags=0, stream=No
     _check(lib().e4b_moe_forward(ctypes.byref(w), _ptr(x), T, k, _ptr(ids), _ptr(gates), _ptr(y),
                                  _ptr(ws), ws.numel() * ws.element_size(), flags, _stream(stream)),
            "e4b_moe_forward")
+
+
+def e4b_moe_forward_noalloc(layer: PackedLayer, x, ids, gates, y, flags=0, stream=None):
+    """The layer forward with the library's static scratch instead of a
+    workspace, for callers that cannot allocate device memory (see e4b.h)."""
+    _dev(x, ids, gates, y)
+    T, k = ids.shape
+    w = layer.c_struct()
+    _check(lib().e4b_moe_forward_noalloc(ctypes.byref(w), _ptr(x), T, k, _ptr(ids), _ptr(gates),
+                                         _ptr(y), flags, _stream(stream)),
+           "e4b_moe_forward_noalloc")
 
 
 def e4b_read_device_status(ws, stream=None) -> int:

@@ -57,7 +57,9 @@ typedef enum {
   E4B_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
   E4B_ERR_DEVICE_TIMEOUT = 5,      /* (device) a bounded wait gave up */
   E4B_ERR_BAD_EXPERT_ID = 6,       /* (device) an id outside [0, E); the slot is dropped */
-  E4B_ERR_MISALIGNED = 7           /* a pointer or row stride breaks 16-byte alignment */
+  E4B_ERR_MISALIGNED = 7,          /* a pointer or row stride breaks 16-byte alignment */
+  E4B_ERR_EXCEEDS_STATIC_SCRATCH = 8 /* e4b_moe_forward_noalloc: the call needs more than its
+                                        16 MiB static scratch */
 } e4b_status;
 
 typedef enum { E4B_FMT_NF4 = 0, E4B_FMT_MXFP4 = 1 } e4b_format;
@@ -231,6 +233,39 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
 e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
                            const int32_t* ids, const float* gates, uint16_t* y, void* ws,
                            size_t ws_bytes, uint32_t flags, void* stream);
+
+/*
+ * e4b_moe_forward_noalloc -- the layer forward of e4b_moe_forward for callers
+ * that cannot allocate device memory. The pages describe no such entry
+ * point; it exists for callers that get no allocator: code running while a
+ * stream is being captured into a CUDA graph under a framework that forbids
+ * allocation there, runtimes that hand every byte of HBM to their own pool,
+ * and host plug-in interfaces that pass only input and output buffers. A
+ * cudaMalloc in such a place either fails, synchronises the device, or takes
+ * memory its owner did not budget for.
+ *
+ * Same arguments and results as e4b_moe_forward, without ws / ws_bytes: the
+ * scratch (routing arrays, bf16 intermediate, fp32 accumulator, status word)
+ * lives in a 16 MiB array in the library's device memory, which every GPU
+ * that loads the library keeps until the process exits. A call whose
+ * scratch, as e4b_moe_workspace_size reports it, exceeds 16 MiB returns
+ * E4B_ERR_EXCEEDS_STATIC_SCRATCH and enqueues nothing (a layer with H=4096,
+ * I=14336 and top-2 routing fits up to 227 tokens). Nothing is allocated or
+ * freed.
+ *   - The first call on each device looks up that device's copy of the
+ *     array (set-up, once per device); make that first call before any stream
+ *     capture begins.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; each call re-clears what must start at zero. Calls whose GPU
+ *     work overlaps (different streams, or graphs replayed concurrently) race
+ *     on the array: order them on one stream.
+ *   - The device status word is inside the array and is not readable with
+ *     e4b_read_device_status; use e4b_moe_forward with a workspace when the
+ *     status is needed.
+ */
+e4b_status e4b_moe_forward_noalloc(const e4b_moe_weights* w, const uint16_t* x, int64_t T,
+                                   int32_t top_k, const int32_t* ids, const float* gates,
+                                   uint16_t* y, uint32_t flags, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word that
  * e4b_route / e4b_moe_forward keep at the start of ws. *status_host receives
