@@ -68,7 +68,7 @@ E4B_DEV void load_row_chunk(RowChunk& rc, const uint8_t* crow, const uint8_t* sr
 }
 
 template <int FMT, int EPI>
-__global__ void __launch_bounds__(kGemvWarps * 32)
+__global__ void __launch_bounds__(kGemvWarps * 32, 2)
 gemv_kernel(GemmProblem p) {
   __shared__ int32_t s_act[kMaxExpertsSmem];
   __shared__ int32_t s_nact;
@@ -142,14 +142,18 @@ gemv_kernel(GemmProblem p) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) load_row_chunk<FMT>(rc[m][h], crow[m][h], srow[m][h], kl, K);
         const bool kvalid = kl < K;
+        Lut L[NM][2];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          Lut L[NM][2];
+          // one NF4 block (64 weights) per row and lane: its table serves both
+          // halves; MXFP4 has a block (and table) per half
+          if (FMT == E4B_FMT_MXFP4 || half == 0) {
 #pragma unroll
-          for (int m = 0; m < NM; ++m)
+            for (int m = 0; m < NM; ++m)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-              lut_build<FMT>(L[m][h], rc[m][h].absmax, (rc[m][h].mx >> (8 * half)) & 0xFFu);
+              for (int h = 0; h < 2; ++h)
+                lut_build<FMT>(L[m][h], rc[m][h].absmax, (rc[m][h].mx >> (8 * half)) & 0xFFu);
+          }
 #pragma unroll
           for (int ss = 0; ss < 8; ++ss) {
             const int s = half * 8 + ss;  // MMA k-step within the chunk
