@@ -36,7 +36,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace of the layer forward.
 struct MoeWs {
-  size_t status, counts, offsets, perm, inv, h, acc, total;
+  size_t status, sync, nsync, counts, offsets, perm, inv, h, acc, total;
 };
 
 MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
@@ -44,6 +44,8 @@ MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
   const int64_t R = T * top_k;
   size_t o = 0;
   w.status = o;  o += kStatusBytes;
+  w.nsync = smallm_sync_ints(int(E), int(H));
+  w.sync = o;    o = align_up(o + w.nsync * 4, 256);
   w.counts = o;  o = align_up(o + size_t(E) * 4, 256);
   w.offsets = o; o = align_up(o + size_t(E + 1) * 8, 256);
   w.perm = o;    o = align_up(o + size_t(R) * 4, 256);
@@ -265,9 +267,44 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   mark(0, s);
+  int32_t* sync = reinterpret_cast<int32_t*>(base + L.sync);
   cudaError_t ce = launch_route(ids, int32_t(R), int32_t(E), counts, offsets, perm, inv, nullptr,
-                                status, s);
+                                status, s, sync, int32_t(L.nsync));
   if (ce != cudaSuccess) return E4B_ERR_CUDA;
+
+  if (gemv) {
+    // small-M: both projections, SwiGLU, combine and bf16 output in one launch
+    SmallMLayer sl{};
+    sl.fmt = w->fmt;
+    sl.E = int(E);
+    sl.H = int(H);
+    sl.I = int(I);
+    sl.top_k = top_k;
+    sl.T = T;
+    sl.gu_codes = w->gate_up_codes;
+    sl.gu_scales = w->gate_up_scales;
+    sl.dn_codes = w->down_codes;
+    sl.dn_scales = w->down_scales;
+    sl.x = x;
+    sl.perm = perm;
+    sl.offsets = offsets;
+    sl.gates = gates;
+    sl.h = h;
+    sl.acc = acc;
+    sl.y = y;
+    sl.sync = sync;
+    sl.status = status;
+    sl.flags = flags;
+    mark(1, s);
+    mark(2, s);
+    ce = launch_smallm_layer(sl, s, sm_count());
+    if (ce != cudaSuccess) return E4B_ERR_CUDA;
+    mark(3, s);
+    mark(4, s);
+    g_last_path = E4B_PATH_GEMV;
+    g_last_launches = 2;
+    return E4B_OK;
+  }
 
   GemmProblem g{};
   g.fmt = w->fmt;

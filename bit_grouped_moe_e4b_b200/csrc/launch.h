@@ -20,7 +20,7 @@ void host_nf4_levels(float* out);
 size_t route_smem_bytes(int32_t E);
 cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* counts, int64_t* offsets,
                          int32_t* perm, int32_t* inv, int32_t* active, int32_t* status,
-                         cudaStream_t st);
+                         cudaStream_t st, int32_t* clear = nullptr, int32_t nclear = 0);
 
 // Description of one grouped projection as the kernels see it.
 struct GemmProblem {
@@ -47,6 +47,28 @@ struct GemmProblem {
 };
 
 cudaError_t launch_gemv(const GemmProblem& p, cudaStream_t st, int sms);
+
+// The whole small-M layer in one persistent launch (csrc/smallm.cu).
+struct SmallMLayer {
+  int fmt, E, H, I, top_k;
+  int64_t T;
+  const uint8_t* gu_codes;
+  const void* gu_scales;
+  const uint8_t* dn_codes;
+  const void* dn_scales;
+  const uint16_t* x;
+  const int32_t* perm;
+  const int64_t* offsets;
+  const float* gates;
+  uint16_t* h;
+  float* acc;
+  uint16_t* y;
+  int32_t* sync;   // smallm_sync_ints(E, H) ints, zero on entry
+  int32_t* status;
+  uint32_t flags;
+};
+size_t smallm_sync_ints(int E, int H);
+cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms);
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms);
 cudaError_t launch_finalize(const float* acc, int64_t n, uint16_t* y, cudaStream_t st, int sms);
 

@@ -21,7 +21,8 @@ constexpr int kRouteWarps = kRouteThreads / 32;
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __restrict__ counts,
              int64_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-             int32_t* __restrict__ active, int32_t* __restrict__ status) {
+             int32_t* __restrict__ active, int32_t* __restrict__ status, int32_t* __restrict__ clear,
+             int32_t nclear) {
   extern __shared__ int32_t smem[];
   int32_t* wcnt = smem;                        // [kRouteWarps][E] counts, then bases
   int32_t* scan = smem + kRouteWarps * E;      // [kRouteThreads] scan scratch
@@ -30,6 +31,8 @@ route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __r
   const int lane = tid & 31;
   const int warp = tid >> 5;
   for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) wcnt[i] = 0;
+  // counters the following layer kernels expect at zero
+  for (int i = tid; i < nclear; i += kRouteThreads) clear[i] = 0;
   if (tid == 0) {
     s_bad = 0;
     // The status word describes the most recent call: route runs first.
@@ -131,16 +134,19 @@ size_t route_smem_bytes(int32_t E) { return size_t(kRouteWarps) * E * 4 + kRoute
 
 cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* counts, int64_t* offsets,
                          int32_t* perm, int32_t* inv, int32_t* active, int32_t* status,
-                         cudaStream_t st) {
+                         cudaStream_t st, int32_t* clear, int32_t nclear) {
   const size_t smem = route_smem_bytes(E);
-  static bool configured = false;  // the attribute is per function, set once
-  if (!configured) {
+  static int configured = -1;  // the attribute is per device context
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
     cudaError_t err = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            int(route_smem_bytes(1024)));
     if (err != cudaSuccess) return err;
-    configured = true;
+    configured = dev;
   }
-  route_kernel<<<1, kRouteThreads, smem, st>>>(ids, R, E, counts, offsets, perm, inv, active, status);
+  route_kernel<<<1, kRouteThreads, smem, st>>>(ids, R, E, counts, offsets, perm, inv, active, status,
+                                                clear, nclear);
   return cudaGetLastError();
 }
 

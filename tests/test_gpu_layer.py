@@ -42,7 +42,8 @@ def test_tiny_workload(path):
     assert_close(y, y_ref, f"tiny workload, {path}")
     if path != "auto":
         assert e4b.e4b_last_path() == (e4b.E4B_PATH_GEMV if path == "gemv" else e4b.E4B_PATH_TCGEN05)
-    assert e4b.e4b_last_launch_count() == 4
+    # small-M: routing + one fused layer kernel; tcgen05: routing, two GEMMs, conversion
+    assert e4b.e4b_last_launch_count() == (2 if e4b.e4b_last_path() == e4b.E4B_PATH_GEMV else 4)
 
 
 # shapes that span several tiles of both kernels and leave ragged tails:
@@ -109,17 +110,21 @@ def test_bad_expert_ids_drop_only_their_slots():
     assert_close(y, oracle_layer("nf4", x, ids2, g2, ref, E, H, I), "bad ids")
 
 
-def test_bounded_wait_reports_timeout_and_returns():
+@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+def test_bounded_wait_reports_timeout_and_returns(path):
+    # the test flag makes the kernels' bounded waits give up at once: the
+    # kernel must record E4B_ERR_DEVICE_TIMEOUT and return (no hang, no trap)
     E, H, I, T = 2, 128, 128, 40
-    layer, _ = small_layer("nf4", E, H, I, seed=12)
+    layer, ref = small_layer("nf4", E, H, I, seed=12)
     x = _x(T, H, seed=6)
     ids = np.zeros((T, 1), np.int32)
     gates = np.ones((T, 1), np.float32)
-    _, status, ws = run_layer(layer, x, ids, gates, e4b.FLAG_FORCE_TCGEN05 | e4b.FLAG_TEST_TIMEOUT)
+    _, status, ws = run_layer(layer, x, ids, gates, PATHS[path] | e4b.FLAG_TEST_TIMEOUT)
     assert status == 5
     # the context is still usable: a normal call right after succeeds
-    y, status, _ = run_layer(layer, x, ids, gates, e4b.FLAG_FORCE_TCGEN05)
-    assert status == 0 and np.all(np.isfinite(y))
+    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    assert status == 0
+    assert_close(y, oracle_layer("nf4", x, ids, gates, ref, E, H, I), f"after timeout {path}")
 
 
 def test_grouped_gemm_store_epilogue():
