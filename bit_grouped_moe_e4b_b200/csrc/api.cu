@@ -77,7 +77,7 @@ bool choose_gemv(int64_t R, int64_t E, uint32_t flags) {
   if (flags & E4B_FLAG_FORCE_GEMV) return true;
   if (flags & E4B_FLAG_FORCE_TCGEN05) return false;
   if (E > 256) return true;
-  return R <= 32 * E;
+  return R <= 16 * E;
 }
 
 e4b_status run_projection(const GemmProblem& p, bool gemv, cudaStream_t st) {

@@ -32,6 +32,8 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kChunk = 256;              // K per step of a warp
 constexpr int kSlotBytesPerLane = 128;   // 2 rows x (2 matrices) x 32 B
 constexpr int kSlots = 2;
+constexpr int kMaxNT = 2;                // token chunks of 8 per pass (16 rows)
+constexpr int kGroup = 8 * kMaxNT;
 constexpr uint32_t kPolls = 1u << 24;
 
 // sync words (int32) at the start of the layer's sync area:
@@ -127,111 +129,124 @@ E4B_DEV uint32_t load_scale(const uint8_t* srow, int kl, int K) {
   }
 }
 
-// One warp-item over the K range [k0, k1) for NM weight matrices (row
-// pointers crow/srow per matrix and row half) and up to 4 chunks of 8 token
-// rows (brow: activation row of this lane's token in each chunk, or null).
-// Accumulates into acc[m][j][4].
-template <int FMT, int NM, bool COHERENT_B>
-E4B_DEV void run_item(const uint8_t* const (&crow)[NM][2], const uint8_t* const (&srow)[NM][2],
-                      const uint16_t* const (&brow)[4], int nt, int k0, int k1, int K,
-                      uint32_t slot_base, float (&acc)[NM][4][4]) {
+// One warp-item over the K range [k0, k1) of one weight matrix (row
+// pointers crow/srow for rows g and g+8 of the 16-row tile) and NT chunks of
+// 8 token rows (brow: activation row of this lane's token in each chunk, or
+// null). Accumulates into acc[j][4].
+template <int FMT, int NT, bool COHERENT_B>
+E4B_DEV void run_item(const uint8_t* const (&crow)[2], const uint8_t* const (&srow)[2],
+                      const uint16_t* const (&brow)[kMaxNT], int k0, int k1, int K, uint32_t slot_base,
+                      float (&acc)[kMaxNT][4]) {
   const int lane = threadIdx.x & 31;
   const int c = lane & 3;
+  const int kend = min(K, k1);
   const int nchunks = (k1 - k0 + kChunk - 1) / kChunk;
 
   auto issue = [&](int ci, int slot) {
     const int kl = k0 + ci * kChunk + c * 64;
-    const int left = min(K, k1) - kl;  // weights this lane may copy
+    const int left = kend - kl;  // weights this lane may copy
 #pragma unroll
-    for (int m = 0; m < NM; ++m)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int piece = 0; piece < 2; ++piece) {
-          const uint32_t dst = slot_base + uint32_t(slot * kSlotBytesPerLane * 32) +
-                               uint32_t(((m * 2 + h) * 2 + piece) * 512 + lane * 16);
-          const bool ok = left >= 32 * (piece + 1);
-          cp16(dst, ok ? (const void*)(crow[m][h] + (kl >> 1) + piece * 16) : (const void*)crow[m][h],
-               ok ? 16u : 0u);
-        }
+      for (int piece = 0; piece < 2; ++piece) {
+        const uint32_t dst = slot_base + uint32_t(slot * kSlotBytesPerLane * 32) +
+                             uint32_t((h * 2 + piece) * 512 + lane * 16);
+        const bool ok = left >= 32 * (piece + 1);
+        cp16(dst, ok ? (const void*)(crow[h] + (kl >> 1) + piece * 16) : (const void*)crow[h],
+             ok ? 16u : 0u);
+      }
     cp_commit();
   };
+  auto load_b = [&](int koff, uint4 (&b)[NT]) {
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      b[j] = make_uint4(0, 0, 0, 0);
+      if (brow[j] && koff < kend) {
+        if constexpr (COHERENT_B) b[j] = ld_cg_v4(brow[j] + koff);
+        else b[j] = __ldg(reinterpret_cast<const uint4*>(brow[j] + koff));
+      }
+    }
+  };
+
+  // two accumulator sets (the two MMA sub-steps of a word) shorten the
+  // dependency chains through the tensor pipe
+  float acc2[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc2[j][q] = 0.f;
 
   issue(0, 0);
-  uint32_t sc_next[NM][2];
-#pragma unroll
-  for (int m = 0; m < NM; ++m)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) sc_next[m][h] = load_scale<FMT>(srow[m][h], k0 + c * 64, min(K, k1));
+  uint32_t sc_next0 = load_scale<FMT>(srow[0], k0 + c * 64, kend);
+  uint32_t sc_next1 = load_scale<FMT>(srow[1], k0 + c * 64, kend);
+  uint4 bcur[NT];
+  load_b(k0 + c * 64, bcur);
 
   for (int ci = 0; ci < nchunks; ++ci) {
     const int slot = ci & 1;
     const int kl = k0 + ci * kChunk + c * 64;
-    const bool full = (k0 + (ci + 1) * kChunk) <= min(K, k1);
-    uint32_t sc[NM][2];
-#pragma unroll
-    for (int m = 0; m < NM; ++m)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) sc[m][h] = sc_next[m][h];
+    const uint32_t sc0 = sc_next0, sc1 = sc_next1;
     if (ci + 1 < nchunks) {
       issue(ci + 1, slot ^ 1);
-#pragma unroll
-      for (int m = 0; m < NM; ++m)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          sc_next[m][h] = load_scale<FMT>(srow[m][h], kl + kChunk, min(K, k1));
+      sc_next0 = load_scale<FMT>(srow[0], kl + kChunk, kend);
+      sc_next1 = load_scale<FMT>(srow[1], kl + kChunk, kend);
       cp_wait1();
     } else {
       cp_wait0();
     }
     const uint32_t sbase = slot_base + uint32_t(slot * kSlotBytesPerLane * 32) + uint32_t(lane * 16);
-
+    Lut L0, L1;
+    if constexpr (FMT == E4B_FMT_NF4) {  // one 64-weight block per row and lane
+      lut_nf4(L0, __uint_as_float(sc0));
+      lut_nf4(L1, __uint_as_float(sc1));
+    }
 #pragma unroll
-    for (int m = 0; m < NM; ++m) {
+    for (int half = 0; half < 2; ++half) {
+      const uint4 w0 = lds128(sbase + uint32_t((0 * 2 + half) * 512));
+      const uint4 w1 = lds128(sbase + uint32_t((1 * 2 + half) * 512));
+      if constexpr (FMT == E4B_FMT_MXFP4) {  // one 32-weight block per half
+        lut_mxfp4(L0, (sc0 >> (8 * half)) & 0xFFu);
+        lut_mxfp4(L1, (sc1 >> (8 * half)) & 0xFFu);
+      }
+      const uint32_t r0w[4] = {w0.x, w0.y, w0.z, w0.w};
+      const uint32_t r1w[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // 4 words (32 weights) of each row half
-        const uint4 w0 = lds128(sbase + uint32_t(((m * 2 + 0) * 2 + half) * 512));
-        const uint4 w1 = lds128(sbase + uint32_t(((m * 2 + 1) * 2 + half) * 512));
-        Lut L0, L1;
-        if constexpr (FMT == E4B_FMT_NF4) {
-          lut_nf4(L0, __uint_as_float(sc[m][0]));
-          lut_nf4(L1, __uint_as_float(sc[m][1]));
-        } else {
-          lut_mxfp4(L0, (sc[m][0] >> (8 * half)) & 0xFFu);
-          lut_mxfp4(L1, (sc[m][1] >> (8 * half)) & 0xFFu);
+      for (int wi = 0; wi < 4; ++wi) {
+        // prefetch the next word's activations (next chunk's first word at the end)
+        uint4 bnext[NT];
+        const int knext = (half == 1 && wi == 3) ? kl + kChunk : kl + half * 32 + wi * 8 + 8;
+        const bool more = !(half == 1 && wi == 3) || (ci + 1 < nchunks);
+        if (more) load_b(knext, bnext);
+        uint32_t o0[4], o1[4];
+        lut_decode8<FMT>(L0, r0w[wi], o0);
+        lut_decode8<FMT>(L1, r1w[wi], o1);
+        // sub-step 0: weights 0..3 of the word, sub-step 1: weights 4..7;
+        // fragment registers {row g | row g+8} x {cols 2c,2c+1 | 2c+8,2c+9}
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          mma16816(acc[j], o0[0], o1[0], o0[1], o1[1], bcur[j].x, bcur[j].y);
+          mma16816(acc2[j], o0[2], o1[2], o0[3], o1[3], bcur[j].z, bcur[j].w);
         }
-        const uint32_t r0w[4] = {w0.x, w0.y, w0.z, w0.w};
-        const uint32_t r1w[4] = {w1.x, w1.y, w1.z, w1.w};
+        if (more) {
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-          uint32_t a[2][4];  // [sub-step][a0a1, a2a3, a4a5, a6a7]
-          {
-            uint32_t o0[4], o1[4];
-            lut_decode8<FMT>(L0, r0w[wi], o0);
-            lut_decode8<FMT>(L1, r1w[wi], o1);
-            // sub-step 0: weights 0..3 of the word; sub-step 1: 4..7
-            a[0][0] = o0[0]; a[0][1] = o1[0]; a[0][2] = o0[1]; a[0][3] = o1[1];
-            a[1][0] = o0[2]; a[1][1] = o1[2]; a[1][2] = o0[3]; a[1][3] = o1[3];
-          }
-          // activation fragments: 8 consecutive bf16 of this lane's token row
-          const int koff = kl + half * 32 + wi * 8;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j < nt) {
-              uint4 b = make_uint4(0, 0, 0, 0);
-              if (brow[j] && (full || koff < K)) {
-                if constexpr (COHERENT_B) b = ld_cg_v4(brow[j] + koff);
-                else b = __ldg(reinterpret_cast<const uint4*>(brow[j] + koff));
-              }
-              mma16816(acc[m][j], a[0][0], a[0][1], a[0][2], a[0][3], b.x, b.y);
-              mma16816(acc[m][j], a[1][0], a[1][1], a[1][2], a[1][3], b.z, b.w);
-            }
-          }
+          for (int j = 0; j < NT; ++j) bcur[j] = bnext[j];
         }
       }
     }
   }
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[j][q] += acc2[j][q];
+}
+
+// run_item with the token-chunk count as a compile-time constant
+template <int FMT, bool COHERENT_B>
+E4B_DEV void run_item_nt(int nt, const uint8_t* const (&crow)[2], const uint8_t* const (&srow)[2],
+                         const uint16_t* const (&brow)[kMaxNT], int k0, int k1, int K, uint32_t slot_base,
+                         float (&acc)[kMaxNT][4]) {
+  if (nt == 1) run_item<FMT, 1, COHERENT_B>(crow, srow, brow, k0, k1, K, slot_base, acc);
+  else run_item<FMT, 2, COHERENT_B>(crow, srow, brow, k0, k1, K, slot_base, acc);
 }
 
 template <int FMT>
@@ -295,46 +310,46 @@ __global__ void __launch_bounds__(kThreads, 2) smallm_layer_kernel(Params p) {
       const int mt = item % MTA;
       const int e = s_act[ai];
       const int64_t p0 = p.offsets[e], p1 = p.offsets[e + 1];
-      const uint8_t* crow[1][2];
-      const uint8_t* srow[1][2];
+      const uint8_t* crow[2];
+      const uint8_t* srow[2];
       const int64_t sstride = FMT == E4B_FMT_NF4 ? (H / 64) * 4 : (H / 32);
-      for (int64_t tg = p0; tg < p1; tg += 32) {
-        const int nt = int((min(p1 - tg, int64_t(32)) + 7) / 8);
-        const uint16_t* brow[4];
+      for (int64_t tg = p0; tg < p1; tg += kGroup) {
+        const int nt = int((min(p1 - tg, int64_t(kGroup)) + 7) / 8);
+        const uint16_t* brow[kMaxNT];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kMaxNT; ++j) {
           const int64_t pr = tg + 8 * j + g;
           brow[j] = (j < nt && pr < p1) ? p.x + int64_t(p.perm[pr] / p.top_k) * H : nullptr;
         }
-        float accg[1][4][4], accu[1][4][4];
+        float accg[kMaxNT][4], accu[kMaxNT][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < kMaxNT; ++j)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) accg[0][j][q] = accu[0][j][q] = 0.f;
+          for (int q = 0; q < 4; ++q) accg[j][q] = accu[j][q] = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int64_t row = int64_t(e) * 2 * I + mt * 16 + g + 8 * hh;
-          crow[0][hh] = p.gu_codes + row * (H / 2);
-          srow[0][hh] = p.gu_scales + row * sstride;
+          crow[hh] = p.gu_codes + row * (H / 2);
+          srow[hh] = p.gu_scales + row * sstride;
         }
-        run_item<FMT, 1, false>(crow, srow, brow, nt, 0, H, H, slot_base, accg);
+        run_item_nt<FMT, false>(nt, crow, srow, brow, 0, H, H, slot_base, accg);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int64_t row = int64_t(e) * 2 * I + I + mt * 16 + g + 8 * hh;
-          crow[0][hh] = p.gu_codes + row * (H / 2);
-          srow[0][hh] = p.gu_scales + row * sstride;
+          crow[hh] = p.gu_codes + row * (H / 2);
+          srow[hh] = p.gu_scales + row * sstride;
         }
-        run_item<FMT, 1, false>(crow, srow, brow, nt, 0, H, H, slot_base, accu);
+        run_item_nt<FMT, false>(nt, crow, srow, brow, 0, H, H, slot_base, accu);
         // h[p][n] = bf16(silu(g) * u); fragment (row g / g+8, tokens 2c, 2c+1)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < kMaxNT; ++j) {
           if (j >= nt) continue;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int64_t pr = tg + 8 * j + 2 * c + (q & 1);
             if (pr < p1) {
               const int n = mt * 16 + g + ((q & 2) ? 8 : 0);
-              p.h[pr * I + n] = to_bf16_bits(silu_mul(accg[0][j][q], accu[0][j][q]));
+              p.h[pr * I + n] = to_bf16_bits(silu_mul(accg[j][q], accu[j][q]));
             }
           }
         }
@@ -361,31 +376,31 @@ __global__ void __launch_bounds__(kThreads, 2) smallm_layer_kernel(Params p) {
         const int64_t p0 = p.offsets[e], p1 = p.offsets[e + 1];
         const int k0 = ks * p.ksplit;
         const int k1 = min(I, k0 + p.ksplit);
-        const uint8_t* crow[1][2];
-        const uint8_t* srow[1][2];
+        const uint8_t* crow[2];
+        const uint8_t* srow[2];
         const int64_t sstride = FMT == E4B_FMT_NF4 ? (I / 64) * 4 : (I / 32);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int64_t row = int64_t(e) * H + mt * 16 + g + 8 * hh;
-          crow[0][hh] = p.dn_codes + row * (I / 2);
-          srow[0][hh] = p.dn_scales + row * sstride;
+          crow[hh] = p.dn_codes + row * (I / 2);
+          srow[hh] = p.dn_scales + row * sstride;
         }
-        for (int64_t tg = p0; tg < p1; tg += 32) {
-          const int nt = int((min(p1 - tg, int64_t(32)) + 7) / 8);
-          const uint16_t* brow[4];
+        for (int64_t tg = p0; tg < p1; tg += kGroup) {
+          const int nt = int((min(p1 - tg, int64_t(kGroup)) + 7) / 8);
+          const uint16_t* brow[kMaxNT];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < kMaxNT; ++j) {
             const int64_t pr = tg + 8 * j + g;
             brow[j] = (j < nt && pr < p1) ? p.h + pr * I : nullptr;
           }
-          float acc[1][4][4];
+          float acc[kMaxNT][4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < kMaxNT; ++j)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) acc[0][j][q] = 0.f;
-          run_item<FMT, 1, true>(crow, srow, brow, nt, k0, k1, I, slot_base, acc);
+            for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+          run_item_nt<FMT, true>(nt, crow, srow, brow, k0, k1, I, slot_base, acc);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < kMaxNT; ++j) {
             if (j >= nt) continue;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -393,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 2) smallm_layer_kernel(Params p) {
               if (pr < p1) {
                 const int slot = p.perm[pr];
                 const int n = mt * 16 + g + ((q & 2) ? 8 : 0);
-                atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * acc[0][j][q]);
+                atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * acc[j][q]);
               }
             }
           }
