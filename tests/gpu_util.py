@@ -31,12 +31,24 @@ def oracle_quantize(fmt, w: np.ndarray):
     return oracle.quantize_pack_mxfp4(w)
 
 
-def small_layer(fmt, E, H, I, seed, std=0.02):
+def _spread(rng, w):
+    """Multiplies every 32-wide block along K by its own power of two in
+    [2^-2, 2^2], so neighbouring blocks get different scales."""
+    E, N, K = w.shape
+    f = np.exp2(rng.integers(-2, 3, size=(E, N, K // 32))).astype(np.float32)
+    return (w.reshape(E, N, K // 32, 32) * f[..., None]).reshape(E, N, K)
+
+
+def small_layer(fmt, E, H, I, seed, std=0.02, spread=False):
     """Random layer quantised by the GPU and by the oracle; checks the codes
-    agree bit for bit. Returns (PackedLayer, oracle tuple (gc, gs, dc, ds))."""
+    agree bit for bit. Returns (PackedLayer, oracle tuple (gc, gs, dc, ds)).
+    spread=True varies the block scales along K by powers of two."""
     rng = np.random.default_rng(seed)
     wgu = (rng.standard_normal((E, 2 * I, H)) * std).astype(np.float32)
     wd = (rng.standard_normal((E, H, I)) * std).astype(np.float32)
+    if spread:
+        wgu = _spread(rng, wgu)
+        wd = _spread(rng, wd)
     gc_d, gs_d = e4b.quantize(fmt, torch.from_numpy(wgu).cuda())
     dc_d, ds_d = e4b.quantize(fmt, torch.from_numpy(wd).cuda())
     gc, gs = oracle_quantize(fmt, wgu)

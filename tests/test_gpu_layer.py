@@ -69,6 +69,24 @@ def test_ragged_shapes(fmt, E, H, I, T, k, path):
     assert_close(y, oracle_layer(fmt, x, ids, gates, ref, E, H, I), f"{fmt} {E}x{H}x{I} T={T} {path}")
 
 
+@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("fmt,E,H,I,T,k", [("nf4", 3, 256, 320, 40, 2), ("mxfp4", 3, 288, 224, 40, 2),
+                                           ("mxfp4", 2, 96, 160, 9, 1)])
+def test_block_scales_and_large_outputs(fmt, E, H, I, T, k, path):
+    # outputs of order 1-10 (where the tolerance is effectively relative) and
+    # block scales that differ by powers of two between neighbouring 32-blocks
+    # along K: a decode that applies one block's scale to another block's
+    # weights fails here
+    layer, ref = small_layer(fmt, E, H, I, seed=T + H, std=0.06, spread=True)
+    x = _x(T, H, seed=2)
+    rng = np.random.default_rng(4)
+    ids, gates = synth.random_ids(rng, T, k, E)
+    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    y_ref = oracle_layer(fmt, x, ids, gates, ref, E, H, I)
+    assert status == 0 and 3.0 < np.abs(y_ref).max() < 100.0
+    assert_close(y, y_ref, f"{fmt} spread {E}x{H}x{I} {path}")
+
+
 EDGE = {
     "single_slot": (1, 1, lambda T, k, E: np.zeros((1, 1), np.int32)),
     "all_on_one_expert": (300, 2, lambda T, k, E: np.full((T, k), 3, np.int32)),
