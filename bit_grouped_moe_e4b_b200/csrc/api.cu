@@ -34,9 +34,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace of the layer forward.
+// Workspace of the layer forward. Everything up to total_min is required;
+// xs (the routed rows of x in expert order) is the large-M path's staging
+// copy, used when the workspace reaches total.
 struct MoeWs {
-  size_t status, sync, nsync, counts, offsets, perm, inv, h, acc, total;
+  size_t status, sync, nsync, counts, offsets, perm, inv, h, acc, total_min, xs, total;
 };
 
 MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
@@ -52,9 +54,19 @@ MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
   w.inv = o;     o = align_up(o + size_t(R) * 4, 256);
   w.h = o;       o = align_up(o + size_t(R) * size_t(I) * 2, 256);
   w.acc = o;     o = align_up(o + size_t(T) * size_t(H) * 4, 256);
+  w.total_min = o;
+  w.xs = o;      o = align_up(o + size_t(R) * size_t(H) * 2, 256);
   w.total = o;
   return w;
 }
+
+}  // namespace
+
+size_t e4b::moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
+  return moe_ws_layout(E, H, I, T, top_k).total_min;
+}
+
+namespace {
 
 e4b_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return E4B_OK;
@@ -251,7 +263,7 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
       !aligned16(w->down_codes) || !aligned16(w->gate_up_scales) || !aligned16(w->down_scales))
     return E4B_ERR_MISALIGNED;
   const MoeWs L = moe_ws_layout(E, H, I, T, top_k);
-  if (ws_bytes < L.total) return E4B_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < L.total_min) return E4B_ERR_WORKSPACE_TOO_SMALL;
 
   const int64_t R = T * top_k;
   const bool gemv = choose_gemv(R, E, flags);
@@ -306,6 +318,15 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
     return E4B_OK;
   }
 
+  // Large-M: stage the routed rows of x in expert order when the workspace
+  // holds the copy (contiguous TMA row tiles), else gather them in the kernel.
+  const bool staged = ws_bytes >= L.total;
+  uint16_t* xs = staged ? reinterpret_cast<uint16_t*>(base + L.xs) : nullptr;
+  if (staged) {
+    ce = launch_gather_rows(x, H, perm, top_k, offsets, int32_t(E), R, xs, s, sm_count());
+    if (ce != cudaSuccess) return E4B_ERR_CUDA;
+  }
+
   GemmProblem g{};
   g.fmt = w->fmt;
   g.epilogue = E4B_EPI_SWIGLU;
@@ -316,9 +337,9 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   g.R_max = R;
   g.codes = w->gate_up_codes;
   g.scales = w->gate_up_scales;
-  g.a = x;
+  g.a = staged ? xs : x;
   g.lda = H;
-  g.row_slot = perm;
+  g.row_slot = staged ? nullptr : perm;
   g.out_slot = perm;
   g.offsets = offsets;
   g.out = h;
@@ -355,7 +376,7 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   if (ce != cudaSuccess) return E4B_ERR_CUDA;
   mark(4, s);
   g_last_path = gemv ? E4B_PATH_GEMV : E4B_PATH_TCGEN05;
-  g_last_launches = 4;
+  g_last_launches = staged ? 5 : 4;
   return E4B_OK;
 }
 

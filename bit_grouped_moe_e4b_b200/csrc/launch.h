@@ -21,6 +21,13 @@ size_t route_smem_bytes(int32_t E);
 cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* counts, int64_t* offsets,
                          int32_t* perm, int32_t* inv, int32_t* active, int32_t* status,
                          cudaStream_t st, int32_t* clear = nullptr, int32_t nclear = 0);
+// xs[p] = x[perm[p] / top_k] for p < offsets[E] (H % 8 == 0, 16-byte aligned).
+cudaError_t launch_gather_rows(const uint16_t* x, int64_t H, const int32_t* perm, int32_t top_k,
+                               const int64_t* offsets, int32_t E, int64_t R_max, uint16_t* xs,
+                               cudaStream_t st, int sms);
+// Smallest workspace e4b_moe_forward accepts (without the staging copy of the
+// routed rows that e4b_moe_workspace_size includes).
+size_t moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k);
 
 // Description of one grouped projection as the kernels see it.
 struct GemmProblem {

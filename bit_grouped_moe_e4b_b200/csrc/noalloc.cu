@@ -41,10 +41,13 @@ extern "C" e4b_status e4b_moe_forward_noalloc(const e4b_moe_weights* w, const ui
                                               const float* gates, uint16_t* y, uint32_t flags,
                                               void* stream) {
   if (!w || T < 0 || top_k <= 0) return E4B_ERR_INVALID_ARG;
-  size_t need = 0;
-  e4b_status st = e4b_moe_workspace_size(w, T, top_k, &need);
+  size_t full = 0;
+  e4b_status st = e4b_moe_workspace_size(w, T, top_k, &full);
   if (st != E4B_OK) return st;
-  if (need > kNoallocScratchBytes) return E4B_ERR_EXCEEDS_STATIC_SCRATCH;
+  // The staging copy of the routed rows is optional: without room for it the
+  // large-M path gathers the rows inside its kernel.
+  if (e4b::moe_workspace_min_bytes(w->E, w->H, w->I, T, top_k) > kNoallocScratchBytes)
+    return E4B_ERR_EXCEEDS_STATIC_SCRATCH;
   if (T == 0) return e4b_moe_forward(w, x, T, top_k, ids, gates, y, nullptr, 0, flags, stream);
   void* scratch = nullptr;
   st = scratch_for_current_device(&scratch);

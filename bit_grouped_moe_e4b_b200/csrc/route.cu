@@ -150,4 +150,37 @@ cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* coun
   return cudaGetLastError();
 }
 
+// The routed activation rows in expert order, xs[p] = x[perm[p] / top_k] for
+// p < offsets[E], so that the large-M projection reads its B operand as
+// contiguous row tiles. One warp per row, 16-byte copies; rows of dropped
+// slots (p >= offsets[E]) are not written.
+constexpr int kGatherThreads = 256;
+
+__global__ void __launch_bounds__(kGatherThreads)
+gather_rows_kernel(const uint16_t* __restrict__ x, int64_t H, const int32_t* __restrict__ perm,
+                   int32_t top_k, const int64_t* __restrict__ offsets, int32_t E,
+                   uint16_t* __restrict__ xs) {
+  const int64_t R = offsets[E];
+  const int64_t chunks = H / 8;
+  const int warps = kGatherThreads / 32;
+  const int lane = threadIdx.x & 31;
+  for (int64_t p = int64_t(blockIdx.x) * warps + (threadIdx.x >> 5); p < R;
+       p += int64_t(gridDim.x) * warps) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + int64_t(perm[p] / top_k) * H);
+    uint4* dst = reinterpret_cast<uint4*>(xs + p * H);
+    for (int64_t c = lane; c < chunks; c += 32) dst[c] = __ldg(src + c);
+  }
+}
+
+cudaError_t launch_gather_rows(const uint16_t* x, int64_t H, const int32_t* perm, int32_t top_k,
+                               const int64_t* offsets, int32_t E, int64_t R_max, uint16_t* xs,
+                               cudaStream_t st, int sms) {
+  const int64_t warps = kGatherThreads / 32;
+  int64_t grid = (R_max + warps - 1) / warps;
+  if (grid > int64_t(sms) * 8) grid = int64_t(sms) * 8;
+  if (grid < 1) grid = 1;
+  gather_rows_kernel<<<int(grid), kGatherThreads, 0, st>>>(x, H, perm, top_k, offsets, E, xs);
+  return cudaGetLastError();
+}
+
 }  // namespace e4b

@@ -1,6 +1,6 @@
 // Thin wrappers over the sm_100a PTX used by the tcgen05 grouped GEMM:
-// mbarriers (with bounded waits), TMA tile loads, cp.async, proxy fences and
-// the tcgen05 family (TMEM allocation, MMA, commit, loads).
+// mbarriers (with bounded waits), TMA tile and row-gather loads, cp.async,
+// proxy fences and the tcgen05 family (TMEM allocation, MMA, commit, loads).
 #pragma once
 
 #include <cstdint>
@@ -66,6 +66,18 @@ E4B_DEV void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int32_t x, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
       "%4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Four rows of a 2-D tensor (rows r0..r3, columns [x, x + box width)) into
+// four consecutive rows of the destination tile. The tensor map's box must be
+// one row high.
+E4B_DEV void tma_gather4_2d(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t r0,
+                            int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
       : "memory");
 }
 

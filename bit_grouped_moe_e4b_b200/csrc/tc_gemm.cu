@@ -5,20 +5,27 @@
 // accumulation; bf16 epilogue. bitsandbytes PR #1984, Design: gated SiLU
 // (SwiGLU) between the projections; the top-k weighted sum after the second.
 //
-// sm_100a design, one persistent CTA per SM, warp-specialised:
-//   warp 0      TMA: packed codes of the tile's weight rows, [128 rows x 32 B]
-//               per matrix and 64-wide K block, into a staging ring.
+// sm_100a design, one persistent CTA per SM, warp-specialised, with three
+// independent shared-memory rings so that no producer waits on a consumer
+// further down the chain than its own ring:
+//   codes ring  (warp 0, TMA)  packed codes of the tile's weight rows,
+//               [128 rows x 32 B] per matrix and 64-wide K block; a slot is
+//               released by the decoders as soon as they hold the codes in
+//               registers, so code fetches run far ahead of the MMAs;
+//   B ring      (warp 2, TMA)  the routed activation rows, 128B-swizzled
+//               K-major: rows gathered four at a time (tile::gather4) from
+//               a[row_slot[p] / top_k], or one 256-row tile when the rows are
+//               contiguous; released by the MMA;
+//   A ring      (warps 4-11)   decoders: each thread takes one weight row of a
+//               job, builds its block's 16-entry bf16 table and writes 64
+//               decoded weights (128B-swizzled K-major); released by the MMA.
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer
 //               (M = 128 weight rows, N = 256 routed rows, K = 16 per MMA).
-//   warps 2-3   cp.async gather of the routed activation rows (row p of an
-//               expert reads a[row_slot[p] / top_k]) into the B ring, written
-//               in the 128B-swizzled K-major layout; missing rows zero-filled.
-//   warps 4-11  decoders: each thread owns one weight row of a stage, builds
-//               its block's 16-entry bf16 table and writes 64 decoded weights
-//               as the A operand (128B-swizzled K-major) for the MMA.
 //   warps 12-15 epilogue: tcgen05.ld of the fp32 accumulators, then SwiGLU
 //               (gate and up accumulate in two TMEM column ranges of the same
 //               lanes, so it is thread-local) or the gate-weighted combine.
+//               A single-matrix projection has two accumulators in TMEM, so
+//               the epilogue of one tile overlaps the MMAs of the next.
 // Tiles: per active expert, (weight-row block of 128) x (routed-row block of
 // 256), routed-row blocks fastest so CTAs running together share A in L2.
 // Every wait is bounded; a wait that gives up records E4B_ERR_DEVICE_TIMEOUT,
@@ -37,31 +44,43 @@ using namespace sm100;
 
 constexpr int BM = 128;   // weight rows per matrix per tile (MMA M)
 constexpr int BN = 256;   // routed rows per tile (MMA N)
-constexpr int BK = 64;    // K per stage: one 128-byte swizzle row of bf16
+constexpr int BK = 64;    // K per job: one 128-byte swizzle row of bf16
 constexpr int kThreads = 512;
 constexpr int kMaxE = 256;
-constexpr int kLoaderThreads = 64;
 constexpr int kDecoderThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kATileBytes = BM * BK * 2;   // 16 KB
 constexpr uint32_t kBTileBytes = BN * BK * 2;   // 32 KB
 constexpr uint32_t kCTileBytes = BM * BK / 2;   // 4 KB packed codes
+constexpr int kScalePrefetch = 4;               // jobs of absmax / scale loads in flight
 
 template <int NMAT>
 struct Cfg {
-  static constexpr int NS = NMAT == 2 ? 3 : 4;
+  static constexpr int CS = NMAT == 2 ? 6 : 10;    // codes stages
+  static constexpr int AS = NMAT == 2 ? 2 : 4;     // decoded-A stages
+  static constexpr int BS = 3;                     // activation stages
+  static constexpr int NACC = NMAT == 2 ? 1 : 2;   // accumulators in TMEM
+  static constexpr int kDecPerJob = NMAT == 2 ? kDecoderThreads : kDecoderThreads / 2;
   static constexpr uint32_t kA = 0;
-  static constexpr uint32_t kB = kA + NS * NMAT * kATileBytes;
-  static constexpr uint32_t kC = kB + NS * kBTileBytes;
-  static constexpr uint32_t kMisc = kC + NS * NMAT * kCTileBytes;
-  // misc: barriers, then scalars, then the expert tables
-  static constexpr uint32_t kBars = kMisc;                      // (4*NS + 2) x 8 B
-  static constexpr uint32_t kScal = kBars + (4 * NS + 2) * 8;   // 16 B
+  static constexpr uint32_t kB = kA + AS * NMAT * kATileBytes;
+  static constexpr uint32_t kC = kB + BS * kBTileBytes;
+  static constexpr uint32_t kMisc = kC + CS * NMAT * kCTileBytes;
+  // misc: barriers, scalars, the expert tables
+  static constexpr int kNumBars = 2 * (CS + AS + BS + 2);
+  static constexpr uint32_t kBars = kMisc;
+  static constexpr uint32_t kScal = kBars + kNumBars * 8;       // 16 B
   static constexpr uint32_t kAct = kScal + 16;                  // kMaxE x 4
   static constexpr uint32_t kPre = kAct + kMaxE * 4;            // (kMaxE + 1) x 4
   static constexpr uint32_t kEnd = kPre + (kMaxE + 1) * 4;
   static constexpr uint32_t kSmemBytes = kEnd + 1024;           // + alignment slack
-  static constexpr uint32_t kTmemCols = NMAT * BN;              // 256 or 512
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  // With one matrix the decoders split into two groups that take alternate
+  // jobs. A parity wait must never run two phases ahead of its barrier, so
+  // every slot of a ring the groups wait on must belong to one group only:
+  // an even number of slots.
+  static_assert(NMAT == 2 || (CS % 2 == 0 && AS % 2 == 0), "decoder groups own alternate slots");
+  static_assert(NMAT * BN * (NMAT == 2 ? 1 : NACC) <= 512, "TMEM budget");
 };
 
 struct Tile {
@@ -100,21 +119,27 @@ struct Sched {
 
 template <int FMT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, GemmProblem p) {
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
+               const __grid_constant__ CUtensorMap tmap_act, GemmProblem p) {
   constexpr int NMAT = (EPI == E4B_EPI_SWIGLU) ? 2 : 1;
   using C = Cfg<NMAT>;
-  constexpr int NS = C::NS;
+  constexpr int CS = C::CS;
+  constexpr int AS = C::AS;
+  constexpr int BS = C::BS;
+  constexpr int NACC = C::NACC;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBars);
-  uint64_t* tma_full = bars;
-  uint64_t* a_full = bars + NS;
-  uint64_t* b_full = bars + 2 * NS;
-  uint64_t* empty = bars + 3 * NS;
-  uint64_t* acc_full = bars + 4 * NS;
-  uint64_t* acc_empty = bars + 4 * NS + 1;
+  uint64_t* c_full = bars;
+  uint64_t* c_empty = c_full + CS;
+  uint64_t* a_full = c_empty + CS;
+  uint64_t* a_empty = a_full + AS;
+  uint64_t* b_full = a_empty + AS;
+  uint64_t* b_empty = b_full + BS;
+  uint64_t* acc_full = b_empty + BS;
+  uint64_t* acc_empty = acc_full + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kScal);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kScal + 4);
   int32_t* s_n = reinterpret_cast<int32_t*>(smem + C::kScal + 8);
@@ -170,14 +195,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, GemmProblem p) {
   if (int(blockIdx.x) >= sc.total) return;  // no tile for this CTA (uniform)
 
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&tma_full[s], 1);
-      mbar_init(&a_full[s], NMAT == 2 ? kDecoderThreads : kDecoderThreads / 2);
-      mbar_init(&b_full[s], kLoaderThreads);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < CS; ++s) {
+      mbar_init(&c_full[s], 1);
+      mbar_init(&c_empty[s], C::kDecPerJob);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiThreads);
+    for (int s = 0; s < AS; ++s) {
+      mbar_init(&a_full[s], C::kDecPerJob);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < BS; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiThreads);
+    }
     *s_abort = 0;
     mbar_init_fence();
   }
@@ -196,34 +229,34 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, GemmProblem p) {
   };
 
   const int my_tiles = (sc.total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x);
-  const int64_t njobs = int64_t(my_tiles) * KB;  // k-blocks this CTA walks
+  const int64_t njobs = int64_t(my_tiles) * KB;  // (tile, k-block) jobs this CTA walks
 
   if (warp == 0) {
-    // ---------------------------------------------------------- TMA codes
+    // --------------------------------------------------- codes ring (TMA)
     if (lane == 0) {
       int64_t i = 0;
-      for (int j = 0; j < my_tiles && !*s_abort; ++j) {
+      bool aborted = false;
+      for (int j = 0; j < my_tiles && !aborted; ++j) {
         const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
         for (int kb = 0; kb < KB; ++kb, ++i) {
-          const int s = int(i % NS);
-          const uint32_t ph = uint32_t(i / NS) & 1u;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, s_abort)) {
+          const int s = int(i % CS);
+          if (!mbar_wait_bounded(&c_empty[s], (uint32_t(i / CS) & 1u) ^ 1u, limit, s_abort)) {
             give_up();
+            aborted = true;
             break;
           }
-          mbar_arrive_expect_tx(&tma_full[s], NMAT * kCTileBytes);
+          mbar_arrive_expect_tx(&c_full[s], NMAT * kCTileBytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             const int64_t row = int64_t(T.e) * N + m * rows_per_mat + T.mt * BM;
-            tma_load_2d(smem + C::kC + (s * NMAT + m) * kCTileBytes, &tmap_codes, &tma_full[s],
+            tma_load_2d(smem + C::kC + (s * NMAT + m) * kCTileBytes, &tmap_codes, &c_full[s],
                         kb * (BK / 2), int32_t(row));
           }
         }
       }
       // Drain: every load issued must land before the CTA can exit.
-      const int64_t first = i > NS ? i - NS : 0;
-      for (int64_t q = first; q < i; ++q)
-        mbar_wait_bounded(&tma_full[q % NS], uint32_t(q / NS) & 1u, kWaitPolls, nullptr);
+      for (int64_t q = i > CS ? i - CS : 0; q < i; ++q)
+        mbar_wait_bounded(&c_full[q % CS], uint32_t(q / CS) & 1u, kWaitPolls, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
@@ -232,169 +265,181 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, GemmProblem p) {
       int64_t i = 0;
       uint64_t* last_bar = nullptr;
       uint32_t last_ph = 0;
-      for (int j = 0; j < my_tiles && !*s_abort; ++j) {
-        if (!mbar_wait_bounded(acc_empty, (uint32_t(j) & 1u) ^ 1u, limit, s_abort)) {
+      bool aborted = false;
+      for (int j = 0; j < my_tiles && !aborted; ++j) {
+        const int ab = j % NACC;
+        if (!mbar_wait_bounded(&acc_empty[ab], (uint32_t(j / NACC) & 1u) ^ 1u, limit, s_abort)) {
           give_up();
           break;
         }
         tc_fence_after();
-        bool ok = true;
+        const uint32_t dcol = tmem + uint32_t(NMAT == 2 ? 0 : ab * BN);
         for (int kb = 0; kb < KB; ++kb, ++i) {
-          const int s = int(i % NS);
-          const uint32_t ph = uint32_t(i / NS) & 1u;
-          if (!mbar_wait_bounded(&a_full[s], ph, limit, s_abort) ||
-              !mbar_wait_bounded(&b_full[s], ph, limit, s_abort)) {
+          const int as = int(i % AS);
+          const int bs = int(i % BS);
+          if (!mbar_wait_bounded(&a_full[as], uint32_t(i / AS) & 1u, limit, s_abort) ||
+              !mbar_wait_bounded(&b_full[bs], uint32_t(i / BS) & 1u, limit, s_abort)) {
             give_up();
-            ok = false;
+            aborted = true;
             break;
           }
           tc_fence_after();
-          const uint32_t bbase = smem_u32(smem + C::kB + s * kBTileBytes);
+          const uint32_t bbase = smem_u32(smem + C::kB + bs * kBTileBytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
-            const uint32_t abase = smem_u32(smem + C::kA + (s * NMAT + m) * kATileBytes);
+            const uint32_t abase = smem_u32(smem + C::kA + (as * NMAT + m) * kATileBytes);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              mma_bf16_ss(tmem + uint32_t(m * BN), sw128_kmajor_desc(abase + kk * 32),
+              mma_bf16_ss(dcol + uint32_t(m * BN), sw128_kmajor_desc(abase + kk * 32),
                           sw128_kmajor_desc(bbase + kk * 32), idesc, (kb | kk) ? 1u : 0u);
             }
           }
-          mma_commit(&empty[s]);
-          last_bar = &empty[s];
-          last_ph = ph;
+          mma_commit(&a_empty[as]);
+          mma_commit(&b_empty[bs]);
+          last_bar = &b_empty[bs];
+          last_ph = uint32_t(i / BS) & 1u;
         }
-        if (!ok) break;
-        mma_commit(acc_full);
-        last_bar = acc_full;
-        last_ph = uint32_t(j) & 1u;
+        if (aborted) break;
+        mma_commit(&acc_full[ab]);
       }
       // Drain: the MMAs issued so far must finish before TMEM is freed.
       if (*s_abort && last_bar) mbar_wait_bounded(last_bar, last_ph, kWaitPolls, nullptr);
     }
-  } else if (warp < 4) {
-    // ------------------------------------------- activation rows (B operand)
-    const int lt = tid - 64;  // 0..63
-    const uint16_t* src[4];
+  } else if (warp == 2) {
+    // ------------------------------------ activation rows, B ring (TMA)
+    // Gathered rows: lane l issues the four-row gathers l and l + 32 of each
+    // job (rows 4l..4l+3 and 128+4l..128+4l+3 of the tile), so the 64 copies
+    // of a job leave in two warp-wide instructions.
+    const bool gather = p.row_slot != nullptr;
     int64_t i = 0;
-    int64_t signaled = 0;
-    constexpr int LAG = NS - 1;
     bool aborted = false;
     for (int j = 0; j < my_tiles && !aborted; ++j) {
       const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
+      int32_t gr[8];
+      if (gather) {
+        // rows past the expert's end repeat its first row (products discarded)
+        const int32_t first = p.row_slot[T.p0] / p.top_k;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int64_t pr = T.p0 + lt + 64 * q;
-        src[q] = nullptr;
-        if (pr < T.p1) {
-          const int64_t ar = p.row_slot ? int64_t(p.row_slot[pr] / p.top_k) : pr;
-          src[q] = p.a + ar * p.lda;
+        for (int q = 0; q < 8; ++q) {
+          const int64_t pr = T.p0 + 4 * lane + (q >> 2) * 128 + (q & 3);
+          gr[q] = pr < T.p1 ? p.row_slot[pr] / p.top_k : first;
         }
       }
       for (int kb = 0; kb < KB; ++kb, ++i) {
-        const int s = int(i % NS);
-        const uint32_t ph = uint32_t(i / NS) & 1u;
-        if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, s_abort)) {
-          give_up();
+        const int s = int(i % BS);
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait_bounded(&b_empty[s], (uint32_t(i / BS) & 1u) ^ 1u, limit, s_abort);
+          if (ok) mbar_arrive_expect_tx(&b_full[s], kBTileBytes);
+          else give_up();
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
           aborted = true;
           break;
         }
-        uint8_t* bt = smem + C::kB + s * kBTileBytes;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int r = lt + 64 * q;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const int64_t k = int64_t(kb) * BK + c * 8;
-            const bool v = src[q] != nullptr && k < K;
-            cp_async_16(bt + r * 128 + ((c ^ (r & 7)) << 4), v ? (const void*)(src[q] + k) : (const void*)p.a,
-                        v ? 16u : 0u);
-          }
-        }
-        cp_async_commit();
-        if (i - signaled >= LAG) {
-          cp_async_wait<LAG>();
-          fence_proxy_async_smem();
-          mbar_arrive(&b_full[signaled % NS]);
-          ++signaled;
+        uint8_t* dst = smem + C::kB + s * kBTileBytes;
+        if (gather) {
+          tma_gather4_2d(dst + lane * 512, &tmap_act, &b_full[s], kb * BK, gr[0], gr[1], gr[2], gr[3]);
+          tma_gather4_2d(dst + (lane + 32) * 512, &tmap_act, &b_full[s], kb * BK, gr[4], gr[5], gr[6],
+                         gr[7]);
+        } else if (lane == 0) {
+          tma_load_2d(dst, &tmap_act, &b_full[s], kb * BK, int32_t(T.p0));
         }
       }
     }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    if (!aborted) {
-      for (; signaled < i; ++signaled) mbar_arrive(&b_full[signaled % NS]);
+    if (lane == 0) {
+      for (int64_t q = i > BS ? i - BS : 0; q < i; ++q)
+        mbar_wait_bounded(&b_full[q % BS], uint32_t(q / BS) & 1u, kWaitPolls, nullptr);
     }
-  } else if (warp < 12) {
+  } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------ decoders (A operand)
     const int d = tid - 128;                  // 0..255
     const int m = NMAT == 2 ? (d >> 7) : 0;   // matrix (gate / up)
     const int r = d & 127;                    // row within the tile
-    const int grp = NMAT == 2 ? 0 : (d >> 7); // NMAT == 1: two groups take alternate k-blocks
-    const int step = NMAT == 2 ? 1 : 2;
+    const int grp = NMAT == 2 ? 0 : (d >> 7); // NMAT == 1: two groups take alternate jobs
+    constexpr int step = NMAT == 2 ? 1 : 2;
     const uint8_t* scales = static_cast<const uint8_t*>(p.scales);
     const int64_t sstride = FMT == E4B_FMT_NF4 ? (K / 64) * 4 : (K / 32);
 
-    // Scale of this thread's row at job i (k-block i % KB of its tile).
+    // Absmax (NF4, as fp32 bits) or the two scale bytes (MXFP4) of this
+    // thread's row at job q.
     int cached_j = -1;
     const uint8_t* srow = nullptr;
-    auto scale_at = [&](int64_t i, int& cj, const uint8_t*& sr) -> uint32_t {
-      if (i >= njobs) return 0u;
-      const int j = int(i / KB);
-      const int kb = int(i % KB);
-      if (j != cj) {
-        cj = j;
+    auto scale_at = [&](int64_t q) -> uint32_t {
+      if (q >= njobs) return 0u;
+      const int j = int(q / KB);
+      const int kb = int(q % KB);
+      if (j != cached_j) {
+        cached_j = j;
         const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
         const int64_t n = T.mt * BM + r;
-        sr = n < rows_per_mat ? scales + (int64_t(T.e) * N + m * rows_per_mat + n) * sstride : nullptr;
+        srow = n < rows_per_mat ? scales + (int64_t(T.e) * N + m * rows_per_mat + n) * sstride
+                                : nullptr;
       }
-      if (!sr) return 0u;
+      if (!srow) return 0u;
       if constexpr (FMT == E4B_FMT_NF4) {
-        return __float_as_uint(__ldg(reinterpret_cast<const float*>(sr) + kb));
+        return __float_as_uint(__ldg(reinterpret_cast<const float*>(srow) + kb));
       } else {
         const int64_t b0 = int64_t(kb) * 2;
-        const uint32_t lo = b0 < K / 32 ? uint32_t(__ldg(sr + b0)) : 0u;
-        const uint32_t hi = b0 + 1 < K / 32 ? uint32_t(__ldg(sr + b0 + 1)) : 0u;
+        const uint32_t lo = b0 < K / 32 ? uint32_t(__ldg(srow + b0)) : 0u;
+        const uint32_t hi = b0 + 1 < K / 32 ? uint32_t(__ldg(srow + b0 + 1)) : 0u;
         return lo | (hi << 8);
       }
     };
-    int cj2 = -1;
-    const uint8_t* sr2 = nullptr;
-    int64_t i = grp;
-    uint32_t sc1 = scale_at(i, cached_j, srow);
-    uint32_t sc2 = scale_at(i + step, cj2, sr2);
-    for (; i < njobs; i += step) {
-      const uint32_t cur = sc1;
-      sc1 = sc2;
-      sc2 = scale_at(i + 2 * step, cj2, sr2);
-      const int s = int(i % NS);
-      const uint32_t ph = uint32_t(i / NS) & 1u;
-      if (!mbar_wait_bounded(&tma_full[s], ph, limit, s_abort)) {
-        give_up();
-        break;
-      }
-      const uint4* crow = reinterpret_cast<const uint4*>(smem + C::kC + (s * NMAT + m) * kCTileBytes + r * 32);
-      const uint4 c0 = crow[0];
-      const uint4 c1 = crow[1];
-      const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      uint8_t* arow = smem + C::kA + (s * NMAT + m) * kATileBytes + r * 128;
-      Lut L;
-      lut_build<FMT>(L, __uint_as_float(cur), cur & 0xFFu);
+    uint32_t ring[kScalePrefetch];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (FMT == E4B_FMT_MXFP4 && c == 4) lut_build<FMT>(L, 0.f, (cur >> 8) & 0xFFu);
-        uint32_t o[4];
-        lut_decode8<FMT>(L, words[c], o);
-        *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int u = 0; u < kScalePrefetch; ++u) ring[u] = scale_at(grp + int64_t(u) * step);
+
+    bool aborted = false;
+    for (int64_t i0 = grp; i0 < njobs && !aborted; i0 += int64_t(kScalePrefetch) * step) {
+#pragma unroll
+      for (int u = 0; u < kScalePrefetch; ++u) {
+        const int64_t i = i0 + int64_t(u) * step;
+        if (i >= njobs) break;
+        const uint32_t cur = ring[u];
+        ring[u] = scale_at(i + int64_t(kScalePrefetch) * step);
+        const int cs = int(i % CS);
+        if (!mbar_wait_bounded(&c_full[cs], uint32_t(i / CS) & 1u, limit, s_abort)) {
+          give_up();
+          aborted = true;
+          break;
+        }
+        const uint4* crow =
+            reinterpret_cast<const uint4*>(smem + C::kC + (cs * NMAT + m) * kCTileBytes + r * 32);
+        const uint4 c0 = crow[0];
+        const uint4 c1 = crow[1];
+        // The slot's next fill is a TMA write (async proxy); without this
+        // fence it can overtake the generic-proxy reads just issued.
+        fence_proxy_async_smem();
+        mbar_arrive(&c_empty[cs]);
+        const int as = int(i % AS);
+        if (!mbar_wait_bounded(&a_empty[as], (uint32_t(i / AS) & 1u) ^ 1u, limit, s_abort)) {
+          give_up();
+          aborted = true;
+          break;
+        }
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint8_t* arow = smem + C::kA + (as * NMAT + m) * kATileBytes + r * 128;
+        Lut L;
+        lut_build<FMT>(L, __uint_as_float(cur), cur & 0xFFu);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (FMT == E4B_FMT_MXFP4 && c == 4) lut_build<FMT>(L, 0.f, (cur >> 8) & 0xFFu);
+          uint32_t o[4];
+          lut_decode8<FMT>(L, words[c], o);
+          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&a_full[as]);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&a_full[s]);
     }
-  } else {
+  } else if (warp >= 12) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may read
     const int rloc = q * 32 + lane;
     for (int j = 0; j < my_tiles; ++j) {
-      if (!mbar_wait_bounded(acc_full, uint32_t(j) & 1u, limit, s_abort)) {
+      const int ab = j % NACC;
+      if (!mbar_wait_bounded(&acc_full[ab], uint32_t(j / NACC) & 1u, limit, s_abort)) {
         give_up();
         break;
       }
@@ -402,15 +447,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, GemmProblem p) {
       const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
       const int64_t n = T.mt * BM + rloc;
       const bool nvalid = n < rows_per_mat;
-      const uint32_t lane_base = tmem + (uint32_t(q * 32) << 16);
+      const uint32_t lane_base =
+          tmem + (uint32_t(q * 32) << 16) + uint32_t(NMAT == 2 ? 0 : ab * BN);
       for (int cc = 0; cc < BN / 16; ++cc) {
+        const int64_t pbase = T.p0 + cc * 16;
+        if (pbase >= T.p1) break;  // uniform: the rest of the tile is past the expert's rows
         uint32_t g[16];
         uint32_t u[16];
         tmem_ld_32x32b_x16(lane_base + uint32_t(cc * 16), g);
         if constexpr (NMAT == 2) tmem_ld_32x32b_x16(lane_base + uint32_t(BN + cc * 16), u);
         tmem_ld_wait();
-        const int64_t pbase = T.p0 + cc * 16;
-        if (!nvalid || pbase >= T.p1) continue;
+        if (!nvalid) continue;
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int64_t pr = pbase + t;
@@ -429,7 +476,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, GemmProblem p) {
         }
       }
       tc_fence_before();
-      mbar_arrive(acc_empty);
+      mbar_arrive(&acc_empty[ab]);
     }
   }
 
@@ -462,18 +509,37 @@ template <int FMT, int EPI>
 cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
   constexpr int NMAT = (EPI == E4B_EPI_SWIGLU) ? 2 : 1;
   using C = Cfg<NMAT>;
-  // Packed codes viewed as a 2-D byte tensor [E*N rows, K/2 bytes].
-  CUtensorMap tmap;
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return cudaErrorInitializationError;
-  const cuuint64_t gdim[2] = {cuuint64_t(p.K / 2), cuuint64_t(int64_t(p.E) * p.N)};
-  const cuuint64_t gstride[1] = {cuuint64_t(p.K / 2)};
-  const cuuint32_t box[2] = {BK / 2, BM};
-  const cuuint32_t estride[2] = {1, 1};
-  CUresult cr = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.codes), gdim,
-                    gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // Packed codes viewed as a 2-D byte tensor [E*N rows, K/2 bytes].
+  CUtensorMap tmap_codes;
+  {
+    const cuuint64_t gdim[2] = {cuuint64_t(p.K / 2), cuuint64_t(int64_t(p.E) * p.N)};
+    const cuuint64_t gstride[1] = {cuuint64_t(p.K / 2)};
+    const cuuint32_t box[2] = {BK / 2, BM};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = enc(&tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.codes),
+                      gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  // Activations [rows, K] bf16 with row stride lda, landing 128B-swizzled:
+  // single rows for the four-row gather, 256-row tiles for contiguous rows.
+  CUtensorMap tmap_act;
+  {
+    const bool gather = p.row_slot != nullptr;
+    const int64_t rows = gather ? (p.R_max + p.top_k - 1) / p.top_k : p.R_max;
+    const cuuint64_t gdim[2] = {cuuint64_t(p.K), cuuint64_t(rows)};
+    const cuuint64_t gstride[1] = {cuuint64_t(p.lda) * 2};
+    const cuuint32_t box[2] = {BK, gather ? 1u : cuuint32_t(BN)};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = enc(&tmap_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(p.a),
+                      gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
 
   auto kern = tc_gemm_kernel<FMT, EPI>;
   static int configured_dev = -1;
@@ -490,7 +556,7 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
   const int64_t max_tiles = MT * ((p.R_max + BN - 1) / BN + p.E);
   int grid = int(max_tiles < sms ? max_tiles : sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kThreads, C::kSmemBytes, st>>>(tmap, p);
+  kern<<<grid, kThreads, C::kSmemBytes, st>>>(tmap_codes, tmap_act, p);
   return cudaGetLastError();
 }
 

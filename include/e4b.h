@@ -211,7 +211,12 @@ e4b_status e4b_grouped_gemm(const e4b_gemm_args* args, uint32_t flags, void* str
 
 /* ---------------------------------------------------------- whole layer */
 
-/* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots. */
+/* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots.
+ * The size includes a staging copy of the routed rows of x in expert order
+ * ([T*top_k, H] bf16) that the large-M path uses; a smaller workspace that
+ * still holds the routing arrays, h, the accumulator and the status word is
+ * accepted, and the large-M path then gathers the rows inside its kernel
+ * (same results, slower). */
 e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
                                   size_t* bytes);
 
@@ -225,7 +230,8 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
  *   y     bf16 [T, H] output: y[t] = bf16( sum_j gates[t,j] * down_e(
  *         bf16(silu(gate_e(x[t])) * up_e(x[t])) ) ), e = ids[t,j]
  *   ws    device scratch of e4b_moe_workspace_size bytes (routing, the bf16
- *         intermediate h [T*top_k, I], an fp32 accumulator [T, H], status)
+ *         intermediate h [T*top_k, I], an fp32 accumulator [T, H], status,
+ *         the optional staging copy of the routed rows)
  *   flags E4B_FLAG_* (0 = choose the path from the shape)
  * The path is chosen on the host from T*top_k/E with no device sync, so the
  * call is graph-capturable. T == 0 is a no-op.
@@ -248,10 +254,11 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
  * scratch (routing arrays, bf16 intermediate, fp32 accumulator, status word)
  * lives in a 16 MiB array in the library's device memory, which every GPU
  * that loads the library keeps until the process exits. A call whose
- * scratch, as e4b_moe_workspace_size reports it, exceeds 16 MiB returns
- * E4B_ERR_EXCEEDS_STATIC_SCRATCH and enqueues nothing (a layer with H=4096,
- * I=14336 and top-2 routing fits up to 227 tokens). Nothing is allocated or
- * freed.
+ * required scratch (e4b_moe_workspace_size without the optional staging
+ * copy) exceeds 16 MiB returns E4B_ERR_EXCEEDS_STATIC_SCRATCH and enqueues
+ * nothing (a layer with H=4096, I=14336 and top-2 routing fits up to 227
+ * tokens; the staging copy is used while it also fits). Nothing is allocated
+ * or freed.
  *   - The first call on each device looks up that device's copy of the
  *     array (set-up, once per device); make that first call before any stream
  *     capture begins.

@@ -59,11 +59,16 @@ def small_layer(fmt, E, H, I, seed, std=0.02, spread=False):
     return layer, (gc, gs, dc, ds)
 
 
-def run_layer(layer, x_bf16: torch.Tensor, ids: np.ndarray, gates: np.ndarray, flags=0):
+def run_layer(layer, x_bf16: torch.Tensor, ids: np.ndarray, gates: np.ndarray, flags=0, staged=True):
+    """staged=False hands the layer a workspace without room for the staging
+    copy of the routed rows (the last [T*k, H] bf16 region), so the large-M
+    path gathers the rows inside its kernel."""
     ids_d = torch.from_numpy(np.ascontiguousarray(ids, np.int32)).cuda()
     g_d = torch.from_numpy(np.ascontiguousarray(gates, np.float32)).cuda()
     x_d = x_bf16.cuda()
     ws = e4b.workspace(layer, ids.shape[0], ids.shape[1])
+    if not staged:
+        ws = ws[: ws.numel() - (ids.size * layer.H * 2 + 255) // 256 * 256]
     y = e4b.moe_forward(layer, x_d, ids_d, g_d, ws=ws, flags=flags)
     status = e4b.e4b_read_device_status(ws)
     return y.float().cpu().numpy(), status, ws

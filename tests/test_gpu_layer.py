@@ -13,7 +13,14 @@ from gpu_util import assert_close, oracle_layer, run_layer, small_layer
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"gemv": e4b.FLAG_FORCE_GEMV, "tcgen05": e4b.FLAG_FORCE_TCGEN05}
+PATHS = {"gemv": e4b.FLAG_FORCE_GEMV, "tcgen05": e4b.FLAG_FORCE_TCGEN05,
+         "tcgen05_gather": e4b.FLAG_FORCE_TCGEN05}
+
+
+def _run(layer, x, ids, gates, path):
+    # "tcgen05_gather": a workspace without the staging copy of the routed
+    # rows, so the tcgen05 kernel gathers them with four-row TMA copies
+    return run_layer(layer, x, ids, gates, PATHS[path], staged=path != "tcgen05_gather")
 
 
 def _x(T, H, seed):
@@ -42,8 +49,9 @@ def test_tiny_workload(path):
     assert_close(y, y_ref, f"tiny workload, {path}")
     if path != "auto":
         assert e4b.e4b_last_path() == (e4b.E4B_PATH_GEMV if path == "gemv" else e4b.E4B_PATH_TCGEN05)
-    # small-M: routing + one fused layer kernel; tcgen05: routing, two GEMMs, conversion
-    assert e4b.e4b_last_launch_count() == (2 if e4b.e4b_last_path() == e4b.E4B_PATH_GEMV else 4)
+    # small-M: routing + one fused layer kernel; tcgen05: routing, staging of
+    # the routed rows, two GEMMs, conversion
+    assert e4b.e4b_last_launch_count() == (2 if e4b.e4b_last_path() == e4b.E4B_PATH_GEMV else 5)
 
 
 # shapes that span several tiles of both kernels and leave ragged tails:
@@ -57,16 +65,37 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
 @pytest.mark.parametrize("fmt,E,H,I,T,k", SHAPES)
 def test_ragged_shapes(fmt, E, H, I, T, k, path):
     layer, ref = small_layer(fmt, E, H, I, seed=E * 100 + H)
     x = _x(T, H, seed=T)
     rng = np.random.default_rng(T + k)
     ids, gates = synth.random_ids(rng, T, k, E)
-    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    y, status, _ = _run(layer, x, ids, gates, path)
     assert status == 0
     assert_close(y, oracle_layer(fmt, x, ids, gates, ref, E, H, I), f"{fmt} {E}x{H}x{I} T={T} {path}")
+
+
+_many = {}
+
+
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+def test_many_tiles_per_cta(path):
+    # 64 experts x 4 weight-row tiles per projection = 256 tcgen05 tiles, more
+    # than one per SM, with 8 k-blocks each: the persistent kernels walk
+    # several tiles per CTA and their staging rings wrap many times
+    fmt, E, H, I, T, k = "nf4", 64, 512, 512, 256, 4
+    if not _many:
+        _many["layer"] = small_layer(fmt, E, H, I, seed=64)
+        x = _x(T, H, seed=5)
+        ids, gates = synth.random_ids(np.random.default_rng(6), T, k, E)
+        _many["case"] = (x, ids, gates, oracle_layer(fmt, x, ids, gates, _many["layer"][1], E, H, I))
+    layer, _ = _many["layer"]
+    x, ids, gates, y_ref = _many["case"]
+    y, status, _ = _run(layer, x, ids, gates, path)
+    assert status == 0
+    assert_close(y, y_ref, f"{fmt} {E}x{H}x{I} T={T} {path}")
 
 
 @pytest.mark.parametrize("path", ["gemv", "tcgen05"])
@@ -96,7 +125,7 @@ EDGE = {
 }
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
 @pytest.mark.parametrize("case", list(EDGE))
 def test_degenerate_routing(case, path):
     E, H, I = 4, 128, 256
@@ -107,18 +136,19 @@ def test_degenerate_routing(case, path):
     x = _x(T, H, seed=3)
     ids = make(T, k, E)
     gates = np.random.default_rng(1).random((T, k)).astype(np.float32)
-    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    y, status, _ = _run(layer, x, ids, gates, path)
     assert status == 0
     assert_close(y, oracle_layer("nf4", x, ids, gates, ref, E, H, I), f"{case} {path}")
 
 
-def test_bad_expert_ids_drop_only_their_slots():
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+def test_bad_expert_ids_drop_only_their_slots(path):
     E, H, I, T = 4, 128, 128, 6
     layer, ref = small_layer("nf4", E, H, I, seed=11)
     x = _x(T, H, seed=5)
     ids = np.array([[0, 1], [9, 2], [3, -4], [1, 1], [2, 0], [3, 3]], np.int32)
     gates = np.random.default_rng(2).random((T, 2)).astype(np.float32)
-    y, status, _ = run_layer(layer, x, ids, gates)
+    y, status, _ = _run(layer, x, ids, gates, path)
     assert status == 6
     g2 = gates.copy()
     ids2 = ids.copy()

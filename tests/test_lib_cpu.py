@@ -65,8 +65,10 @@ def test_host_argument_checks_return_before_launch():
     assert fwd(ctypes.byref(_w(H=96)), p, 4, 2, p, p, p, p, need, 0, None) == 2
     # misaligned
     assert fwd(ctypes.byref(w), ctypes.c_void_p(4098), 4, 2, p, p, p, p, need, 0, None) == 7
-    # workspace too small
-    assert fwd(ctypes.byref(w), p, 64, 2, p, p, p, p, need - 1, 0, None) == 3
+    # workspace too small: below the required part (the size query adds an
+    # optional [T*k, H] bf16 staging copy at the end, 256-byte aligned)
+    required = need - (64 * 2 * 256 * 2 + 255) // 256 * 256
+    assert fwd(ctypes.byref(w), p, 64, 2, p, p, p, p, required - 1, 0, None) == 3
     # bad format
     assert fwd(ctypes.byref(_w(fmt=5)), p, 4, 2, p, p, p, p, need, 0, None) == 1
     # (every call above and below fails validation, so nothing is launched
