@@ -177,7 +177,8 @@ def kernel_bytes(wl, T, ids):
     R = ids.size
     gu = active * 2 * wl.I * wl.H * bpw + 2 * T * wl.H + 4 * R
     dn = active * wl.H * wl.I * bpw + 2 * T * wl.H + 4 * R
-    return {"gate_up": gu, "down": dn, "smallm_layer": gu + dn, "active_experts": active,
+    return {"gate_up": gu, "down": dn, "smallm_layer": gu + dn, "finalize": 6 * T * wl.H,
+            "active_experts": active,
             "packed_bytes": active * 3 * wl.H * wl.I * bpw,
             "layer": active * 3 * wl.H * wl.I * bpw + 4 * T * wl.H + 8 * R}
 
@@ -380,7 +381,6 @@ def main():
         kb = kernel_bytes(wl_i, T_i, r["ids"])
         dominant = max((k for k in r["phases"] if not k.startswith("route")), key=lambda k: r["phases"][k])
         dur_s = r["phases"][dominant] * 1e-3
-        achieved = kb[dominant] / dur_s / 1e9
         step_s = r["ms"] * 1e-3 / args.steps
         tokens_s = world * T_i / step_s
         flops = 2.0 * r["ids"].size * 3 * wl_i.H * wl_i.I
