@@ -36,10 +36,8 @@ route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __r
   if (tid == 0) {
     s_bad = 0;
     // The status word describes the most recent call: route runs first.
-    if (status) {
-      status[0] = 0;
-      status[1] = 0;
-    }
+    if (status)
+      for (int i = 0; i < 8; ++i) status[i] = 0;  // error code, dropped slots, wait diagnostics
   }
   __syncthreads();
 

@@ -6,41 +6,58 @@
 // bitsandbytes PR #1984, Design: gated SiLU between the projections and the
 // weighted sum over the chosen experts.
 //
-// With few routed rows per expert every packed byte is read once, and the
-// cost is the integer work of decoding (B200 issues the byte-permute /
-// logic / shift ops at half the fp32 rate), so the kernel is organised to
-// spend nothing else on the integer pipe and to keep every SM busy to the end:
-//  * warps take work items from one atomic counter: first gate_up items
-//    (one expert, 16 gate rows + the same 16 up rows, all of K), then down
-//    items (one expert, 16 output rows, one K slice). A down item waits,
-//    bounded, until every gate_up item of its expert has stored h;
-//  * a lane owns 32 contiguous packed bytes (64 weights) of two rows per
-//    256-wide K chunk, copied ahead into a private shared-memory slot with
-//    cp.async; it decodes them through the block's 16-entry bf16 table straight
-//    into the A fragment of mma.sync m16n8k16 (bf16 in, fp32 accumulate), with
-//    the K order permuted so that fragment columns are the lane's own weights;
-//  * down items add gate * output into an fp32 accumulator; the last item to
-//    finish a 16-row slice of the output converts that slice to bf16.
+// With few routed rows per expert every packed byte is read once and the
+// layer streams the packed weights from HBM. What limits such a stream is how
+// many bytes each SM keeps in flight, so the kernel is a pipeline with one
+// persistent CTA per SM:
+//  * a producer warp takes work items from one atomic counter and fetches, for
+//    each 256-wide K chunk of an item, the packed codes of the item's 256
+//    weight rows (two TMA tiles, 128B-swizzled), the chunk of each routed
+//    activation row (four-row TMA gathers from x, or TMA tiles of h) and the
+//    block scales into a shared-memory stage (four stages of 44 KB);
+//  * eight consumer warps take 32 weight rows each from a stage, decode the
+//    codes through a 256-entry byte table (conflict-free shared loads) into
+//    the A fragments of mma.sync m16n8k16 (bf16 in, fp32 accumulate), with the
+//    activations of the stage as B, and release the stage;
+//  * gate_up items (one expert, 128 gate rows and the matching 128 up rows,
+//    all of K) end in the SwiGLU and store bf16 h; down items (one expert,
+//    256 output rows, a 2048-wide K slice) wait, bounded, until every gate_up
+//    item of their expert has stored h, and end in gate-weighted fp32 atomics
+//    into the accumulator; the last warp to finish a 256-row output slice
+//    converts it to bf16.
+// Every wait is bounded; a wait that gives up records E4B_ERR_DEVICE_TIMEOUT
+// and all warps stop.
 #include "common.cuh"
 #include "launch.h"
+#include "sm100.cuh"
+#include "tmap.h"
 
 namespace e4b {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 256;              // K per step of a warp
-constexpr int kSlotBytesPerLane = 128;   // 2 rows x (2 matrices) x 32 B
-constexpr int kSlots = 2;
-constexpr int kMaxNT = 2;                // token chunks of 8 per pass (16 rows)
-constexpr int kGroup = 8 * kMaxNT;
-constexpr uint32_t kPolls = 1u << 24;
+using namespace sm100;
+
+constexpr int kConsumers = 16;                   // consumer warps
+constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
+constexpr int kChunk = 256;                      // K per stage
+constexpr int kStages = 4;
+constexpr int kRows = 256;                       // weight rows per stage (16 per consumer)
+constexpr int kMaxTok = 16;                      // routed rows per pass (two chunks of 8)
+// Byte-to-weight-pair table, 256 entries of 128 bytes each, replicated so
+// that the lanes' lookups never conflict. NF4: two fp32 levels per entry, one
+// copy per half-warp lane (entry v of lane l at v * 128 + 8 * (l % 16)).
+// MXFP4: two bf16 values per entry, one copy per lane (v * 128 + 4 * l).
+constexpr int kLutBytes = 256 * 128;
+constexpr uint64_t kStageWaitNs = 100000000;  // 100 ms for a stage; 16x that for h of an expert
+constexpr uint64_t kDrainNs = 1000000000;     // the copies still landing at exit
+constexpr int kKSplit = 2048;                    // K slice of a down item
 
 // sync words (int32) at the start of the layer's sync area:
 //   work item counter, zeroing-chunk counter, zeroed-chunk count, then
-//   done_A[E] (gate_up items finished per active expert) and arrive[H/16]
-//   (down items finished per 16-row output slice). Cleared by the routing
-//   kernel before every layer call.
+//   done_A[E] (finished gate_up passes per active expert, one count per
+//   consumer warp) and arrive[] (finished down passes per 256-row output
+//   slice, one count per consumer warp). Cleared by the routing kernel before
+//   every layer call.
 enum : int { kWork = 0, kZeroWork = 1, kZeroDone = 2, kDoneA = 3 };
 constexpr int64_t kZeroChunk = 16384;  // floats per zeroing chunk
 
@@ -53,28 +70,42 @@ E4B_DEV void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-E4B_DEV void cp16(uint32_t dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+// 4-byte copy; the first src_bytes bytes come from src, the rest are zero.
+E4B_DEV void cp4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
 }
-E4B_DEV void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-E4B_DEV void cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-E4B_DEV void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+// Arrives on the mbarrier once every cp.async this thread issued so far has
+// landed (the barrier's expected count includes this arrival).
+E4B_DEV void cp_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+E4B_DEV void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-E4B_DEV uint4 lds128(uint32_t addr) {
-  uint4 r;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "r"(addr));
-  return r;
+E4B_DEV uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
 }
 
-E4B_DEV uint4 ld_cg_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
+// Bounded waits of this kernel: they give up after `ns` nanoseconds (at once
+// when ns == 0, the test flag) or when *abort becomes nonzero.
+E4B_DEV bool wait_phase(uint64_t* bar, uint32_t parity, uint64_t ns, const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (ns == 0 || (abort && *abort) || now_ns() - t0 > ns) return false;
+    __nanosleep(32);
+  }
+}
+
+// Records the first wait that gave up: status[2] = site, [3] = CTA, [4] = stage.
+E4B_DEV void record_wait_site(int32_t* status, int site, int64_t stage) {
+  if (status && atomicCAS(status + 2, 0, site) == 0) {
+    status[3] = int32_t(blockIdx.x);
+    status[4] = int32_t(stage);
+  }
 }
 
 E4B_DEV int ld_acquire(const int* p) {
@@ -83,20 +114,41 @@ E4B_DEV int ld_acquire(const int* p) {
   return v;
 }
 
-// Bounded wait until *p >= target; false if it gave up. limit == 0 (the
-// test flag) gives up at once, so the error path can be exercised.
-E4B_DEV bool wait_geq(const int* p, int target, uint32_t limit) {
-  if (limit == 0) return false;
-  uint32_t polls = 0;
+// Bounded wait until *p >= target (same rules as wait_phase).
+E4B_DEV bool wait_geq(const int* p, int target, uint64_t ns, const volatile int* abort) {
+  if (ld_acquire(p) >= target) return true;
+  const uint64_t t0 = now_ns();
   while (ld_acquire(p) < target) {
-    if (++polls > limit) return false;
+    if (ns == 0 || *abort || now_ns() - t0 > ns) return false;
     __nanosleep(128);
   }
   return true;
 }
 
+E4B_DEV uint32_t lds32(uint32_t addr) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+  return r;
+}
+E4B_DEV uint4 lds128(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+  return r;
+}
+
+// TMA descriptors of the operands (see launch_smallm_layer).
+struct Maps {
+  CUtensorMap gu_codes;   // [E*2I rows, H/2 bytes], box 128 x 128, 128B swizzle
+  CUtensorMap dn_codes;   // [E*H rows, I/2 bytes], box 128 x 128, 128B swizzle
+  CUtensorMap x;          // [T rows, H] bf16, box 32 x 1 (four-row gathers)
+  CUtensorMap h;          // [T*top_k rows, I] bf16, box 32 x 16
+  CUtensorMap gu_scales;  // NF4 absmax [E*2I rows, H/64*4 bytes], box 16 x 128 (when gu_scales_tma)
+  CUtensorMap dn_scales;  // NF4 absmax [E*H rows, I/64*4 bytes], box 16 x 128 (when dn_scales_tma)
+};
+
 struct Params {
   int E, H, I, top_k;
+  int gu_scales_tma, dn_scales_tma;  // NF4 scale rows 16-byte aligned: fetch them by TMA
   int64_t T;
   const uint8_t* gu_codes;
   const uint8_t* gu_scales;
@@ -109,164 +161,508 @@ struct Params {
   uint16_t* h;       // [R, I] bf16, expert-ordered rows
   float* acc;        // [T, H] fp32
   uint16_t* y;       // [T, H] bf16
-  int32_t* sync;     // work, zero_done, done_A[E], arrive[H/16]
+  int32_t* sync;     // see the sync words above
   int32_t* status;
-  int ksplit;        // K slice of a down item (multiple of 256)
   uint32_t flags;
 };
 
-// Scale words of one row for the chunk: NF4 = the absmax of the lane's
-// 64-weight block (bits of a float); MXFP4 = its two e8m0 bytes.
+// What a stage holds (written by the producer before it releases the stage).
+struct StageInfo {
+  int kind;    // 0 gate_up, 1 down, -1 no more work
+  int ai;      // index of the expert among the active ones
+  int e;       // expert
+  int mt;      // row block: 128 gate/up outputs (gate_up) or 256 outputs (down)
+  int kc;      // first weight of the chunk along K
+  int last;    // last chunk of the pass: the consumers finish the pass
+  int p0;      // first routed row of the pass
+  int ntok;    // routed rows in the pass (1..16)
+};
+
+// How a block's scale is applied. NF4 (false): each weight is decoded to
+// bf16(fp32(level * absmax)) before the MMA, the decoded value every path of
+// the library and the oracle use. MXFP4 (true): the table holds the exact
+// e2m1 values and the power-of-two scale multiplies the block's fp32 MMA
+// result, which is the same product exactly.
+constexpr bool kNf4ScaleAfter = false;
 template <int FMT>
-E4B_DEV uint32_t load_scale(const uint8_t* srow, int kl, int K) {
-  if (kl >= K) return 0u;
-  if constexpr (FMT == E4B_FMT_NF4) {
-    return __float_as_uint(__ldg(reinterpret_cast<const float*>(srow) + (kl >> 6)));
+constexpr bool kScaleAfter = FMT == E4B_FMT_MXFP4 || kNf4ScaleAfter;
+
+// Fills the byte table (whole CTA). The earlier weight of a byte is the high
+// nibble for NF4 and the low nibble for MXFP4; it goes first in the entry.
+template <int FMT>
+E4B_DEV void build_lut(uint8_t* lut) {
+  if constexpr (!kScaleAfter<FMT>) {
+    for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x)
+      reinterpret_cast<float2*>(lut)[i] = make_float2(nf4_level(i >> 8), nf4_level((i >> 4) & 15));
   } else {
-    const uint32_t b0 = __ldg(srow + (kl >> 5));
-    const uint32_t b1 = (kl + 32 < K) ? uint32_t(__ldg(srow + (kl >> 5) + 1)) : 0u;
-    return b0 | (b1 << 8);
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+      const int v = i >> 5, lo = v & 15, hi = v >> 4;
+      float a = (lo & 8) ? -e2m1_magnitude(lo & 7) : e2m1_magnitude(lo & 7);
+      float b = (hi & 8) ? -e2m1_magnitude(hi & 7) : e2m1_magnitude(hi & 7);
+      if (FMT == E4B_FMT_NF4) {
+        a = nf4_level(hi);
+        b = nf4_level(lo);
+      }
+      reinterpret_cast<uint32_t*>(lut)[i] = pack_bf16x2(a, b);
+    }
   }
 }
 
-// One warp-item over the K range [k0, k1) of one weight matrix (row
-// pointers crow/srow for rows g and g+8 of the 16-row tile) and NT chunks of
-// 8 token rows (brow: activation row of this lane's token in each chunk, or
-// null). Accumulates into acc[j][4].
-template <int FMT, int NT, bool COHERENT_B>
-E4B_DEV void run_item(const uint8_t* const (&crow)[2], const uint8_t* const (&srow)[2],
-                      const uint16_t* const (&brow)[kMaxNT], int k0, int k1, int K, uint32_t slot_base,
-                      float (&acc)[kMaxNT][4]) {
-  const int lane = threadIdx.x & 31;
-  const int c = lane & 3;
-  const int kend = min(K, k1);
-  const int nchunks = (k1 - k0 + kChunk - 1) / kChunk;
-
-  auto issue = [&](int ci, int slot) {
-    const int kl = k0 + ci * kChunk + c * 64;
-    const int left = kend - kl;  // weights this lane may copy
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int piece = 0; piece < 2; ++piece) {
-        const uint32_t dst = slot_base + uint32_t(slot * kSlotBytesPerLane * 32) +
-                             uint32_t((h * 2 + piece) * 512 + lane * 16);
-        const bool ok = left >= 32 * (piece + 1);
-        cp16(dst, ok ? (const void*)(crow[h] + (kl >> 1) + piece * 16) : (const void*)crow[h],
-             ok ? 16u : 0u);
-      }
-    cp_commit();
-  };
-  auto load_b = [&](int koff, uint4 (&b)[NT]) {
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      b[j] = make_uint4(0, 0, 0, 0);
-      if (brow[j] && koff < kend) {
-        if constexpr (COHERENT_B) b[j] = ld_cg_v4(brow[j] + koff);
-        else b[j] = __ldg(reinterpret_cast<const uint4*>(brow[j] + koff));
-      }
-    }
-  };
-
-  // two accumulator sets (the two MMA sub-steps of a word) shorten the
-  // dependency chains through the tensor pipe
-  float acc2[NT][4];
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc2[j][q] = 0.f;
-
-  issue(0, 0);
-  uint32_t sc_next0 = load_scale<FMT>(srow[0], k0 + c * 64, kend);
-  uint32_t sc_next1 = load_scale<FMT>(srow[1], k0 + c * 64, kend);
-  uint4 bcur[NT];
-  load_b(k0 + c * 64, bcur);
-
-  for (int ci = 0; ci < nchunks; ++ci) {
-    const int slot = ci & 1;
-    const int kl = k0 + ci * kChunk + c * 64;
-    const uint32_t sc0 = sc_next0, sc1 = sc_next1;
-    if (ci + 1 < nchunks) {
-      issue(ci + 1, slot ^ 1);
-      sc_next0 = load_scale<FMT>(srow[0], kl + kChunk, kend);
-      sc_next1 = load_scale<FMT>(srow[1], kl + kChunk, kend);
-      cp_wait1();
-    } else {
-      cp_wait0();
-    }
-    const uint32_t sbase = slot_base + uint32_t(slot * kSlotBytesPerLane * 32) + uint32_t(lane * 16);
-    Lut L0, L1;
-    if constexpr (FMT == E4B_FMT_NF4) {  // one 64-weight block per row and lane
-      lut_nf4(L0, __uint_as_float(sc0));
-      lut_nf4(L1, __uint_as_float(sc1));
-    }
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint4 w0 = lds128(sbase + uint32_t((0 * 2 + half) * 512));
-      const uint4 w1 = lds128(sbase + uint32_t((1 * 2 + half) * 512));
-      if constexpr (FMT == E4B_FMT_MXFP4) {  // one 32-weight block per half
-        lut_mxfp4(L0, (sc0 >> (8 * half)) & 0xFFu);
-        lut_mxfp4(L1, (sc1 >> (8 * half)) & 0xFFu);
-      }
-      const uint32_t r0w[4] = {w0.x, w0.y, w0.z, w0.w};
-      const uint32_t r1w[4] = {w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-      for (int wi = 0; wi < 4; ++wi) {
-        // prefetch the next word's activations (next chunk's first word at the end)
-        uint4 bnext[NT];
-        const int knext = (half == 1 && wi == 3) ? kl + kChunk : kl + half * 32 + wi * 8 + 8;
-        const bool more = !(half == 1 && wi == 3) || (ci + 1 < nchunks);
-        if (more) load_b(knext, bnext);
-        uint32_t o0[4], o1[4];
-        lut_decode8<FMT>(L0, r0w[wi], o0);
-        lut_decode8<FMT>(L1, r1w[wi], o1);
-        // sub-step 0: weights 0..3 of the word, sub-step 1: weights 4..7;
-        // fragment registers {row g | row g+8} x {cols 2c,2c+1 | 2c+8,2c+9}
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          mma16816(acc[j], o0[0], o1[0], o0[1], o1[1], bcur[j].x, bcur[j].y);
-          mma16816(acc2[j], o0[2], o1[2], o0[3], o1[3], bcur[j].z, bcur[j].w);
-        }
-        if (more) {
-#pragma unroll
-          for (int j = 0; j < NT; ++j) bcur[j] = bnext[j];
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[j][q] += acc2[j][q];
-}
-
-// run_item with the token-chunk count as a compile-time constant
-template <int FMT, bool COHERENT_B>
-E4B_DEV void run_item_nt(int nt, const uint8_t* const (&crow)[2], const uint8_t* const (&srow)[2],
-                         const uint16_t* const (&brow)[kMaxNT], int k0, int k1, int K, uint32_t slot_base,
-                         float (&acc)[kMaxNT][4]) {
-  if (nt == 1) run_item<FMT, 1, COHERENT_B>(crow, srow, brow, k0, k1, K, slot_base, acc);
-  else run_item<FMT, 2, COHERENT_B>(crow, srow, brow, k0, k1, K, slot_base, acc);
+// 8 codes (one 32-bit word, weights in byte order) -> 4 bf16x2 weight pairs,
+// one byte extract and one conflict-free shared load per pair.
+// NF4 pair: both fp32 levels of the entry at `addr` times the absmax (one
+// packed f32x2 multiply, round-to-nearest per element), rounded to bf16x2.
+E4B_DEV uint32_t scaled_pair(uint32_t addr, uint64_t absmax2) {
+  uint32_t r;
+  asm("{\n\t.reg .b64 l, p;\n\t.reg .f32 a, b;\n\t"
+      "ld.shared.b64 l, [%1];\n\t"
+      "mul.rn.f32x2 p, l, %2;\n\t"
+      "mov.b64 {a, b}, p;\n\t"
+      "cvt.rn.bf16x2.f32 %0, b, a;\n\t}"
+      : "=r"(r)
+      : "r"(addr), "l"(absmax2));
+  return r;
 }
 
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 2) smallm_layer_kernel(Params p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  __shared__ int32_t s_act[1024];
-  __shared__ int32_t s_n;
-  __shared__ int32_t s_wscr[kWarps + 1];
+E4B_DEV void lut_lookup8(uint32_t lut_lane, uint32_t w, uint64_t absmax2, uint32_t* o) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t a = lut_lane + (prmt(w, 0u, 0x4440u | uint32_t(j)) << 7);
+    if constexpr (!kScaleAfter<FMT>) o[j] = scaled_pair(a, absmax2);
+    else o[j] = lds32(a);
+  }
+}
+
+// Scale of block b of a stage row (staged bytes at `slot`): NF4 the absmax,
+// MXFP4 2^(s-127) with byte 0 = 2^-127 and byte 255 = NaN. `off` is the row's
+// byte offset inside its staged MXFP4 scale words.
+template <int FMT>
+E4B_DEV float stage_scale(uint32_t slot, int b, uint32_t off) {
+  if constexpr (FMT == E4B_FMT_NF4) {
+    return __uint_as_float(lds32(slot + uint32_t(4 * b)));
+  } else {
+    uint32_t e;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(slot + off + uint32_t(b)));
+    return (e - 1u < 254u) ? __uint_as_float(e << 23) : e8m0_to_f32(e);
+  }
+}
+
+// Stage layout (1024-byte aligned, as the 128B swizzle needs):
+//   codes   256 rows x 128 bytes, 16-byte chunk q of row r at chunk q ^ (r % 8)
+//   x       8 slabs of 32 K values: 16 routed rows x 64 bytes each
+//   scales  256 rows x 16 bytes
+constexpr int kCodeOff = 0;
+constexpr int kXOff = kRows * 128;
+constexpr int kSOff = kXOff + 8 * kMaxTok * 64;
+constexpr int kStageBytesMax = kSOff + kRows * 16;
+static_assert(kStageBytesMax % 1024 == 0, "stages stay 1024-byte aligned");
+constexpr int kSmemBytes = 1024 + kLutBytes + kStages * kStageBytesMax + 256;  // + alignment, barriers, stage info
+
+// Work items: gate_up items ai * MTA + mt (mt: a block of 128 gate rows and
+// the matching 128 up rows), then down items nA + (ai * NKS + ks) * MTB + mt
+// (mt: a block of 256 output rows, ks: a 2048-wide K slice). Each item runs
+// one pass per group of up to 16 routed rows of its expert.
+struct Work {
+  int MTA, MTB, NKS, nA, nB;
+};
+
+// Producer warp: fills the stages, chunk by chunk, item after item, then
+// posts one stage with kind -1. Returns early, with the abort flag set, if a
+// bounded wait gives up.
+template <int FMT>
+E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int32_t* s_act, uint8_t* stages,
+                     uint64_t* full, uint64_t* empty, StageInfo* info, volatile int* s_abort, int nzero,
+                     uint64_t limit) {
   const int lane = threadIdx.x & 31;
-  const int wid = threadIdx.x >> 5;
+  const int H = p.H, I = p.I;
+  int64_t i = 0;  // stages posted
+  bool aborted = false;
+  auto give_up = [&]() {
+    if (lane == 0) {
+      *s_abort = 1;
+      record_status(p.status, E4B_ERR_DEVICE_TIMEOUT);
+    }
+    aborted = true;
+  };
+  // waits (bounded) until stage s of post i is free and announces `tx` bytes
+  // of TMA copies to it; false if it gave up
+  auto acquire_stage = [&](int s, uint32_t tx) -> bool {
+    int ok = 1;
+    if (lane == 0) {
+      ok = wait_phase(&empty[s], (uint32_t(i / kStages) & 1u) ^ 1u, limit, s_abort);
+      if (!ok) record_wait_site(p.status, 1, i);
+      if (ok && tx) mbar_expect_tx(&full[s], tx);
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+
+  while (!aborted) {
+    int item = 0;
+    if (lane == 0) item = atomicAdd(p.sync + kWork, 1);
+    item = __shfl_sync(0xffffffffu, item, 0);
+    if (item >= W.nA + W.nB) break;
+    const bool down = item >= W.nA;
+    int ai, mt, ks = 0;
+    if (!down) {
+      ai = item / W.MTA;
+      mt = item % W.MTA;
+    } else {
+      const int b = item - W.nA;
+      ai = b / (W.MTB * W.NKS);
+      const int r = b % (W.MTB * W.NKS);
+      ks = r / W.MTB;
+      mt = r % W.MTB;
+    }
+    const int e = s_act[ai];
+    const int64_t p0 = p.offsets[e], p1 = p.offsets[e + 1];
+    const int ngroups = int((p1 - p0 + kMaxTok - 1) / kMaxTok);
+    if (down) {
+      // h of this expert complete (every gate_up pass of it, one count per
+      // consumer warp) and the accumulator cleared
+      int ok = 1;
+      if (lane == 0)
+      {
+        ok = wait_geq(p.sync + kDoneA + ai, W.MTA * ngroups * kConsumers, 16 * limit, s_abort);
+        if (!ok) record_wait_site(p.status, 2, i);
+        ok = ok && wait_geq(p.sync + kZeroDone, nzero, 16 * limit, s_abort);
+        if (!ok) record_wait_site(p.status, 3, i);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        give_up();
+        break;
+      }
+      ld_acquire(p.sync + kDoneA + ai);  // every lane reads h after the acquire
+      // h was written through the generic proxy; the TMA reads it through the async one
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    const int K = down ? I : H;
+    const int k0 = down ? ks * kKSplit : 0;
+    const int k1 = down ? min(I, k0 + kKSplit) : H;
+    const uint8_t* scales = down ? p.dn_scales : p.gu_scales;
+    const int64_t sstride = FMT == E4B_FMT_NF4 ? (K / 64) * 4 : K / 32;  // scale bytes per row
+    const int64_t sbytes = int64_t(p.E) * (down ? H : 2 * I) * sstride;
+    // global weight row of stage row r, or -1 past the matrix
+    auto wrow = [&](int r) -> int64_t {
+      if (down) {
+        const int n = mt * 256 + r;
+        return n < H ? int64_t(e) * H + n : -1;
+      }
+      const int n = mt * 128 + (r & 127);
+      return n < I ? int64_t(e) * 2 * I + int64_t(r >> 7) * I + n : -1;
+    };
+
+    const CUtensorMap* cmap = down ? &maps.dn_codes : &maps.gu_codes;
+    const bool scales_tma = FMT == E4B_FMT_NF4 && (down ? p.dn_scales_tma : p.gu_scales_tma);
+    const CUtensorMap* smap = down ? &maps.dn_scales : &maps.gu_scales;
+    // first global weight row of the stage's two 128-row halves
+    const int64_t row0 = down ? int64_t(e) * H + int64_t(mt) * 256 : int64_t(e) * 2 * I + int64_t(mt) * 128;
+    const int64_t row1 = down ? row0 + 128 : row0 + I;
+    const uint32_t tx = uint32_t(kRows * 128 + 8 * kMaxTok * 64 + (scales_tma ? kRows * 16 : 0));
+
+    for (int64_t tg = p0; tg < p1 && !aborted; tg += kMaxTok) {
+      const int ntok = int(min(p1 - tg, int64_t(kMaxTok)));
+      // gate_up: the x row of each of the pass's routed rows (rows past the
+      // pass repeat its first row; their products are never stored)
+      int32_t xrow = 0;
+      if (!down) xrow = p.perm[tg + (lane < ntok ? lane : 0)] / p.top_k;
+      int32_t gr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) gr[u] = __shfl_sync(0xffffffffu, xrow, 4 * (lane & 3) + u);
+      for (int kc = k0; kc < k1; kc += kChunk, ++i) {
+        const int s = int(i % kStages);
+        if (!acquire_stage(s, tx)) {
+          give_up();
+          break;
+        }
+        uint8_t* st = stages + s * kStageBytesMax;
+        if (lane == 0) {
+          tma_load_2d(st + kCodeOff, cmap, &full[s], kc / 2, int32_t(row0));
+          tma_load_2d(st + kCodeOff + 128 * 128, cmap, &full[s], kc / 2, int32_t(row1));
+          if (scales_tma) {
+            tma_load_2d(st + kSOff, smap, &full[s], (kc / 64) * 4, int32_t(row0));
+            tma_load_2d(st + kSOff + 128 * 16, smap, &full[s], (kc / 64) * 4, int32_t(row1));
+          }
+        }
+        if (down) {
+          // h rows tg.. are contiguous: one 16-row tile per 32-wide slab
+          if (lane < 8) tma_load_2d(st + kXOff + lane * kMaxTok * 64, &maps.h, &full[s], kc + 32 * lane, int32_t(tg));
+        } else {
+          // lane l gathers routed rows 4(l%4)..+3 of slab l/4
+          const int slab = lane >> 2;
+          tma_gather4_2d(st + kXOff + slab * kMaxTok * 64 + (lane & 3) * 4 * 64, &maps.x, &full[s], kc + 32 * slab,
+                         gr[0], gr[1], gr[2], gr[3]);
+        }
+        if (!scales_tma) {
+          // scales by cp.async, 16 bytes per row. NF4: the chunk's 4 absmax
+          // words. MXFP4: the 3 aligned words that hold the chunk's 8 bytes.
+          const uint32_t sbase = smem_u32(st + kSOff);
+          for (int m = 0; m < kRows / 8; ++m) {
+            const int q = lane + 32 * m, r = q >> 2, w = q & 3;
+            const int64_t grow = wrow(r);
+            const uint32_t dst = sbase + uint32_t(r * 16 + 4 * w);
+            if constexpr (FMT == E4B_FMT_NF4) {
+              const bool v = grow >= 0 && kc + 64 * w < k1;
+              cp4(dst, v ? (const void*)(scales + grow * sstride + (kc / 64 + w) * 4) : (const void*)scales,
+                  v ? 4u : 0u);
+            } else {
+              const int64_t a = ((grow * sstride + kc / 32) & ~int64_t(3)) + 4 * w;
+              const int64_t left = sbytes - a;
+              const bool v = grow >= 0 && w < 3 && left > 0;
+              cp4(dst, v ? (const void*)(scales + a) : (const void*)scales, v ? uint32_t(left < 4 ? left : 4) : 0u);
+            }
+          }
+        }
+        if (lane == 0) {
+          StageInfo& f = info[s];
+          f.kind = down ? 1 : 0;
+          f.ai = ai;
+          f.e = e;
+          f.mt = mt;
+          f.kc = kc;
+          f.last = kc + kChunk >= k1;
+          f.p0 = int(tg);
+          f.ntok = ntok;
+        }
+        cp_arrive_noinc(&full[s]);
+        if (lane == 0) mbar_arrive(&full[s]);
+      }
+    }
+  }
+  // the end-of-work stage
+  if (!aborted) {
+    const int s = int(i % kStages);
+    if (acquire_stage(s, 0u)) {
+      if (lane == 0) info[s].kind = -1;
+      cp_arrive_noinc(&full[s]);
+      if (lane == 0) mbar_arrive(&full[s]);
+      ++i;  // a post like any other: the drain below must not alias its slot
+    } else {
+      give_up();
+    }
+  }
+  cp_wait_all();  // no cp.async may land after the CTA has exited
+  // ... nor a TMA copy: wait (bounded) for the stages posted last
+  if (lane == 0)
+    for (int64_t q = i > kStages ? i - kStages : 0; q < i; ++q)
+      if (!wait_phase(&full[q % kStages], uint32_t(q / kStages) & 1u, kDrainNs, nullptr))
+        record_wait_site(p.status, 5, q);
+}
+
+// One stage for one consumer warp: one 16-row tile (MMA rows g from stage
+// row rA + g, rows g + 8 from stage row rB + g) times NT chunks of 8 routed
+// rows, accumulated into acc.
+// K order: the stage's 256 K values are 8 chunks of 32 (16 code bytes); in
+// every chunk, lane c of a quad takes the 8 consecutive weights 8c..8c+7
+// (code word c), so every mma k16 step stays inside one 32-wide chunk and
+// hence inside one scale block of each row.
+template <int FMT, int NT>
+E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, int rB, uint32_t soffA,
+                           uint32_t soffB, uint32_t lut_lane, float (&acc)[2][4]) {
+  constexpr bool SA = kScaleAfter<FMT>;
+  constexpr int BLK = FMT == E4B_FMT_NF4 ? 64 : 32;  // weights per scale block
+  constexpr int NB = kChunk / BLK;                     // blocks per stage
+  constexpr int CPB = BLK / 32;                        // 32-wide chunks per block
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;
+  const int c = lane & 3;
+  const uint32_t cA = st + uint32_t(kCodeOff + (rA + g) * 128 + 4 * c);  // both rows are g modulo 8
+  const uint32_t cB = st + uint32_t(kCodeOff + (rB + g) * 128 + 4 * c);
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const bool live = f.kc + BLK * b < kend;  // blocks past K: codes are zero, scale 0
+    const float sA = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rA + g) * 16), b, soffA) : 0.f;
+    const float sB = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rB + g) * 16), b, soffB) : 0.f;
+    const uint64_t sA2 = (uint64_t(__float_as_uint(sA)) << 32) | __float_as_uint(sA);
+    const uint64_t sB2 = (uint64_t(__float_as_uint(sB)) << 32) | __float_as_uint(sB);
+    float P[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) P[j][q] = 0.f;
+#pragma unroll
+    for (int it = 0; it < CPB; ++it) {
+      const int ch = CPB * b + it;  // 32-wide chunk of the stage
+      // activations: 8 values of this lane's token in each chunk of 8 routed rows
+      uint4 xv[NT];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const int tok = 8 * j + g;
+        xv[j] = tok < f.ntok ? lds128(st + uint32_t(kXOff + ch * kMaxTok * 64 + tok * 64 + 16 * c))
+                             : make_uint4(0, 0, 0, 0);
+      }
+      const uint32_t sw = uint32_t((ch ^ g) << 4);  // the 128B swizzle of chunk ch in row g (mod 8)
+      uint32_t dA[4], dB[4];
+      lut_lookup8<FMT>(lut_lane, lds32(cA + sw), sA2, dA);
+      lut_lookup8<FMT>(lut_lane, lds32(cB + sw), sB2, dB);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        float(&D)[4] = SA ? P[j] : acc[j];
+        // fragment registers {row g | row g+8} x {pair 0,2 | pair 1,3}
+        mma16816(D, dA[0], dB[0], dA[1], dB[1], xv[j].x, xv[j].y);
+        mma16816(D, dA[2], dB[2], dA[3], dB[3], xv[j].z, xv[j].w);
+      }
+    }
+    if constexpr (SA) {
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        acc[j][0] = fmaf(sA, P[j][0], acc[j][0]);
+        acc[j][1] = fmaf(sA, P[j][1], acc[j][1]);
+        acc[j][2] = fmaf(sB, P[j][2], acc[j][2]);
+        acc[j][3] = fmaf(sB, P[j][3], acc[j][3]);
+      }
+    }
+  }
+}
+
+// Consumer warps: take the stages in order until the kind -1 stage, finishing
+// each pass with its epilogue. Warp w takes, per stage, gate rows 8w..8w+7
+// (MMA rows g) and the matching up rows 128+8w.. (MMA rows g+8) for gate_up,
+// so gate and up of an output sit in the same lane; output rows 16w..16w+15
+// for down.
+template <int FMT>
+E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
+                     const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, int arrive_target,
+                     uint64_t limit) {
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;  // 0 .. kConsumers-1
   const int g = lane >> 2;
   const int c = lane & 3;
   const int H = p.H, I = p.I;
-  const uint32_t limit = (p.flags & E4B_FLAG_TEST_TIMEOUT) ? 0u : kPolls;
+  int32_t* done_A = p.sync + kDoneA;
+  int32_t* arrive = p.sync + kDoneA + p.E;
+  float acc[2][4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+
+  for (int64_t i = 0;; ++i) {
+    const int s = int(i % kStages);
+    if (!wait_phase(&full[s], uint32_t(i / kStages) & 1u, limit, s_abort)) {
+      if (!*s_abort) {
+        record_wait_site(p.status, 4, i);
+        *s_abort = 1;
+        record_status(p.status, E4B_ERR_DEVICE_TIMEOUT);
+      }
+      break;
+    }
+    const StageInfo f = info[s];
+    if (f.kind < 0) break;
+    const bool down = f.kind == 1;
+    const int kend = down ? min(I, (f.kc / kKSplit + 1) * kKSplit) : H;
+    const uint32_t st = smem_u32(stages + s * kStageBytesMax);
+    const int rA = down ? 16 * w : 8 * w;
+    const int rB = down ? 16 * w + 8 : 128 + 8 * w;
+    // MXFP4: byte offset of each of the two rows' scales inside their staged words
+    uint32_t soffA = 0, soffB = 0;
+    if constexpr (FMT == E4B_FMT_MXFP4) {
+      const int64_t k32 = (down ? I : H) / 32;
+      auto grow = [&](int r) -> int64_t {
+        return down ? int64_t(f.e) * H + int64_t(f.mt) * 256 + r
+                    : int64_t(f.e) * 2 * I + int64_t(r >> 7) * I + int64_t(f.mt) * 128 + (r & 127);
+      };
+      soffA = uint32_t((grow(rA + g) * k32) & 3);
+      soffB = uint32_t((grow(rB + g) * k32) & 3);
+    }
+    if (f.ntok > 8) consume_stage<FMT, 2>(st, f, kend, rA, rB, soffA, soffB, lut_lane, acc);
+    else consume_stage<FMT, 1>(st, f, kend, rA, rB, soffA, soffB, lut_lane, acc);
+    mbar_arrive(&empty[s]);  // this lane's reads of the stage are done
+    if (!f.last) continue;
+
+    // ---------------------------------------------------- end of a pass
+    const int nt = f.ntok > 8 ? 2 : 1;
+    if (!down) {
+      // h[p][n] = bf16(silu(gate) * up): gate in fragment rows g (d0, d1),
+      // up in rows g + 8 (d2, d3), tokens 2c, 2c+1
+      const int n = f.mt * 128 + 8 * w + g;
+      for (int j = 0; j < nt; ++j)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int tok = 8 * j + 2 * c + q;
+          if (tok < f.ntok && n < I)
+            p.h[int64_t(f.p0 + tok) * I + n] = to_bf16_bits(silu_mul(acc[j][q], acc[j][q + 2]));
+        }
+      __threadfence();
+      // h is read next by TMA (the async proxy) in other CTAs
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) atomicAdd(done_A + f.ai, 1);
+    } else {
+      for (int j = 0; j < nt; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int tok = 8 * j + 2 * c + (q & 1);
+          const int n = f.mt * 256 + 16 * w + g + ((q & 2) ? 8 : 0);
+          if (tok >= f.ntok || n >= H) continue;
+          const int slot = p.perm[f.p0 + tok];
+          atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * acc[j][q]);
+        }
+      // the last warp to finish a pass over this 256-row output slice
+      // converts the slice to bf16
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = atomicAdd(arrive + f.mt, 1) == arrive_target - 1;
+      if (__shfl_sync(0xffffffffu, last, 0)) {
+        __threadfence();
+        const int n0 = f.mt * 256;
+        const int width = min(256, H - n0);  // a multiple of 32
+        for (int64_t q = lane; q < p.T * (width / 4); q += 32) {
+          const int64_t t = q / (width / 4);
+          const int part = int(q % (width / 4));
+          const float* src = p.acc + t * H + n0 + part * 4;
+          float4 v;
+          asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                       : "l"(src));
+          *reinterpret_cast<uint2*>(p.y + t * H + n0 + part * 4) =
+              make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ int32_t s_act[1024];
+  __shared__ int32_t s_n;
+  __shared__ int32_t s_wscr[kThreads / 32 + 1];
+  __shared__ int s_zc;
+  __shared__ int s_arrive_target;
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int H = p.H, I = p.I;
+  const uint64_t limit = (p.flags & E4B_FLAG_TEST_TIMEOUT) ? 0u : kStageWaitNs;
+  uint8_t* stages = smem + kLutBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytesMax);
+  uint64_t* empty = full + kStages;
+  StageInfo* info = reinterpret_cast<StageInfo*>(empty + kStages);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(info + kStages);
+
+  // The byte table (made visible by the barriers of the clearing loop below).
+  build_lut<FMT>(smem);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 33);                  // 32 producer lanes' copies + the stage info
+      mbar_init(&empty[s], kConsumers * 32);    // every consumer lane
+    }
+    *s_abort = 0;
+    mbar_init_fence();
+  }
 
   // Clear the fp32 accumulator in chunks handed out by a counter, so that
-  // waiting on the zeroed count only depends on CTAs that are running.
+  // waiting on the cleared count only depends on CTAs that are running.
   const int64_t nacc = p.T * int64_t(H);
   const int nzero = int((nacc + kZeroChunk - 1) / kZeroChunk);
-  __shared__ int s_zc;
   while (true) {
     if (threadIdx.x == 0) s_zc = atomicAdd(p.sync + kZeroWork, 1);
     __syncthreads();
@@ -289,152 +685,31 @@ __global__ void __launch_bounds__(kThreads, 2) smallm_layer_kernel(Params p) {
       p.y[i] = 0;
     return;
   }
-  const int MTA = I / 16;                  // gate_up items per expert
-  const int MTB = H / 16;                  // down row tiles
-  const int NKS = (I + p.ksplit - 1) / p.ksplit;
-  const int nA = nact * MTA;
-  const int nB = nact * MTB * NKS;
-  int32_t* done_A = p.sync + kDoneA;
-  int32_t* arrive = p.sync + kDoneA + p.E;
-  const uint32_t slot_base = uint32_t(__cvta_generic_to_shared(smem)) + uint32_t(wid * kSlots * kSlotBytesPerLane * 32);
-
-  while (true) {
-    int item = 0;
-    if (lane == 0) item = atomicAdd(p.sync + kWork, 1);
-    item = __shfl_sync(0xffffffffu, item, 0);
-    if (item >= nA + nB) break;
-
-    if (item < nA) {
-      // ------------------------------------------------ gate_up + SwiGLU
-      const int ai = item / MTA;
-      const int mt = item % MTA;
-      const int e = s_act[ai];
-      const int64_t p0 = p.offsets[e], p1 = p.offsets[e + 1];
-      const uint8_t* crow[2];
-      const uint8_t* srow[2];
-      const int64_t sstride = FMT == E4B_FMT_NF4 ? (H / 64) * 4 : (H / 32);
-      for (int64_t tg = p0; tg < p1; tg += kGroup) {
-        const int nt = int((min(p1 - tg, int64_t(kGroup)) + 7) / 8);
-        const uint16_t* brow[kMaxNT];
-#pragma unroll
-        for (int j = 0; j < kMaxNT; ++j) {
-          const int64_t pr = tg + 8 * j + g;
-          brow[j] = (j < nt && pr < p1) ? p.x + int64_t(p.perm[pr] / p.top_k) * H : nullptr;
-        }
-        float accg[kMaxNT][4], accu[kMaxNT][4];
-#pragma unroll
-        for (int j = 0; j < kMaxNT; ++j)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) accg[j][q] = accu[j][q] = 0.f;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int64_t row = int64_t(e) * 2 * I + mt * 16 + g + 8 * hh;
-          crow[hh] = p.gu_codes + row * (H / 2);
-          srow[hh] = p.gu_scales + row * sstride;
-        }
-        run_item_nt<FMT, false>(nt, crow, srow, brow, 0, H, H, slot_base, accg);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int64_t row = int64_t(e) * 2 * I + I + mt * 16 + g + 8 * hh;
-          crow[hh] = p.gu_codes + row * (H / 2);
-          srow[hh] = p.gu_scales + row * sstride;
-        }
-        run_item_nt<FMT, false>(nt, crow, srow, brow, 0, H, H, slot_base, accu);
-        // h[p][n] = bf16(silu(g) * u); fragment (row g / g+8, tokens 2c, 2c+1)
-#pragma unroll
-        for (int j = 0; j < kMaxNT; ++j) {
-          if (j >= nt) continue;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int64_t pr = tg + 8 * j + 2 * c + (q & 1);
-            if (pr < p1) {
-              const int n = mt * 16 + g + ((q & 2) ? 8 : 0);
-              p.h[pr * I + n] = to_bf16_bits(silu_mul(accg[j][q], accu[j][q]));
-            }
-          }
-        }
-      }
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) atomicAdd(done_A + ai, 1);
-    } else {
-      // ------------------------------------------------ down + combine
-      const int b = item - nA;
-      const int ai = b / (MTB * NKS);
-      const int rem = b % (MTB * NKS);
-      const int ks = rem / MTB;
-      const int mt = rem % MTB;
-      const int e = s_act[ai];
-      bool ok = true;
-      if (lane == 0) {
-        ok = wait_geq(done_A + ai, MTA, limit) && wait_geq(p.sync + kZeroDone, nzero, limit);
-        if (!ok) record_status(p.status, E4B_ERR_DEVICE_TIMEOUT);
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      __syncwarp();
-      if (ok) {
-        const int64_t p0 = p.offsets[e], p1 = p.offsets[e + 1];
-        const int k0 = ks * p.ksplit;
-        const int k1 = min(I, k0 + p.ksplit);
-        const uint8_t* crow[2];
-        const uint8_t* srow[2];
-        const int64_t sstride = FMT == E4B_FMT_NF4 ? (I / 64) * 4 : (I / 32);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int64_t row = int64_t(e) * H + mt * 16 + g + 8 * hh;
-          crow[hh] = p.dn_codes + row * (I / 2);
-          srow[hh] = p.dn_scales + row * sstride;
-        }
-        for (int64_t tg = p0; tg < p1; tg += kGroup) {
-          const int nt = int((min(p1 - tg, int64_t(kGroup)) + 7) / 8);
-          const uint16_t* brow[kMaxNT];
-#pragma unroll
-          for (int j = 0; j < kMaxNT; ++j) {
-            const int64_t pr = tg + 8 * j + g;
-            brow[j] = (j < nt && pr < p1) ? p.h + pr * I : nullptr;
-          }
-          float acc[kMaxNT][4];
-#pragma unroll
-          for (int j = 0; j < kMaxNT; ++j)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
-          run_item_nt<FMT, true>(nt, crow, srow, brow, k0, k1, I, slot_base, acc);
-#pragma unroll
-          for (int j = 0; j < kMaxNT; ++j) {
-            if (j >= nt) continue;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int64_t pr = tg + 8 * j + 2 * c + (q & 1);
-              if (pr < p1) {
-                const int slot = p.perm[pr];
-                const int n = mt * 16 + g + ((q & 2) ? 8 : 0);
-                atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * acc[j][q]);
-              }
-            }
-          }
-        }
-      }
-      // the last item of this 16-row output slice converts it to bf16
-      __threadfence();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = (atomicAdd(arrive + mt, 1) == nact * NKS - 1) ? 1 : 0;
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        for (int64_t i = lane; i < p.T * 4; i += 32) {
-          const int64_t t = i >> 2;
-          const int part = int(i & 3);
-          const float* src = p.acc + t * H + mt * 16 + part * 4;
-          float4 v;
-          asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
-                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                       : "l"(src));
-          *reinterpret_cast<uint2*>(p.y + t * H + mt * 16 + part * 4) =
-              make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-        }
-      }
+  Work W;
+  W.MTA = (I + 127) / 128;
+  W.MTB = (H + 255) / 256;
+  W.NKS = (I + kKSplit - 1) / kKSplit;
+  W.nA = nact * W.MTA;
+  W.nB = nact * W.MTB * W.NKS;
+  // passes over each 256-row output slice: every K slice of every routed-row
+  // group of every active expert, one count per consumer warp
+  if (wid == 0) {
+    int groups = 0;
+    for (int a = lane; a < nact; a += 32) {
+      const int e = s_act[a];
+      groups += int((p.offsets[e + 1] - p.offsets[e] + kMaxTok - 1) / kMaxTok);
     }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) groups += __shfl_xor_sync(0xffffffffu, groups, d);
+    if (lane == 0) s_arrive_target = groups * W.NKS * kConsumers;
+  }
+  __syncthreads();
+
+  if (wid == kConsumers) {
+    produce<FMT>(maps, p, W, s_act, stages, full, empty, info, s_abort, nzero, limit);
+  } else {
+    const uint32_t lut_lane = smem_u32(smem) + uint32_t(!kScaleAfter<FMT> ? 8 * (lane & 15) : 4 * lane);
+    consume<FMT>(p, stages, full, empty, info, s_abort, lut_lane, s_arrive_target, limit);
   }
 }
 
@@ -462,9 +737,30 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
   p.y = L.y;
   p.sync = L.sync;
   p.status = L.status;
-  p.ksplit = 2048;
   p.flags = L.flags;
-  const size_t smem = size_t(kWarps) * kSlots * kSlotBytesPerLane * 32;
+  const int64_t E = L.E, H = L.H, I = L.I;
+  Maps m;
+  bool ok = encode_2d(&m.gu_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.gu_codes, uint64_t(H / 2), uint64_t(E * 2 * I),
+                      uint64_t(H / 2), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&m.dn_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.dn_codes, uint64_t(I / 2), uint64_t(E * H),
+                      uint64_t(I / 2), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&m.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x, uint64_t(H), uint64_t(L.T), uint64_t(H) * 2, 32, 1,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) &&
+            encode_2d(&m.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.h, uint64_t(I), uint64_t(L.T * L.top_k),
+                      uint64_t(I) * 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+  // NF4 absmax rows by TMA when their byte stride is a multiple of 16
+  p.gu_scales_tma = L.fmt == E4B_FMT_NF4 && H % 256 == 0;
+  p.dn_scales_tma = L.fmt == E4B_FMT_NF4 && I % 256 == 0;
+  m.gu_scales = m.gu_codes;
+  m.dn_scales = m.dn_codes;
+  if (ok && p.gu_scales_tma)
+    ok = encode_2d(&m.gu_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.gu_scales, uint64_t(H / 64 * 4), uint64_t(E * 2 * I),
+                   uint64_t(H / 64 * 4), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (ok && p.dn_scales_tma)
+    ok = encode_2d(&m.dn_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.dn_scales, uint64_t(I / 64 * 4), uint64_t(E * H),
+                   uint64_t(I / 64 * 4), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
+  const size_t smem = size_t(kSmemBytes);
   static int configured = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -477,12 +773,11 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
     if (e2 != cudaSuccess) return e2;
     configured = dev;
   }
-  // persistent: every CTA resident at once (2 per SM)
-  const int grid = sms * 2;
+  // persistent: one CTA per SM, all resident at once
   if (L.fmt == E4B_FMT_NF4)
-    smallm_layer_kernel<E4B_FMT_NF4><<<grid, kThreads, smem, st>>>(p);
+    smallm_layer_kernel<E4B_FMT_NF4><<<sms, kThreads, smem, st>>>(m, p);
   else
-    smallm_layer_kernel<E4B_FMT_MXFP4><<<grid, kThreads, smem, st>>>(p);
+    smallm_layer_kernel<E4B_FMT_MXFP4><<<sms, kThreads, smem, st>>>(m, p);
   return cudaGetLastError();
 }
 
