@@ -40,7 +40,6 @@ using namespace sm100;
 constexpr int kConsumers = 16;                   // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;  // + the producer warp
 constexpr int kChunk = 256;                      // K per stage
-constexpr int kStages = 4;
 constexpr int kRows = 256;                       // weight rows per stage (16 per consumer)
 constexpr int kMaxTok = 16;                      // routed rows per pass (two chunks of 8)
 // Byte-to-weight-pair table, 256 entries of 128 bytes each, replicated so
@@ -142,13 +141,14 @@ struct Maps {
   CUtensorMap dn_codes;   // [E*H rows, I/2 bytes], box 128 x 128, 128B swizzle
   CUtensorMap x;          // [T rows, H] bf16, box 32 x 1 (four-row gathers)
   CUtensorMap h;          // [T*top_k rows, I] bf16, box 32 x 16
-  CUtensorMap gu_scales;  // NF4 absmax [E*2I rows, H/64*4 bytes], box 16 x 128 (when gu_scales_tma)
-  CUtensorMap dn_scales;  // NF4 absmax [E*H rows, I/64*4 bytes], box 16 x 128 (when dn_scales_tma)
+  // NF4 absmax rows [E*N rows, K/64*4 bytes], box 16 x 128 (when *_scales_tma)
+  CUtensorMap gu_scales;
+  CUtensorMap dn_scales;
 };
 
 struct Params {
   int E, H, I, top_k;
-  int gu_scales_tma, dn_scales_tma;  // NF4 scale rows 16-byte aligned: fetch them by TMA
+  int gu_scales_tma, dn_scales_tma;  // NF4: fetch the absmax rows by TMA (else cp.async)
   int64_t T;
   const uint8_t* gu_codes;
   const uint8_t* gu_scales;
@@ -234,18 +234,40 @@ E4B_DEV void lut_lookup8(uint32_t lut_lane, uint32_t w, uint64_t absmax2, uint32
   }
 }
 
-// Scale of block b of a stage row (staged bytes at `slot`): NF4 the absmax,
-// MXFP4 2^(s-127) with byte 0 = 2^-127 and byte 255 = NaN. `off` is the row's
-// byte offset inside its staged MXFP4 scale words.
+// Scale of block b of a row in a stage. NF4: the absmax staged at `slot`.
+// MXFP4: 2^(s-127) of byte b of `mx` (the row's 8 scale bytes of the chunk),
+// with byte 0 = 2^-127 and byte 255 = NaN.
 template <int FMT>
-E4B_DEV float stage_scale(uint32_t slot, int b, uint32_t off) {
+E4B_DEV float stage_scale(uint32_t slot, int b, uint64_t mx) {
   if constexpr (FMT == E4B_FMT_NF4) {
     return __uint_as_float(lds32(slot + uint32_t(4 * b)));
   } else {
-    uint32_t e;
-    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(e) : "r"(slot + off + uint32_t(b)));
+    const uint32_t e = uint32_t(mx >> (8 * b)) & 0xFFu;
     return (e - 1u < 254u) ? __uint_as_float(e << 23) : e8m0_to_f32(e);
   }
+}
+
+// MXFP4: the 3 aligned words of the scale array (total bytes `n`) that hold
+// bytes [o, o + 8), read through L1; words past the end read as zero bytes.
+E4B_DEV void mx_words(const uint8_t* scales, int64_t n, int64_t o, uint32_t (&w)[3]) {
+  const int64_t a = o & ~int64_t(3);
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int64_t q = a + 4 * j;
+    if (q + 4 <= n) {
+      w[j] = __ldg(reinterpret_cast<const uint32_t*>(scales + q));
+    } else {
+      w[j] = 0;
+      for (int64_t t = q; t < n && t < q + 4; ++t) w[j] |= uint32_t(__ldg(scales + t)) << (8 * (t - q));
+    }
+  }
+}
+
+// The 8 bytes [o, o + 8) out of mx_words' result.
+E4B_DEV uint64_t mx_bytes(const uint32_t (&w)[3], int64_t o) {
+  const uint32_t sh = uint32_t(o & 3) * 8;
+  const uint64_t lo = (uint64_t(w[1]) << 32) | w[0];
+  return sh ? (lo >> sh) | (uint64_t(w[2]) << (64 - sh)) : lo;
 }
 
 // Stage layout (1024-byte aligned, as the 128B swizzle needs):
@@ -255,9 +277,17 @@ E4B_DEV float stage_scale(uint32_t slot, int b, uint32_t off) {
 constexpr int kCodeOff = 0;
 constexpr int kXOff = kRows * 128;
 constexpr int kSOff = kXOff + 8 * kMaxTok * 64;
-constexpr int kStageBytesMax = kSOff + kRows * 16;
-static_assert(kStageBytesMax % 1024 == 0, "stages stay 1024-byte aligned");
-constexpr int kSmemBytes = 1024 + kLutBytes + kStages * kStageBytesMax + 256;  // + alignment, barriers, stage info
+// Scale bytes per row (NF4: the chunk's 4 absmax words; MXFP4: the 3 aligned
+// words that hold its 8 scale bytes), stage size, stage count.
+template <int FMT>
+struct Geo {
+  static constexpr int kSlot = 16;
+  static constexpr int kStageBytes = kSOff + kRows * kSlot;
+  static constexpr int kStages = 4;
+  static constexpr int kSmemBytes = 1024 + kLutBytes + kStages * kStageBytes + 256;  // + alignment, barriers, info
+  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+  static_assert(kSmemBytes + 8192 <= 232448, "shared memory budget");
+};
 
 // Work items: gate_up items ai * MTA + mt (mt: a block of 128 gate rows and
 // the matching 128 up rows), then down items nA + (ai * NKS + ks) * MTB + mt
@@ -274,6 +304,8 @@ template <int FMT>
 E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int32_t* s_act, uint8_t* stages,
                      uint64_t* full, uint64_t* empty, StageInfo* info, volatile int* s_abort, int nzero,
                      uint64_t limit) {
+  constexpr int kStages = Geo<FMT>::kStages;
+  constexpr int kSlot = Geo<FMT>::kSlot;
   const int lane = threadIdx.x & 31;
   const int H = p.H, I = p.I;
   int64_t i = 0;  // stages posted
@@ -341,7 +373,6 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
     const int k1 = down ? min(I, k0 + kKSplit) : H;
     const uint8_t* scales = down ? p.dn_scales : p.gu_scales;
     const int64_t sstride = FMT == E4B_FMT_NF4 ? (K / 64) * 4 : K / 32;  // scale bytes per row
-    const int64_t sbytes = int64_t(p.E) * (down ? H : 2 * I) * sstride;
     // global weight row of stage row r, or -1 past the matrix
     auto wrow = [&](int r) -> int64_t {
       if (down) {
@@ -353,12 +384,12 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
     };
 
     const CUtensorMap* cmap = down ? &maps.dn_codes : &maps.gu_codes;
-    const bool scales_tma = FMT == E4B_FMT_NF4 && (down ? p.dn_scales_tma : p.gu_scales_tma);
+    const bool scales_tma = down ? p.dn_scales_tma : p.gu_scales_tma;
     const CUtensorMap* smap = down ? &maps.dn_scales : &maps.gu_scales;
     // first global weight row of the stage's two 128-row halves
     const int64_t row0 = down ? int64_t(e) * H + int64_t(mt) * 256 : int64_t(e) * 2 * I + int64_t(mt) * 128;
     const int64_t row1 = down ? row0 + 128 : row0 + I;
-    const uint32_t tx = uint32_t(kRows * 128 + 8 * kMaxTok * 64 + (scales_tma ? kRows * 16 : 0));
+    const uint32_t tx = uint32_t(kRows * 128 + 8 * kMaxTok * 64 + (FMT == E4B_FMT_NF4 && scales_tma ? kRows * 16 : 0));
 
     for (int64_t tg = p0; tg < p1 && !aborted; tg += kMaxTok) {
       const int ntok = int(min(p1 - tg, int64_t(kMaxTok)));
@@ -375,11 +406,11 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
           give_up();
           break;
         }
-        uint8_t* st = stages + s * kStageBytesMax;
+        uint8_t* st = stages + s * Geo<FMT>::kStageBytes;
         if (lane == 0) {
           tma_load_2d(st + kCodeOff, cmap, &full[s], kc / 2, int32_t(row0));
           tma_load_2d(st + kCodeOff + 128 * 128, cmap, &full[s], kc / 2, int32_t(row1));
-          if (scales_tma) {
+          if (FMT == E4B_FMT_NF4 && scales_tma) {
             tma_load_2d(st + kSOff, smap, &full[s], (kc / 64) * 4, int32_t(row0));
             tma_load_2d(st + kSOff + 128 * 16, smap, &full[s], (kc / 64) * 4, int32_t(row1));
           }
@@ -393,24 +424,16 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
           tma_gather4_2d(st + kXOff + slab * kMaxTok * 64 + (lane & 3) * 4 * 64, &maps.x, &full[s], kc + 32 * slab,
                          gr[0], gr[1], gr[2], gr[3]);
         }
-        if (!scales_tma) {
-          // scales by cp.async, 16 bytes per row. NF4: the chunk's 4 absmax
-          // words. MXFP4: the 3 aligned words that hold the chunk's 8 bytes.
+        if (FMT == E4B_FMT_NF4 && !scales_tma) {
+          // absmax by cp.async: the chunk's 4 words of each row
           const uint32_t sbase = smem_u32(st + kSOff);
           for (int m = 0; m < kRows / 8; ++m) {
             const int q = lane + 32 * m, r = q >> 2, w = q & 3;
             const int64_t grow = wrow(r);
-            const uint32_t dst = sbase + uint32_t(r * 16 + 4 * w);
-            if constexpr (FMT == E4B_FMT_NF4) {
-              const bool v = grow >= 0 && kc + 64 * w < k1;
-              cp4(dst, v ? (const void*)(scales + grow * sstride + (kc / 64 + w) * 4) : (const void*)scales,
-                  v ? 4u : 0u);
-            } else {
-              const int64_t a = ((grow * sstride + kc / 32) & ~int64_t(3)) + 4 * w;
-              const int64_t left = sbytes - a;
-              const bool v = grow >= 0 && w < 3 && left > 0;
-              cp4(dst, v ? (const void*)(scales + a) : (const void*)scales, v ? uint32_t(left < 4 ? left : 4) : 0u);
-            }
+            const uint32_t dst = sbase + uint32_t(r * kSlot + 4 * w);
+            const bool v = grow >= 0 && kc + 64 * w < k1;
+            cp4(dst, v ? (const void*)(scales + grow * sstride + (kc / 64 + w) * 4) : (const void*)scales,
+                v ? 4u : 0u);
           }
         }
         if (lane == 0) {
@@ -457,9 +480,10 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
 // (code word c), so every mma k16 step stays inside one 32-wide chunk and
 // hence inside one scale block of each row.
 template <int FMT, int NT>
-E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, int rB, uint32_t soffA,
-                           uint32_t soffB, uint32_t lut_lane, float (&acc)[2][4]) {
+E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, int rB, uint64_t mxA,
+                           uint64_t mxB, uint32_t lut_lane, float (&acc)[2][4]) {
   constexpr bool SA = kScaleAfter<FMT>;
+  constexpr int kSlot = Geo<FMT>::kSlot;
   constexpr int BLK = FMT == E4B_FMT_NF4 ? 64 : 32;  // weights per scale block
   constexpr int NB = kChunk / BLK;                     // blocks per stage
   constexpr int CPB = BLK / 32;                        // 32-wide chunks per block
@@ -471,8 +495,8 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     const bool live = f.kc + BLK * b < kend;  // blocks past K: codes are zero, scale 0
-    const float sA = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rA + g) * 16), b, soffA) : 0.f;
-    const float sB = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rB + g) * 16), b, soffB) : 0.f;
+    const float sA = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rA + g) * kSlot), b, mxA) : 0.f;
+    const float sB = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rB + g) * kSlot), b, mxB) : 0.f;
     const uint64_t sA2 = (uint64_t(__float_as_uint(sA)) << 32) | __float_as_uint(sA);
     const uint64_t sB2 = (uint64_t(__float_as_uint(sB)) << 32) | __float_as_uint(sB);
     float P[NT][4];
@@ -524,6 +548,7 @@ template <int FMT>
 E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
                      const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, int arrive_target,
                      uint64_t limit) {
+  constexpr int kStages = Geo<FMT>::kStages;
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;  // 0 .. kConsumers-1
   const int g = lane >> 2;
@@ -536,6 +561,8 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
   for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
+  uint32_t pfA[3] = {0, 0, 0}, pfB[3] = {0, 0, 0};  // MXFP4: prefetched scale words
+  int64_t pf_o = -1;                                // ... of the chunk at row-A offset pf_o
 
   for (int64_t i = 0;; ++i) {
     const int s = int(i % kStages);
@@ -551,22 +578,44 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
     if (f.kind < 0) break;
     const bool down = f.kind == 1;
     const int kend = down ? min(I, (f.kc / kKSplit + 1) * kKSplit) : H;
-    const uint32_t st = smem_u32(stages + s * kStageBytesMax);
+    const uint32_t st = smem_u32(stages + s * Geo<FMT>::kStageBytes);
     const int rA = down ? 16 * w : 8 * w;
     const int rB = down ? 16 * w + 8 : 128 + 8 * w;
-    // MXFP4: byte offset of each of the two rows' scales inside their staged words
-    uint32_t soffA = 0, soffB = 0;
+    // MXFP4: each lane reads its two rows' scale bytes of the chunk itself
+    // (L1: consecutive chunks of a row share lines), the next chunk's
+    // prefetched while the pass continues
+    uint64_t mxA = 0, mxB = 0;
     if constexpr (FMT == E4B_FMT_MXFP4) {
       const int64_t k32 = (down ? I : H) / 32;
+      const uint8_t* scales = down ? p.dn_scales : p.gu_scales;
+      const int64_t n = int64_t(p.E) * (down ? H : 2 * I) * k32;
       auto grow = [&](int r) -> int64_t {
         return down ? int64_t(f.e) * H + int64_t(f.mt) * 256 + r
                     : int64_t(f.e) * 2 * I + int64_t(r >> 7) * I + int64_t(f.mt) * 128 + (r & 127);
       };
-      soffA = uint32_t((grow(rA + g) * k32) & 3);
-      soffB = uint32_t((grow(rB + g) * k32) & 3);
+      const int64_t oA = grow(rA + g) * k32 + f.kc / 32, oB = grow(rB + g) * k32 + f.kc / 32;
+      uint32_t wA[3], wB[3];
+      if (oA == pf_o) {
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          wA[j] = pfA[j];
+          wB[j] = pfB[j];
+        }
+      } else {
+        mx_words(scales, n, oA, wA);
+        mx_words(scales, n, oB, wB);
+      }
+      mxA = mx_bytes(wA, oA);
+      mxB = mx_bytes(wB, oB);
+      pf_o = -1;
+      if (!f.last) {
+        pf_o = oA + 8;
+        mx_words(scales, n, oA + 8, pfA);
+        mx_words(scales, n, oB + 8, pfB);
+      }
     }
-    if (f.ntok > 8) consume_stage<FMT, 2>(st, f, kend, rA, rB, soffA, soffB, lut_lane, acc);
-    else consume_stage<FMT, 1>(st, f, kend, rA, rB, soffA, soffB, lut_lane, acc);
+    if (f.ntok > 8) consume_stage<FMT, 2>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
+    else consume_stage<FMT, 1>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
     mbar_arrive(&empty[s]);  // this lane's reads of the stage are done
     if (!f.last) continue;
 
@@ -643,7 +692,8 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   const int H = p.H, I = p.I;
   const uint64_t limit = (p.flags & E4B_FLAG_TEST_TIMEOUT) ? 0u : kStageWaitNs;
   uint8_t* stages = smem + kLutBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytesMax);
+  constexpr int kStages = Geo<FMT>::kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * Geo<FMT>::kStageBytes);
   uint64_t* empty = full + kStages;
   StageInfo* info = reinterpret_cast<StageInfo*>(empty + kStages);
   volatile int* s_abort = reinterpret_cast<volatile int*>(info + kStages);
@@ -748,36 +798,43 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&m.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.h, uint64_t(I), uint64_t(L.T * L.top_k),
                       uint64_t(I) * 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
-  // NF4 absmax rows by TMA when their byte stride is a multiple of 16
-  p.gu_scales_tma = L.fmt == E4B_FMT_NF4 && H % 256 == 0;
-  p.dn_scales_tma = L.fmt == E4B_FMT_NF4 && I % 256 == 0;
+  // Scales by TMA where the layout allows: NF4 absmax rows when their byte
+  // stride is a multiple of 16; MXFP4 scale bytes when their total is.
   m.gu_scales = m.gu_codes;
   m.dn_scales = m.dn_codes;
-  if (ok && p.gu_scales_tma)
-    ok = encode_2d(&m.gu_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.gu_scales, uint64_t(H / 64 * 4), uint64_t(E * 2 * I),
-                   uint64_t(H / 64 * 4), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (ok && p.dn_scales_tma)
-    ok = encode_2d(&m.dn_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.dn_scales, uint64_t(I / 64 * 4), uint64_t(E * H),
-                   uint64_t(I / 64 * 4), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (L.fmt == E4B_FMT_NF4) {
+    p.gu_scales_tma = H % 256 == 0;
+    p.dn_scales_tma = I % 256 == 0;
+    if (ok && p.gu_scales_tma)
+      ok = encode_2d(&m.gu_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.gu_scales, uint64_t(H / 64 * 4),
+                     uint64_t(E * 2 * I), uint64_t(H / 64 * 4), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && p.dn_scales_tma)
+      ok = encode_2d(&m.dn_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.dn_scales, uint64_t(I / 64 * 4),
+                     uint64_t(E * H), uint64_t(I / 64 * 4), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  } else {
+    // MXFP4 scale bytes: 8 per row and chunk at any alignment, fetched by
+    // cp.async (one bulk copy per row measured slower)
+    p.gu_scales_tma = 0;
+    p.dn_scales_tma = 0;
+  }
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = size_t(kSmemBytes);
   static int configured = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured != dev) {
     cudaError_t e1 = cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_NF4>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    cudaError_t e2 = cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_MXFP4>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<E4B_FMT_NF4>::kSmemBytes);
+    cudaError_t e2 = cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          Geo<E4B_FMT_MXFP4>::kSmemBytes);
     if (e1 != cudaSuccess) return e1;
     if (e2 != cudaSuccess) return e2;
     configured = dev;
   }
   // persistent: one CTA per SM, all resident at once
   if (L.fmt == E4B_FMT_NF4)
-    smallm_layer_kernel<E4B_FMT_NF4><<<sms, kThreads, smem, st>>>(m, p);
+    smallm_layer_kernel<E4B_FMT_NF4><<<sms, kThreads, Geo<E4B_FMT_NF4>::kSmemBytes, st>>>(m, p);
   else
-    smallm_layer_kernel<E4B_FMT_MXFP4><<<sms, kThreads, smem, st>>>(m, p);
+    smallm_layer_kernel<E4B_FMT_MXFP4><<<sms, kThreads, Geo<E4B_FMT_MXFP4>::kSmemBytes, st>>>(m, p);
   return cudaGetLastError();
 }
 
