@@ -140,7 +140,7 @@ struct Maps {
   CUtensorMap gu_codes;   // [E*2I rows, H/2 bytes], box 128 x 128, 128B swizzle
   CUtensorMap dn_codes;   // [E*H rows, I/2 bytes], box 128 x 128, 128B swizzle
   CUtensorMap x;          // [T rows, H] bf16, box 32 x 1 (four-row gathers)
-  CUtensorMap h;          // [T*top_k rows, I] bf16, box 32 x 16
+  CUtensorMap h;          // [T*top_k rows, I] bf16, box 32 x 4
   // NF4 absmax rows [E*N rows, K/64*4 bytes], box 16 x 128 (when *_scales_tma)
   CUtensorMap gu_scales;
   CUtensorMap dn_scales;
@@ -389,10 +389,14 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
     // first global weight row of the stage's two 128-row halves
     const int64_t row0 = down ? int64_t(e) * H + int64_t(mt) * 256 : int64_t(e) * 2 * I + int64_t(mt) * 128;
     const int64_t row1 = down ? row0 + 128 : row0 + I;
-    const uint32_t tx = uint32_t(kRows * 128 + 8 * kMaxTok * 64 + (FMT == E4B_FMT_NF4 && scales_tma ? kRows * 16 : 0));
+    const uint32_t tx_fixed = uint32_t(kRows * 128 + (FMT == E4B_FMT_NF4 && scales_tma ? kRows * 16 : 0));
 
     for (int64_t tg = p0; tg < p1 && !aborted; tg += kMaxTok) {
       const int ntok = int(min(p1 - tg, int64_t(kMaxTok)));
+      // activations arrive in groups of 4 routed rows: only the groups that
+      // hold routed rows of the pass are fetched (the consumers read rows < ntok)
+      const int ngrp = (ntok + 3) / 4;
+      const uint32_t tx = tx_fixed + uint32_t(8 * ngrp * 4 * 64);
       // gate_up: the x row of each of the pass's routed rows (rows past the
       // pass repeat its first row; their products are never stored)
       int32_t xrow = 0;
@@ -415,14 +419,15 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
             tma_load_2d(st + kSOff + 128 * 16, smap, &full[s], (kc / 64) * 4, int32_t(row1));
           }
         }
-        if (down) {
-          // h rows tg.. are contiguous: one 16-row tile per 32-wide slab
-          if (lane < 8) tma_load_2d(st + kXOff + lane * kMaxTok * 64, &maps.h, &full[s], kc + 32 * lane, int32_t(tg));
-        } else {
-          // lane l gathers routed rows 4(l%4)..+3 of slab l/4
-          const int slab = lane >> 2;
-          tma_gather4_2d(st + kXOff + slab * kMaxTok * 64 + (lane & 3) * 4 * 64, &maps.x, &full[s], kc + 32 * slab,
-                         gr[0], gr[1], gr[2], gr[3]);
+        {
+          // lane l fetches routed rows 4(l%4)..+3 of 32-wide slab l/4: a
+          // 4-row tile of h (rows tg.. are contiguous) or a four-row gather of x
+          const int slab = lane >> 2, grp = lane & 3;
+          uint8_t* dst = st + kXOff + slab * kMaxTok * 64 + grp * 4 * 64;
+          if (grp < ngrp) {
+            if (down) tma_load_2d(dst, &maps.h, &full[s], kc + 32 * slab, int32_t(tg) + 4 * grp);
+            else tma_gather4_2d(dst, &maps.x, &full[s], kc + 32 * slab, gr[0], gr[1], gr[2], gr[3]);
+          }
         }
         if (FMT == E4B_FMT_NF4 && !scales_tma) {
           // absmax by cp.async: the chunk's 4 words of each row
@@ -797,7 +802,7 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
             encode_2d(&m.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.x, uint64_t(H), uint64_t(L.T), uint64_t(H) * 2, 32, 1,
                       CU_TENSOR_MAP_SWIZZLE_NONE) &&
             encode_2d(&m.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L.h, uint64_t(I), uint64_t(L.T * L.top_k),
-                      uint64_t(I) * 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+                      uint64_t(I) * 2, 32, 4, CU_TENSOR_MAP_SWIZZLE_NONE);
   // Scales by TMA where the layout allows: NF4 absmax rows when their byte
   // stride is a multiple of 16; MXFP4 scale bytes when their total is.
   m.gu_scales = m.gu_codes;
