@@ -45,7 +45,8 @@ from .formats import (
     dequant_mxfp4,
     packed_bytes_per_weight,
 )
-from .moe import route_ref, moe_forward_ref, swiglu_ref, expert_tokens
+from .moe import (route_ref, moe_forward_ref, swiglu_ref, expert_tokens, clamped_glu_ref,
+                  split_gate_up, activation_ref)
 
 __all__ = [
     "NF4_BLOCK", "MXFP4_BLOCK", "E2M1_MAGNITUDES",
@@ -53,5 +54,6 @@ __all__ = [
     "nf4_codebook", "quantize_pack_nf4", "unpack_nf4_codes", "dequant_ref",
     "dequant_ref_exact", "quantize_pack_mxfp4", "unpack_mxfp4_codes",
     "dequant_mxfp4", "packed_bytes_per_weight",
-    "route_ref", "moe_forward_ref", "swiglu_ref", "expert_tokens",
+    "route_ref", "moe_forward_ref", "swiglu_ref", "expert_tokens", "clamped_glu_ref", "split_gate_up",
+    "activation_ref",
 ]

@@ -18,7 +18,7 @@ import subprocess
 import numpy as np
 
 from .formats import bf16_round, nf4_codebook
-from .moe import expert_tokens, swiglu_ref
+from .moe import activation_ref, expert_tokens, split_gate_up
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(_HERE, "oracle_core.c")
@@ -98,22 +98,32 @@ def matvec(W: np.ndarray, X: np.ndarray) -> np.ndarray:
     return Y
 
 
-def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None):
+def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=None):
     """One expert's contribution for the rows X (bf16 values, [n, H]):
-    decode gate_up -> fp64 matmul -> bf16(silu(gate) * up) -> decode down ->
-    fp64 matmul. Returns (O fp64 [n, len(cols)], h)."""
+    decode gate_up -> fp64 matmul (+ bias) -> bf16(activation(gate, up)) ->
+    decode down -> fp64 matmul (+ bias). ``variant``: dict of moe_forward_ref's
+    expert-variant arguments (layout, act, alpha, limit, gu_bias, dn_bias),
+    the biases indexed by expert ``e``. Returns (O fp64 [n, len(cols)], h)."""
+    v = variant or {}
     Wgu = decode(fmt, *packed_gu, 2 * I, H)
     GU = matvec(Wgu, np.asarray(X, np.float64))
     del Wgu
-    h = bf16_round(swiglu_ref(GU[:, :I], GU[:, I:]))
+    if v.get("gu_bias") is not None:
+        GU = GU + np.asarray(v["gu_bias"][e], np.float64)
+    G, U = split_gate_up(GU, v.get("layout", "halves"))
+    h = bf16_round(activation_ref(G, U, v.get("act", "swiglu"), v.get("alpha", 1.702), v.get("limit", 7.0)))
     Wd = decode(fmt, *packed_dn, H, I)
     if cols is not None:
         Wd = np.ascontiguousarray(Wd[cols])
-    return matvec(Wd, h), h
+    O = matvec(Wd, h)
+    if v.get("dn_bias") is not None:
+        b = np.asarray(v["dn_bias"][e], np.float64)
+        O = O + (b if cols is None else b[cols])
+    return O, h
 
 
 def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_rows=None,
-                        packed_fn=None):
+                        packed_fn=None, variant=None):
     """Outputs y[t, n] for the given tokens (and optionally only the given
     output columns n) of the layer whose fp32 expert weights weight_fn(which,
     e) returns ("gate_up" [2I, H], "down" [H, I]); with packed_fn(which, e)
@@ -137,7 +147,7 @@ def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_row
                 packed[(which, e)] = quantize(fmt, weight_fn(which, e))
         X = x[[t for _, t in pairs]]
         O, _ = expert_term(fmt, X, packed[("gate_up", e)], packed[("down", e)], H, I,
-                           None if down_rows is None else cols)
+                           None if down_rows is None else cols, variant, e)
         for r, (slot, _) in enumerate(pairs):
             O_slot[slot] = O[r]
     y = np.zeros((len(tokens), len(cols)), np.float64)

@@ -23,9 +23,25 @@ Definitions followed
   ``dequant_mxfp4`` for MXFP4) and everything else is fp64. The oracle rounds h
   to bf16 because the fused layer stores h as bf16 between its two GEMMs.
 
+* Expert variant ("experts4bit-qlora" README, Scope: gpt-oss MXFP4 experts
+  with per-expert biases and a clamped GLU). The pages name the variant but
+  print neither its row layout nor its activation. Reading, from the released
+  gpt-oss expert definition: gate and up rows interleaved (gate = row 2n, up =
+  row 2n+1 of gate_up), fp32 biases added to each projection's output, and
+
+      g' = min(G, limit),  u' = clamp(U, -limit, limit)
+      h  = bf16_rne((u' + 1) * g' * sigmoid(alpha * g'))
+
+  with alpha and limit parameters of the call (the released model uses 1.702
+  and 7). Bias rows follow the weight rows (gate_up bias [E, 2I] in the
+  gate_up row order, down bias [E, H]).
+
 Parity pins (tests): routing invariants and a brute-force loop; the E=1, k=1,
 gate=1 case reduces to a dense SwiGLU MLP checked against torch on CPU; a
-pure-Python loop agrees with this module on tiny shapes.
+pure-Python loop agrees with this module on tiny shapes. Variant: interleaved
+rows equal the halves layout after a row permutation; the clamped GLU with
+alpha = 1 and no clamp reduces to (U + 1) * silu(G) (checked against torch's
+silu); saturation beyond the limit; biases shift the output linearly.
 """
 
 from __future__ import annotations
@@ -64,6 +80,32 @@ def swiglu_ref(G, U):
     return G / (1.0 + np.exp(-G)) * np.asarray(U, np.float64)
 
 
+def clamped_glu_ref(G, U, alpha: float, limit: float):
+    """(clamp(U, -limit, limit) + 1) * g' * sigmoid(alpha * g'), g' = min(G, limit), in fp64."""
+    g = np.minimum(np.asarray(G, np.float64), np.float64(limit))
+    u = np.clip(np.asarray(U, np.float64), -np.float64(limit), np.float64(limit))
+    return (u + 1.0) * g / (1.0 + np.exp(-np.float64(alpha) * g))
+
+
+def split_gate_up(GU, layout: str):
+    """Gate and up columns of a gate_up projection output [R, 2I]: the two
+    halves, or the even and odd rows (interleaved)."""
+    if layout == "halves":
+        I = GU.shape[-1] // 2
+        return GU[..., :I], GU[..., I:]
+    if layout == "interleaved":
+        return GU[..., 0::2], GU[..., 1::2]
+    raise ValueError(layout)
+
+
+def activation_ref(G, U, act: str, alpha: float = 1.702, limit: float = 7.0):
+    if act == "swiglu":
+        return swiglu_ref(G, U)
+    if act == "clamped_glu":
+        return clamped_glu_ref(G, U, alpha, limit)
+    raise ValueError(act)
+
+
 def _decode(fmt, codes, scales, N, K, exact=False):
     if fmt == "nf4":
         if exact:
@@ -90,7 +132,9 @@ def expert_tokens(ids, tokens=None):
 
 
 def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales,
-                    E, H, I, tokens=None, exact_decode=False, return_h=False):
+                    E, H, I, tokens=None, exact_decode=False, return_h=False,
+                    layout="halves", act="swiglu", alpha=1.702, limit=7.0,
+                    gu_bias=None, dn_bias=None):
     """The MoE layer forward (per-expert dequantise-then-matmul loop).
 
     x: bf16 values as any float array [T, H]; ids int [T, k]; gates fp32
@@ -102,6 +146,10 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
     (an expert's weights are decoded only if a selected token uses it).
     Returns y as fp64 holding bf16 values, [len(tokens) or T, H]; with
     return_h, also {slot: h row (fp64 holding bf16 values)}.
+
+    Expert variant: ``layout`` "halves" | "interleaved", ``act`` "swiglu" |
+    "clamped_glu" (alpha, limit), ``gu_bias`` [E, 2I] and ``dn_bias`` [E, H]
+    fp32 or None.
     """
     x = np.asarray(x, dtype=np.float64)
     ids = np.asarray(ids)
@@ -118,8 +166,13 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
         Wd = _decode(fmt, dn_codes[e], dn_scales[e], H, I, exact_decode)
         X = x[[t for _, t in pairs]]
         GU = X @ Wgu.T
-        h = bf16_round(swiglu_ref(GU[:, :I], GU[:, I:]))
+        if gu_bias is not None:
+            GU = GU + np.asarray(gu_bias[e], np.float64)
+        G, U = split_gate_up(GU, layout)
+        h = bf16_round(activation_ref(G, U, act, alpha, limit))
         O = h @ Wd.T
+        if dn_bias is not None:
+            O = O + np.asarray(dn_bias[e], np.float64)
         for r, (s, _) in enumerate(pairs):
             O_slot[s] = O[r]
             h_slot[s] = h[r]

@@ -75,3 +75,26 @@ def test_sampled_layer_matches_oracle_layer(fmt):
     for (which, e), (c, s) in packed.items():
         ref = (gc[e], gs[e]) if which == "gate_up" else (dc[e], ds[e])
         assert np.array_equal(c, ref[0]) and np.array_equal(s, ref[1])
+
+
+def test_sampled_layer_matches_oracle_layer_for_the_expert_variant():
+    # interleaved gate/up, biases and the clamped GLU through the C-backed path
+    fmt, E, H, I, T, k = "mxfp4", 3, 96, 160, 8, 2
+    rng = np.random.default_rng(5)
+    wgu = (rng.standard_normal((E, 2 * I, H)) * 0.3).astype(np.float32)
+    wd = (rng.standard_normal((E, H, I)) * 0.05).astype(np.float32)
+    gc, gs = oracle.quantize_pack_mxfp4(wgu)
+    dc, ds = oracle.quantize_pack_mxfp4(wd)
+    x = oracle.bf16_round(rng.standard_normal((T, H)))
+    ids = rng.integers(0, E, (T, k)).astype(np.int32)
+    gates = rng.random((T, k)).astype(np.float32)
+    v = dict(layout="interleaved", act="clamped_glu", alpha=1.702, limit=7.0,
+             gu_bias=rng.standard_normal((E, 2 * I)).astype(np.float32),
+             dn_bias=rng.standard_normal((E, H)).astype(np.float32))
+    full = oracle.moe_forward_ref(fmt, x, ids, gates, gc, gs, dc, ds, E, H, I, **v)
+    toks = [0, 3, 7]
+    fn = lambda which, e: wgu[e] if which == "gate_up" else wd[e]
+    y, _, _ = fast.moe_forward_sampled(fmt, x, ids, gates, fn, E, H, I, toks, variant=v)
+    diff = np.abs(y - full[toks])
+    assert np.all(diff <= np.abs(full[toks]) * 2 ** -7 + 1e-30)
+    assert (diff == 0).mean() > 0.99
