@@ -83,6 +83,17 @@ e4b_status check_projection(int fmt, int64_t N, int64_t K, bool swiglu) {
   return E4B_OK;
 }
 
+// Expert-variant fields (include/e4b.h): known codes, a usable clamp limit
+// and a 16-byte aligned bias.
+e4b_status check_variant(int32_t layout, int32_t act, float limit, const float* b0,
+                         const float* b1) {
+  if (layout != E4B_GATE_UP_HALVES && layout != E4B_GATE_UP_INTERLEAVED) return E4B_ERR_INVALID_ARG;
+  if (act != E4B_ACT_SWIGLU && act != E4B_ACT_CLAMPED_GLU) return E4B_ERR_INVALID_ARG;
+  if (act == E4B_ACT_CLAMPED_GLU && !(limit >= 0.f)) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(b0) || !aligned16(b1)) return E4B_ERR_MISALIGNED;
+  return E4B_OK;
+}
+
 // Small-M when an expert sees few rows on average; the tcgen05 kernel needs
 // E <= 256 for its on-chip expert table.
 bool choose_gemv(int64_t R, int64_t E, uint32_t flags) {
@@ -207,6 +218,8 @@ e4b_status e4b_grouped_gemm(const e4b_gemm_args* a, uint32_t flags, void* stream
   if (!aligned16(a->codes) || !aligned16(a->a) || !aligned16(a->out) || a->lda % 8 || a->ldo % 8)
     return E4B_ERR_MISALIGNED;
   if (a->lda < a->K) return E4B_ERR_INVALID_ARG;
+  st = check_variant(a->gate_up_layout, a->activation, a->glu_limit, a->bias, nullptr);
+  if (st != E4B_OK) return st;
   if (a->R_max == 0) return E4B_OK;
   const bool gemv = choose_gemv(a->R_max, a->E, flags);
   if (!gemv && a->E > 256) return E4B_ERR_UNSUPPORTED;
@@ -229,6 +242,11 @@ e4b_status e4b_grouped_gemm(const e4b_gemm_args* a, uint32_t flags, void* stream
   p.out = a->out;
   p.ldo = a->ldo;
   p.flags = flags;
+  p.layout = a->gate_up_layout;
+  p.act = a->activation;
+  p.alpha = a->glu_alpha;
+  p.limit = a->glu_limit;
+  p.bias = a->bias;
   g_last_path = gemv ? E4B_PATH_GEMV : E4B_PATH_TCGEN05;
   g_last_launches = 1;
   return run_projection(p, gemv, static_cast<cudaStream_t>(stream));
@@ -254,6 +272,8 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   if (st != E4B_OK) return st;
   if (H % 8) return E4B_ERR_UNSUPPORTED;
   if (E > 1024 || T * int64_t(top_k) >= (int64_t(1) << 31)) return E4B_ERR_UNSUPPORTED;
+  st = check_variant(w->gate_up_layout, w->activation, w->glu_limit, w->gate_up_bias, w->down_bias);
+  if (st != E4B_OK) return st;
   g_last_launches = 0;
   if (T == 0) return E4B_OK;
   if (!x || !ids || !gates || !y || !ws || !w->gate_up_codes || !w->gate_up_scales ||
@@ -307,6 +327,12 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
     sl.sync = sync;
     sl.status = status;
     sl.flags = flags;
+    sl.layout = w->gate_up_layout;
+    sl.act = w->activation;
+    sl.alpha = w->glu_alpha;
+    sl.limit = w->glu_limit;
+    sl.gu_bias = w->gate_up_bias;
+    sl.dn_bias = w->down_bias;
     mark(1, s);
     mark(2, s);
     ce = launch_smallm_layer(sl, s, sm_count());
@@ -348,6 +374,11 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   g.zero_count = T * H;
   g.status = status;
   g.flags = flags;
+  g.layout = w->gate_up_layout;
+  g.act = w->activation;
+  g.alpha = w->glu_alpha;
+  g.limit = w->glu_limit;
+  g.bias = w->gate_up_bias;
   mark(1, s);
   st = run_projection(g, gemv, s);
   if (st != E4B_OK) return st;
@@ -367,6 +398,7 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   d.ldo = H;
   d.zero_buf = nullptr;
   d.zero_count = 0;
+  d.bias = w->down_bias;
   mark(2, s);
   st = run_projection(d, gemv, s);
   if (st != E4B_OK) return st;

@@ -179,6 +179,24 @@ E4B_DEV uint4 ldg_nc_v4(const void* p) {
 
 E4B_DEV float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// The gate_up activation of the expert variant (include/e4b.h): SwiGLU, or
+// the clamped GLU (u' + 1) * g' * sigmoid(alpha * g') with g' = min(g, limit)
+// and u' = clamp(u, -limit, limit). Comparisons keep NaN inputs NaN.
+E4B_DEV float glu_act(int act, float g, float u, float alpha, float limit) {
+  if (act == E4B_ACT_CLAMPED_GLU) {
+    g = g > limit ? limit : g;
+    u = u > limit ? limit : (u < -limit ? -limit : u);
+    return (u + 1.0f) * g / (1.0f + expf(-alpha * g));
+  }
+  return silu_mul(g, u);
+}
+
+// gate_up row of output n's gate (m = 0) or up (m = 1) row: the two halves,
+// or interleaved (gate 2n, up 2n+1).
+E4B_DEV int64_t gate_up_row(int layout, int64_t I, int m, int64_t n) {
+  return layout == E4B_GATE_UP_INTERLEAVED ? 2 * n + m : int64_t(m) * I + n;
+}
+
 // Compacts the experts with at least one routed row (offsets[e+1] > offsets[e])
 // into s_act[0..*s_n), in expert order. Whole block; ends with __syncthreads.
 // s_warp needs blockDim.x/32 + 1 ints.

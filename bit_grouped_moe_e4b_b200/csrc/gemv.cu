@@ -108,8 +108,9 @@ gemv_kernel(GemmProblem p) {
     for (int m = 0; m < NM; ++m)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int64_t n = int64_t(m) * rows_per_mat + mt * 16 + g + 8 * h;
-        const int64_t row = int64_t(e) * N + n;
+        const int64_t n = mt * 16 + g + 8 * h;
+        const int64_t row =
+            int64_t(e) * N + (NM == 2 ? gate_up_row(p.layout, rows_per_mat, m, n) : n);
         crow[m][h] = p.codes + row * cbytes;
         srow[m][h] = scales + row * sstride;
       }
@@ -193,14 +194,23 @@ gemv_kernel(GemmProblem p) {
           if (pr >= p1) continue;
           const int64_t n = mt * 16 + g + ((i & 2) ? 8 : 0);
           if constexpr (EPI == E4B_EPI_SWIGLU) {
-            const float hv = silu_mul(acc[0][j][i], acc[NM - 1][j][i]);
+            float gv = acc[0][j][i], uv = acc[NM - 1][j][i];
+            if (p.bias) {
+              const float* b = p.bias + int64_t(e) * N;
+              gv += b[gate_up_row(p.layout, rows_per_mat, 0, n)];
+              uv += b[gate_up_row(p.layout, rows_per_mat, 1, n)];
+            }
+            const float hv = glu_act(p.act, gv, uv, p.alpha, p.limit);
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(hv);
-          } else if constexpr (EPI == E4B_EPI_STORE) {
-            static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(acc[0][j][i]);
           } else {
-            const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
-            const int64_t t = slot / p.top_k;
-            atomicAdd(static_cast<float*>(p.out) + t * p.ldo + n, p.gates[slot] * acc[0][j][i]);
+            const float v = acc[0][j][i] + (p.bias ? p.bias[int64_t(e) * N + n] : 0.f);
+            if constexpr (EPI == E4B_EPI_STORE) {
+              static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(v);
+            } else {
+              const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
+              const int64_t t = slot / p.top_k;
+              atomicAdd(static_cast<float*>(p.out) + t * p.ldo + n, p.gates[slot] * v);
+            }
           }
         }
       }

@@ -51,6 +51,10 @@ struct GemmProblem {
   int64_t zero_count;       // floats in zero_buf
   int32_t* status;          // device status word or null
   uint32_t flags;
+  // expert variant (include/e4b.h); bias: fp32 [E, N] per weight row or null
+  int layout, act;
+  float alpha, limit;
+  const float* bias;
 };
 
 cudaError_t launch_gemv(const GemmProblem& p, cudaStream_t st, int sms);
@@ -73,6 +77,10 @@ struct SmallMLayer {
   int32_t* sync;   // smallm_sync_ints(E, H) ints, zero on entry
   int32_t* status;
   uint32_t flags;
+  int layout, act;  // expert variant (include/e4b.h)
+  float alpha, limit;
+  const float* gu_bias;  // fp32 [E, 2I] or null
+  const float* dn_bias;  // fp32 [E, H] or null
 };
 size_t smallm_sync_ints(int E, int H);
 cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms);

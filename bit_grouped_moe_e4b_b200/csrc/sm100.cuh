@@ -75,6 +75,14 @@ E4B_DEV void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int32_t x, 
       : "memory");
 }
 
+E4B_DEV void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Four rows of a 2-D tensor (rows r0..r3, columns [x, x + box width)) into
 // four consecutive rows of the destination tile. The tensor map's box must be
 // one row high.

@@ -164,6 +164,10 @@ struct Params {
   int32_t* sync;     // see the sync words above
   int32_t* status;
   uint32_t flags;
+  int layout, act;       // expert variant: gate_up row layout, activation
+  float alpha, limit;    // clamped GLU constants
+  const float* gu_bias;  // [E, 2I] or null
+  const float* dn_bias;  // [E, H] or null
 };
 
 // What a stage holds (written by the producer before it releases the stage).
@@ -368,6 +372,9 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
       // h was written through the generic proxy; the TMA reads it through the async one
       asm volatile("fence.proxy.async.global;" ::: "memory");
     }
+    // interleaved gate_up: the item's 128 outputs own the 256 consecutive
+    // rows 256 mt .. (gate 2n, up 2n + 1)
+    const bool il = !down && p.layout == E4B_GATE_UP_INTERLEAVED;
     const int K = down ? I : H;
     const int k0 = down ? ks * kKSplit : 0;
     const int k1 = down ? min(I, k0 + kKSplit) : H;
@@ -379,6 +386,10 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
         const int n = mt * 256 + r;
         return n < H ? int64_t(e) * H + n : -1;
       }
+      if (il) {
+        const int q = mt * 256 + r;
+        return q < 2 * I ? int64_t(e) * 2 * I + q : -1;
+      }
       const int n = mt * 128 + (r & 127);
       return n < I ? int64_t(e) * 2 * I + int64_t(r >> 7) * I + n : -1;
     };
@@ -387,8 +398,9 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
     const bool scales_tma = down ? p.dn_scales_tma : p.gu_scales_tma;
     const CUtensorMap* smap = down ? &maps.dn_scales : &maps.gu_scales;
     // first global weight row of the stage's two 128-row halves
-    const int64_t row0 = down ? int64_t(e) * H + int64_t(mt) * 256 : int64_t(e) * 2 * I + int64_t(mt) * 128;
-    const int64_t row1 = down ? row0 + 128 : row0 + I;
+    const int64_t row0 = down ? int64_t(e) * H + int64_t(mt) * 256
+                         : int64_t(e) * 2 * I + int64_t(mt) * (il ? 256 : 128);
+    const int64_t row1 = (down || il) ? row0 + 128 : row0 + I;
     const uint32_t tx_fixed = uint32_t(kRows * 128 + (FMT == E4B_FMT_NF4 && scales_tma ? kRows * 16 : 0));
 
     for (int64_t tg = p0; tg < p1 && !aborted; tg += kMaxTok) {
@@ -546,9 +558,10 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
 
 // Consumer warps: take the stages in order until the kind -1 stage, finishing
 // each pass with its epilogue. Warp w takes, per stage, gate rows 8w..8w+7
-// (MMA rows g) and the matching up rows 128+8w.. (MMA rows g+8) for gate_up,
-// so gate and up of an output sit in the same lane; output rows 16w..16w+15
-// for down.
+// (MMA rows g) and the matching up rows 128+8w.. (MMA rows g+8) for gate_up
+// with the two halves, so gate and up of an output sit in the same lane;
+// stage rows 16w..16w+15 for down and for interleaved gate_up, where the gate
+// and up rows of an output are neighbours, four lanes apart in the fragment.
 template <int FMT>
 E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
                      const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, int arrive_target,
@@ -584,8 +597,9 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
     const bool down = f.kind == 1;
     const int kend = down ? min(I, (f.kc / kKSplit + 1) * kKSplit) : H;
     const uint32_t st = smem_u32(stages + s * Geo<FMT>::kStageBytes);
-    const int rA = down ? 16 * w : 8 * w;
-    const int rB = down ? 16 * w + 8 : 128 + 8 * w;
+    const bool il = !down && p.layout == E4B_GATE_UP_INTERLEAVED;
+    const int rA = (down || il) ? 16 * w : 8 * w;
+    const int rB = (down || il) ? 16 * w + 8 : 128 + 8 * w;
     // MXFP4: each lane reads its two rows' scale bytes of the chunk itself
     // (L1: consecutive chunks of a row share lines), the next chunk's
     // prefetched while the pass continues
@@ -595,8 +609,9 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
       const uint8_t* scales = down ? p.dn_scales : p.gu_scales;
       const int64_t n = int64_t(p.E) * (down ? H : 2 * I) * k32;
       auto grow = [&](int r) -> int64_t {
-        return down ? int64_t(f.e) * H + int64_t(f.mt) * 256 + r
-                    : int64_t(f.e) * 2 * I + int64_t(r >> 7) * I + int64_t(f.mt) * 128 + (r & 127);
+        if (down) return int64_t(f.e) * H + int64_t(f.mt) * 256 + r;
+        if (il) return int64_t(f.e) * 2 * I + int64_t(f.mt) * 256 + r;
+        return int64_t(f.e) * 2 * I + int64_t(r >> 7) * I + int64_t(f.mt) * 128 + (r & 127);
       };
       const int64_t oA = grow(rA + g) * k32 + f.kc / 32, oB = grow(rB + g) * k32 + f.kc / 32;
       uint32_t wA[3], wB[3];
@@ -627,22 +642,46 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
     // ---------------------------------------------------- end of a pass
     const int nt = f.ntok > 8 ? 2 : 1;
     if (!down) {
-      // h[p][n] = bf16(silu(gate) * up): gate in fragment rows g (d0, d1),
-      // up in rows g + 8 (d2, d3), tokens 2c, 2c+1
-      const int n = f.mt * 128 + 8 * w + g;
-      for (int j = 0; j < nt; ++j)
+      // h[p][n] = bf16(act(gate + bias, up + bias)), tokens 2c, 2c+1. Halves:
+      // gate in fragment rows g (d0, d1), up in rows g + 8 (d2, d3).
+      // Interleaved: rows g and g + 8 are stage rows 16w + g and 16w + 8 + g;
+      // an even g holds the gate of output 8w + g/2 in d0, d1 and gets its up
+      // from lane g + 1, an odd g holds the up of output 8w + 4 + (g-1)/2 in
+      // d2, d3 and gets its gate from lane g - 1.
+      const bool odd = g & 1;
+      const int n = f.mt * 128 + 8 * w + (!il ? g : odd ? 4 + (g >> 1) : (g >> 1));
+      const float* gb = p.gu_bias ? p.gu_bias + int64_t(f.e) * 2 * I : nullptr;
+      const float bg = gb && n < I ? gb[gate_up_row(p.layout, I, 0, n)] : 0.f;
+      const float bu = gb && n < I ? gb[gate_up_row(p.layout, I, 1, n)] : 0.f;
+      for (int j = 0; j < nt; ++j) {
+        float gv[2] = {acc[j][0], acc[j][1]}, uv[2] = {acc[j][2], acc[j][3]};
+        if (il) {
+          const float r0 = __shfl_xor_sync(0xffffffffu, odd ? acc[j][0] : acc[j][2], 4);
+          const float r1 = __shfl_xor_sync(0xffffffffu, odd ? acc[j][1] : acc[j][3], 4);
+          if (odd) {
+            gv[0] = r0;
+            gv[1] = r1;
+          } else {
+            uv[0] = r0;
+            uv[1] = r1;
+          }
+        }
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int tok = 8 * j + 2 * c + q;
           if (tok < f.ntok && n < I)
-            p.h[int64_t(f.p0 + tok) * I + n] = to_bf16_bits(silu_mul(acc[j][q], acc[j][q + 2]));
+            p.h[int64_t(f.p0 + tok) * I + n] =
+                to_bf16_bits(glu_act(p.act, gv[q] + bg, uv[q] + bu, p.alpha, p.limit));
         }
+      }
       __threadfence();
       // h is read next by TMA (the async proxy) in other CTAs
       asm volatile("fence.proxy.async.global;" ::: "memory");
       __syncwarp();
       if (lane == 0) atomicAdd(done_A + f.ai, 1);
     } else {
+      // the down bias joins the first K slice's partial sum only
+      const float* db = p.dn_bias && f.kc < kKSplit ? p.dn_bias + int64_t(f.e) * H : nullptr;
       for (int j = 0; j < nt; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -650,7 +689,8 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
           const int n = f.mt * 256 + 16 * w + g + ((q & 2) ? 8 : 0);
           if (tok >= f.ntok || n >= H) continue;
           const int slot = p.perm[f.p0 + tok];
-          atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * acc[j][q]);
+          const float v = acc[j][q] + (db ? db[n] : 0.f);
+          atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * v);
         }
       // the last warp to finish a pass over this 256-row output slice
       // converts the slice to bf16
@@ -793,6 +833,12 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
   p.sync = L.sync;
   p.status = L.status;
   p.flags = L.flags;
+  p.layout = L.layout;
+  p.act = L.act;
+  p.alpha = L.alpha;
+  p.limit = L.limit;
+  p.gu_bias = L.gu_bias;
+  p.dn_bias = L.dn_bias;
   const int64_t E = L.E, H = L.H, I = L.I;
   Maps m;
   bool ok = encode_2d(&m.gu_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, L.gu_codes, uint64_t(H / 2), uint64_t(E * 2 * I),

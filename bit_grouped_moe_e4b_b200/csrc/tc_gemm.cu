@@ -21,9 +21,13 @@
 //               decoded weights (128B-swizzled K-major); released by the MMA.
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer
 //               (M = 128 weight rows, N = 256 routed rows, K = 16 per MMA).
-//   warps 12-15 epilogue: tcgen05.ld of the fp32 accumulators, then SwiGLU
-//               (gate and up accumulate in two TMEM column ranges of the same
-//               lanes, so it is thread-local) or the gate-weighted combine.
+//   warps 12-15 epilogue: tcgen05.ld of the fp32 accumulators, then the
+//               biases and the gated activation (gate and up accumulate in two
+//               TMEM column ranges of the same lanes, so it is thread-local)
+//               or the gate-weighted combine.
+// Interleaved gate/up rows (gate 2n, up 2n+1) reach the same tiles through a
+// 3-D view of the codes, [E*I rows, 2, K/2 bytes]: one box fetches 128 gate
+// (or up) rows at a two-row stride.
 //               A single-matrix projection has two accumulators in TMEM, so
 //               the epilogue of one tile overlaps the MMAs of the next.
 // Tiles: per active expert, (weight-row block of 128) x (routed-row block of
@@ -154,6 +158,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   const int64_t rows_per_mat = NMAT == 2 ? N / 2 : N;
   const int64_t MT = (rows_per_mat + BM - 1) / BM;
   const int KB = int((K + BK - 1) / BK);
+  const bool il = NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED;
   const uint32_t limit = (p.flags & E4B_FLAG_TEST_TIMEOUT) ? 0u : kWaitPolls;
 
   // Clear the caller's fp32 accumulator (the layer's combine buffer) first.
@@ -248,9 +253,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           mbar_arrive_expect_tx(&c_full[s], NMAT * kCTileBytes);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
-            const int64_t row = int64_t(T.e) * N + m * rows_per_mat + T.mt * BM;
-            tma_load_2d(smem + C::kC + (s * NMAT + m) * kCTileBytes, &tmap_codes, &c_full[s],
-                        kb * (BK / 2), int32_t(row));
+            uint8_t* dst = smem + C::kC + (s * NMAT + m) * kCTileBytes;
+            if (il) {
+              tma_load_3d(dst, &tmap_codes, &c_full[s], kb * (BK / 2), m,
+                          int32_t(int64_t(T.e) * rows_per_mat + T.mt * BM));
+            } else {
+              const int64_t row = int64_t(T.e) * N + m * rows_per_mat + T.mt * BM;
+              tma_load_2d(dst, &tmap_codes, &c_full[s], kb * (BK / 2), int32_t(row));
+            }
           }
         }
       }
@@ -373,8 +383,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         cached_j = j;
         const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
         const int64_t n = T.mt * BM + r;
-        srow = n < rows_per_mat ? scales + (int64_t(T.e) * N + m * rows_per_mat + n) * sstride
-                                : nullptr;
+        const int64_t row = NMAT == 2 ? gate_up_row(p.layout, rows_per_mat, m, n) : n;
+        srow = n < rows_per_mat ? scales + (int64_t(T.e) * N + row) * sstride : nullptr;
       }
       if (!srow) return 0u;
       if constexpr (FMT == E4B_FMT_NF4) {
@@ -447,6 +457,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
       const int64_t n = T.mt * BM + rloc;
       const bool nvalid = n < rows_per_mat;
+      // bias of this thread's row(s): gate and up, or the single output row
+      float b0 = 0.f, b1 = 0.f;
+      if (p.bias && nvalid) {
+        const float* b = p.bias + int64_t(T.e) * N;
+        b0 = b[NMAT == 2 ? gate_up_row(p.layout, rows_per_mat, 0, n) : n];
+        if constexpr (NMAT == 2) b1 = b[gate_up_row(p.layout, rows_per_mat, 1, n)];
+      }
       const uint32_t lane_base =
           tmem + (uint32_t(q * 32) << 16) + uint32_t(NMAT == 2 ? 0 : ab * BN);
       for (int cc = 0; cc < BN / 16; ++cc) {
@@ -462,9 +479,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         for (int t = 0; t < 16; ++t) {
           const int64_t pr = pbase + t;
           if (pr >= T.p1) break;
-          const float gv = __uint_as_float(g[t]);
+          const float gv = __uint_as_float(g[t]) + b0;
           if constexpr (EPI == E4B_EPI_SWIGLU) {
-            const float hv = silu_mul(gv, __uint_as_float(u[t]));
+            const float hv = glu_act(p.act, gv, __uint_as_float(u[t]) + b1, p.alpha, p.limit);
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(hv);
           } else if constexpr (EPI == E4B_EPI_STORE) {
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(gv);
@@ -511,9 +528,20 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
   using C = Cfg<NMAT>;
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return cudaErrorInitializationError;
-  // Packed codes viewed as a 2-D byte tensor [E*N rows, K/2 bytes].
+  // Packed codes viewed as a 2-D byte tensor [E*N rows, K/2 bytes], or for
+  // interleaved gate/up rows as [E*I, 2, K/2] (boxes of 128 gate or up rows).
   CUtensorMap tmap_codes;
-  {
+  if (NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED) {
+    const cuuint64_t gdim[3] = {cuuint64_t(p.K / 2), 2, cuuint64_t(int64_t(p.E) * (p.N / 2))};
+    const cuuint64_t gstride[2] = {cuuint64_t(p.K / 2), cuuint64_t(p.K)};
+    const cuuint32_t box[3] = {BK / 2, 1, BM};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    CUresult cr = enc(&tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(p.codes),
+                      gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  } else {
     const cuuint64_t gdim[2] = {cuuint64_t(p.K / 2), cuuint64_t(int64_t(p.E) * p.N)};
     const cuuint64_t gstride[1] = {cuuint64_t(p.K / 2)};
     const cuuint32_t box[2] = {BK / 2, BM};

@@ -53,6 +53,9 @@ class MoeWeights(ctypes.Structure):
         ("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
         ("gate_up_codes", ctypes.c_void_p), ("gate_up_scales", ctypes.c_void_p),
         ("down_codes", ctypes.c_void_p), ("down_scales", ctypes.c_void_p),
+        ("gate_up_layout", ctypes.c_int32), ("activation", ctypes.c_int32),
+        ("glu_alpha", ctypes.c_float), ("glu_limit", ctypes.c_float),
+        ("gate_up_bias", ctypes.c_void_p), ("down_bias", ctypes.c_void_p),
     ]
 
 
@@ -64,7 +67,14 @@ class GemmArgs(ctypes.Structure):
         ("a", ctypes.c_void_p), ("lda", ctypes.c_int64), ("a_row_slot", ctypes.c_void_p),
         ("out_row_slot", ctypes.c_void_p), ("offsets", ctypes.c_void_p), ("gates", ctypes.c_void_p),
         ("out", ctypes.c_void_p), ("ldo", ctypes.c_int64),
+        ("gate_up_layout", ctypes.c_int32), ("activation", ctypes.c_int32),
+        ("glu_alpha", ctypes.c_float), ("glu_limit", ctypes.c_float), ("bias", ctypes.c_void_p),
     ]
+
+
+# expert-variant codes (include/e4b.h)
+LAYOUT = {"halves": 0, "interleaved": 1}
+ACT = {"swiglu": 0, "clamped_glu": 1}
 
 
 _lib = None
@@ -210,11 +220,13 @@ def route(ids: torch.Tensor, E: int):
 
 # --------------------------------------------------------------- grouped GEMM
 def e4b_grouped_gemm(fmt, epilogue, codes, scales, a, offsets, out, *, E, N, K, R_max, top_k=1,
-                     a_row_slot=None, out_row_slot=None, gates=None, flags=0, stream=None):
-    _dev(codes, scales, a, offsets, out, a_row_slot, out_row_slot, gates)
+                     a_row_slot=None, out_row_slot=None, gates=None, flags=0, stream=None,
+                     layout="halves", act="swiglu", alpha=1.702, limit=7.0, bias=None):
+    _dev(codes, scales, a, offsets, out, a_row_slot, out_row_slot, gates, bias)
     args = GemmArgs(FMT.get(fmt, fmt), epilogue, E, top_k, N, K, R_max, _ptr(codes), _ptr(scales),
                     _ptr(a), a.shape[-1], _ptr(a_row_slot), _ptr(out_row_slot), _ptr(offsets),
-                    _ptr(gates), _ptr(out), out.shape[-1])
+                    _ptr(gates), _ptr(out), out.shape[-1], LAYOUT[layout], ACT[act], alpha, limit,
+                    _ptr(bias))
     _check(lib().e4b_grouped_gemm(ctypes.byref(args), flags, _stream(stream)), "e4b_grouped_gemm")
 
 
@@ -230,12 +242,21 @@ class PackedLayer:
     gate_up_scales: torch.Tensor
     down_codes: torch.Tensor
     down_scales: torch.Tensor
+    # expert variant (include/e4b.h): "halves" | "interleaved", "swiglu" | "clamped_glu"
+    layout: str = "halves"
+    act: str = "swiglu"
+    alpha: float = 1.702
+    limit: float = 7.0
+    gate_up_bias: torch.Tensor | None = None  # fp32 [E, 2I]
+    down_bias: torch.Tensor | None = None     # fp32 [E, H]
 
     def c_struct(self) -> MoeWeights:
-        _dev(self.gate_up_codes, self.gate_up_scales, self.down_codes, self.down_scales)
+        _dev(self.gate_up_codes, self.gate_up_scales, self.down_codes, self.down_scales,
+             self.gate_up_bias, self.down_bias)
         return MoeWeights(FMT[self.fmt], self.E, self.H, self.I, self.gate_up_codes.data_ptr(),
                           self.gate_up_scales.data_ptr(), self.down_codes.data_ptr(),
-                          self.down_scales.data_ptr())
+                          self.down_scales.data_ptr(), LAYOUT[self.layout], ACT[self.act],
+                          self.alpha, self.limit, _ptr(self.gate_up_bias), _ptr(self.down_bias))
 
     def packed_bytes_per_expert(self) -> int:
         return (self.gate_up_codes[0].numel() + self.gate_up_scales[0].numel() * self.gate_up_scales.element_size()

@@ -91,9 +91,28 @@ typedef enum {
  *          gate_up_scales uint8 [E, 2I, H/32]     (e8m0: value 2^(byte-127))
  *          down_codes     uint8 [E, H, I/32, 16]
  *          down_scales    uint8 [E, H, I/32]
- * Rows 0..I-1 of gate_up are the gate projection, rows I..2I-1 the up
- * projection. All four arrays must be 16-byte aligned.
+ * With the default layout, rows 0..I-1 of gate_up are the gate projection and
+ * rows I..2I-1 the up projection. All four arrays must be 16-byte aligned.
+ *
+ * Expert variant ("experts4bit-qlora" README, Scope: gpt-oss MXFP4 experts
+ * with per-expert biases and a clamped GLU); all fields zero = the plain
+ * layer. The pages name the variant without its layout or constants; this
+ * library follows the released gpt-oss expert definition:
+ *   gate_up_layout  E4B_GATE_UP_HALVES (default) or E4B_GATE_UP_INTERLEAVED
+ *                   (gate = row 2n, up = row 2n+1 of gate_up)
+ *   activation      E4B_ACT_SWIGLU: h = silu(g) * u (default), or
+ *                   E4B_ACT_CLAMPED_GLU: g' = min(g, limit),
+ *                   u' = clamp(u, -limit, limit), h = (u' + 1) * g' * sigmoid(alpha * g')
+ *   glu_alpha, glu_limit   the clamped GLU's constants (released model: 1.702, 7)
+ *   gate_up_bias    fp32 [E, 2I] in gate_up row order, added to g and u; or null
+ *   down_bias       fp32 [E, H], added to each expert's down output before the
+ *                   gate weighting; or null
+ * Both biases must be 16-byte aligned. Unknown layout or activation codes, or
+ * a clamped GLU whose limit is negative or NaN, return E4B_ERR_INVALID_ARG.
  */
+typedef enum { E4B_GATE_UP_HALVES = 0, E4B_GATE_UP_INTERLEAVED = 1 } e4b_gate_up_layout;
+typedef enum { E4B_ACT_SWIGLU = 0, E4B_ACT_CLAMPED_GLU = 1 } e4b_activation;
+
 typedef struct {
   int32_t fmt; /* e4b_format */
   int32_t E, H, I;
@@ -101,6 +120,11 @@ typedef struct {
   const void* gate_up_scales;
   const uint8_t* down_codes;
   const void* down_scales;
+  int32_t gate_up_layout; /* e4b_gate_up_layout */
+  int32_t activation;     /* e4b_activation */
+  float glu_alpha, glu_limit;
+  const float* gate_up_bias;
+  const float* down_bias;
 } e4b_moe_weights;
 
 /* ---------------------------------------------------------------- formats */
@@ -205,6 +229,13 @@ typedef struct {
   const float* gates;          /* COMBINE: [T*top_k] weight of each slot */
   void* out;
   int64_t ldo;                 /* elements between output rows */
+  /* expert variant (zero = plain), as in e4b_moe_weights: SWIGLU reads
+   * gate_up_layout and activation; bias is per weight row, fp32 [E, N], added
+   * to the accumulator before the epilogue (null = none) */
+  int32_t gate_up_layout;
+  int32_t activation;
+  float glu_alpha, glu_limit;
+  const float* bias;
 } e4b_gemm_args;
 
 e4b_status e4b_grouped_gemm(const e4b_gemm_args* args, uint32_t flags, void* stream);

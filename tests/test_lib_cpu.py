@@ -90,3 +90,56 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         e4b.e4b_quantize_nf4(torch.zeros(1, 4, 64), torch.zeros(1, 4, 32, dtype=torch.uint8),
                              torch.zeros(1, 4, 1))
+
+
+def test_variant_argument_checks():
+    L = e4b.lib()
+    p = ctypes.c_void_p(4096)
+    n = ctypes.c_size_t(0)
+    w = _w()
+    assert L.e4b_moe_workspace_size(ctypes.byref(w), 64, 2, ctypes.byref(n)) == 0
+    fwd = L.e4b_moe_forward
+
+    def variant(**kw):
+        v = _w()
+        v.glu_alpha, v.glu_limit = 1.702, 7.0
+        for k, val in kw.items():
+            setattr(v, k, val)
+        return fwd(ctypes.byref(v), p, 64, 2, p, p, p, p, n.value, 0, None)
+
+    assert variant(gate_up_layout=2) == 1
+    assert variant(activation=-1) == 1
+    assert variant(activation=1, glu_limit=-0.5) == 1
+    assert variant(activation=1, glu_limit=float("nan")) == 1
+    assert variant(gate_up_bias=4100) == 7
+    assert variant(down_bias=4104) == 7
+    ga = e4b.GemmArgs(0, 1, 8, 1, 256, 256, 64, 4096, 4096, 4096, 256, None, None, 4096, None, 4096, 128,
+                      1, 1, 1.702, -1.0, None)
+    assert L.e4b_grouped_gemm(ctypes.byref(ga), 0, None) == 1
+    ga.glu_limit, ga.bias = 7.0, 4108
+    assert L.e4b_grouped_gemm(ctypes.byref(ga), 0, None) == 7
+
+
+def test_binding_structs_match_the_header(tmp_path):
+    # sizes and field offsets of the two argument structs, as a C compiler
+    # lays them out from include/e4b.h, against the ctypes mirrors
+    structs = {"e4b_moe_weights": e4b.MoeWeights, "e4b_gemm_args": e4b.GemmArgs}
+    src = ["#include <stdio.h>", "#include <stddef.h>", '#include "e4b.h"', "int main(void) {"]
+    for cname, py in structs.items():
+        src.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            src.append(f'printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    src += ["return 0; }"]
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(src))
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for cname, py in structs.items():
+        assert got[(cname, "sizeof")] == ctypes.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert got[(cname, f)] == getattr(py, f).offset, (cname, f)
