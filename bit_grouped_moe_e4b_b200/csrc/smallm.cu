@@ -182,20 +182,22 @@ struct StageInfo {
   int ntok;    // routed rows in the pass (1..16)
 };
 
-// How a block's scale is applied. NF4 (false): each weight is decoded to
-// bf16(fp32(level * absmax)) before the MMA, the decoded value every path of
-// the library and the oracle use. MXFP4 (true): the table holds the exact
-// e2m1 values and the power-of-two scale multiplies the block's fp32 MMA
-// result, which is the same product exactly.
-constexpr bool kNf4ScaleAfter = false;
-template <int FMT>
-constexpr bool kScaleAfter = FMT == E4B_FMT_MXFP4 || kNf4ScaleAfter;
+// How a block's scale is applied (template parameter SA).
+//  * SA = true, "level" decode: the table holds bf16 operands and the block's
+//    scale multiplies the block's fp32 MMA result. MXFP4 always: e2m1 values
+//    and 2^(s-127) are exact, so this is the decoded weight exactly. NF4 by
+//    default: the operand is bf16(level) and the weight bf16(level) * absmax
+//    (one 4-byte table entry per code byte).
+//  * SA = false, "product" decode (NF4 with E4B_FLAG_NF4_PRODUCT_DECODE): each
+//    weight is bf16(fp32(level * absmax)) before the MMA, the operand the
+//    tcgen05 path decodes (an 8-byte entry of two fp32 levels per code byte,
+//    twice the shared-memory traffic of the lookups).
 
 // Fills the byte table (whole CTA). The earlier weight of a byte is the high
 // nibble for NF4 and the low nibble for MXFP4; it goes first in the entry.
-template <int FMT>
+template <int FMT, bool SA>
 E4B_DEV void build_lut(uint8_t* lut) {
-  if constexpr (!kScaleAfter<FMT>) {
+  if constexpr (!SA) {
     for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x)
       reinterpret_cast<float2*>(lut)[i] = make_float2(nf4_level(i >> 8), nf4_level((i >> 4) & 15));
   } else {
@@ -228,12 +230,12 @@ E4B_DEV uint32_t scaled_pair(uint32_t addr, uint64_t absmax2) {
   return r;
 }
 
-template <int FMT>
+template <bool SA>
 E4B_DEV void lut_lookup8(uint32_t lut_lane, uint32_t w, uint64_t absmax2, uint32_t* o) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t a = lut_lane + (prmt(w, 0u, 0x4440u | uint32_t(j)) << 7);
-    if constexpr (!kScaleAfter<FMT>) o[j] = scaled_pair(a, absmax2);
+    if constexpr (!SA) o[j] = scaled_pair(a, absmax2);
     else o[j] = lds32(a);
   }
 }
@@ -496,10 +498,10 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
 // every chunk, lane c of a quad takes the 8 consecutive weights 8c..8c+7
 // (code word c), so every mma k16 step stays inside one 32-wide chunk and
 // hence inside one scale block of each row.
-template <int FMT, int NT>
+template <int FMT, int NT, bool SA>
 E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, int rB, uint64_t mxA,
                            uint64_t mxB, uint32_t lut_lane, float (&acc)[2][4]) {
-  constexpr bool SA = kScaleAfter<FMT>;
+  static_assert(SA || FMT == E4B_FMT_NF4, "MXFP4 scales always apply after the block's MMA");
   constexpr int kSlot = Geo<FMT>::kSlot;
   constexpr int BLK = FMT == E4B_FMT_NF4 ? 64 : 32;  // weights per scale block
   constexpr int NB = kChunk / BLK;                     // blocks per stage
@@ -534,8 +536,8 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
       }
       const uint32_t sw = uint32_t((ch ^ g) << 4);  // the 128B swizzle of chunk ch in row g (mod 8)
       uint32_t dA[4], dB[4];
-      lut_lookup8<FMT>(lut_lane, lds32(cA + sw), sA2, dA);
-      lut_lookup8<FMT>(lut_lane, lds32(cB + sw), sB2, dB);
+      lut_lookup8<SA>(lut_lane, lds32(cA + sw), sA2, dA);
+      lut_lookup8<SA>(lut_lane, lds32(cB + sw), sB2, dB);
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         float(&D)[4] = SA ? P[j] : acc[j];
@@ -562,7 +564,7 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
 // with the two halves, so gate and up of an output sit in the same lane;
 // stage rows 16w..16w+15 for down and for interleaved gate_up, where the gate
 // and up rows of an output are neighbours, four lanes apart in the fragment.
-template <int FMT>
+template <int FMT, bool SA>
 E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
                      const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, int arrive_target,
                      uint64_t limit) {
@@ -634,8 +636,8 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
         mx_words(scales, n, oB + 8, pfB);
       }
     }
-    if (f.ntok > 8) consume_stage<FMT, 2>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
-    else consume_stage<FMT, 1>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
+    if (f.ntok > 8) consume_stage<FMT, 2, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
+    else consume_stage<FMT, 1, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
     mbar_arrive(&empty[s]);  // this lane's reads of the stage are done
     if (!f.last) continue;
 
@@ -722,7 +724,7 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
   }
 }
 
-template <int FMT>
+template <int FMT, bool SA>
 __global__ void __launch_bounds__(kThreads, 1)
 smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -744,7 +746,7 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   volatile int* s_abort = reinterpret_cast<volatile int*>(info + kStages);
 
   // The byte table (made visible by the barriers of the clearing loop below).
-  build_lut<FMT>(smem);
+  build_lut<FMT, SA>(smem);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 33);                  // 32 producer lanes' copies + the stage info
@@ -803,8 +805,8 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   if (wid == kConsumers) {
     produce<FMT>(maps, p, W, s_act, stages, full, empty, info, s_abort, nzero, limit);
   } else {
-    const uint32_t lut_lane = smem_u32(smem) + uint32_t(!kScaleAfter<FMT> ? 8 * (lane & 15) : 4 * lane);
-    consume<FMT>(p, stages, full, empty, info, s_abort, lut_lane, s_arrive_target, limit);
+    const uint32_t lut_lane = smem_u32(smem) + uint32_t(!SA ? 8 * (lane & 15) : 4 * lane);
+    consume<FMT, SA>(p, stages, full, empty, info, s_abort, lut_lane, s_arrive_target, limit);
   }
 }
 
@@ -873,19 +875,26 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured != dev) {
-    cudaError_t e1 = cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_NF4>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<E4B_FMT_NF4>::kSmemBytes);
-    cudaError_t e2 = cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          Geo<E4B_FMT_MXFP4>::kSmemBytes);
-    if (e1 != cudaSuccess) return e1;
-    if (e2 != cudaSuccess) return e2;
+    cudaError_t e[3] = {
+        cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_NF4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Geo<E4B_FMT_NF4>::kSmemBytes),
+        cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_NF4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Geo<E4B_FMT_NF4>::kSmemBytes),
+        cudaFuncSetAttribute(smallm_layer_kernel<E4B_FMT_MXFP4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Geo<E4B_FMT_MXFP4>::kSmemBytes)};
+    for (cudaError_t x : e)
+      if (x != cudaSuccess) return x;
     configured = dev;
   }
   // persistent: one CTA per SM, all resident at once
-  if (L.fmt == E4B_FMT_NF4)
-    smallm_layer_kernel<E4B_FMT_NF4><<<sms, kThreads, Geo<E4B_FMT_NF4>::kSmemBytes, st>>>(m, p);
-  else
-    smallm_layer_kernel<E4B_FMT_MXFP4><<<sms, kThreads, Geo<E4B_FMT_MXFP4>::kSmemBytes, st>>>(m, p);
+  if (L.fmt == E4B_FMT_NF4) {
+    if (L.flags & E4B_FLAG_NF4_PRODUCT_DECODE)
+      smallm_layer_kernel<E4B_FMT_NF4, false><<<sms, kThreads, Geo<E4B_FMT_NF4>::kSmemBytes, st>>>(m, p);
+    else
+      smallm_layer_kernel<E4B_FMT_NF4, true><<<sms, kThreads, Geo<E4B_FMT_NF4>::kSmemBytes, st>>>(m, p);
+  } else {
+    smallm_layer_kernel<E4B_FMT_MXFP4, true><<<sms, kThreads, Geo<E4B_FMT_MXFP4>::kSmemBytes, st>>>(m, p);
+  }
   return cudaGetLastError();
 }
 

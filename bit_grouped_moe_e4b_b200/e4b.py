@@ -25,6 +25,7 @@ E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05 = 0, 1, 2
 FLAG_FORCE_GEMV = 0x1
 FLAG_FORCE_TCGEN05 = 0x2
 FLAG_TEST_TIMEOUT = 0x4
+FLAG_NF4_PRODUCT_DECODE = 0x8  # small-M NF4: bf16(level * absmax) operands (the default is bf16(level), absmax after the block MMA)
 STATUS_NAMES = {
     0: "E4B_OK", 1: "E4B_ERR_INVALID_ARG", 2: "E4B_ERR_UNSUPPORTED",
     3: "E4B_ERR_WORKSPACE_TOO_SMALL", 4: "E4B_ERR_CUDA", 5: "E4B_ERR_DEVICE_TIMEOUT",

@@ -75,6 +75,15 @@ typedef enum {
 #define E4B_FLAG_FORCE_GEMV 0x1u     /* use the small-M path whatever the shape */
 #define E4B_FLAG_FORCE_TCGEN05 0x2u  /* use the tcgen05 path whatever the shape */
 #define E4B_FLAG_TEST_TIMEOUT 0x4u   /* bounded waits give up at once (tests the error path) */
+/* Small-M layer path, NF4: decode every weight to bf16_rne(fp32(level *
+ * absmax)) before the MMA, the operand the tcgen05 path and e4b_grouped_gemm
+ * use. Without the flag the small-M layer path takes bf16_rne(level) as the
+ * operand and applies the fp32 absmax to each 64-weight block's fp32 partial
+ * sum, i.e. its decoded weight is bf16_rne(level) * absmax, exactly. The two
+ * decodes differ by at most one bf16 rounding of each weight (both are within
+ * 2^-8 relative of level * absmax); the default needs half the shared-memory
+ * table traffic and is the faster one. */
+#define E4B_FLAG_NF4_PRODUCT_DECODE 0x8u
 
 /* NF4 block size (weights per absmax) and MXFP4 block size (weights per scale). */
 #define E4B_NF4_BLOCK 64

@@ -40,6 +40,7 @@ from .formats import (
     unpack_nf4_codes,
     dequant_ref,
     dequant_ref_exact,
+    dequant_ref_level,
     quantize_pack_mxfp4,
     unpack_mxfp4_codes,
     dequant_mxfp4,
@@ -52,7 +53,7 @@ __all__ = [
     "NF4_BLOCK", "MXFP4_BLOCK", "E2M1_MAGNITUDES",
     "bf16_round", "bf16_bits_from_f32", "f32_from_bf16_bits",
     "nf4_codebook", "quantize_pack_nf4", "unpack_nf4_codes", "dequant_ref",
-    "dequant_ref_exact", "quantize_pack_mxfp4", "unpack_mxfp4_codes",
+    "dequant_ref_exact", "dequant_ref_level", "quantize_pack_mxfp4", "unpack_mxfp4_codes",
     "dequant_mxfp4", "packed_bytes_per_weight",
     "route_ref", "moe_forward_ref", "swiglu_ref", "expert_tokens", "clamped_glu_ref", "split_gate_up",
     "activation_ref",

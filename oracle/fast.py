@@ -45,9 +45,11 @@ def _core():
         L.e4bref_nf4_decode.argtypes = [vp, vp, i64, i64, vp, vp]
         L.e4bref_mxfp4_quantize.argtypes = [vp, i64, i64, vp, vp]
         L.e4bref_mxfp4_decode.argtypes = [vp, vp, i64, i64, vp]
+        L.e4bref_nf4_decode_level.argtypes = [vp, vp, i64, i64, vp, vp]
         L.e4bref_matvec_f64.argtypes = [vp, i64, i64, vp, i64, vp]
-        for f in ("e4bref_nf4_quantize", "e4bref_nf4_decode", "e4bref_mxfp4_quantize",
-                  "e4bref_mxfp4_decode", "e4bref_matvec_f64"):
+        L.e4bref_matvec_f64w.argtypes = [vp, i64, i64, vp, i64, vp]
+        for f in ("e4bref_nf4_quantize", "e4bref_nf4_decode", "e4bref_nf4_decode_level", "e4bref_mxfp4_quantize",
+                  "e4bref_mxfp4_decode", "e4bref_matvec_f64", "e4bref_matvec_f64w"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -74,11 +76,18 @@ def quantize(fmt: str, w: np.ndarray):
     return codes, scales
 
 
-def decode(fmt: str, codes, scales, N: int, K: int) -> np.ndarray:
-    """Parity-contract decode to fp32 [N, K] (bf16 values)."""
-    out = np.empty((N, K), np.float32)
+def decode(fmt: str, codes, scales, N: int, K: int, nf4_decode: str = "product") -> np.ndarray:
+    """Decode to [N, K]: fp32 holding bf16 values (MXFP4, NF4 "product"), or
+    fp64 for NF4 "level" (bf16_rne(level) * absmax exactly)."""
     codes = np.ascontiguousarray(codes)
     scales = np.ascontiguousarray(scales)
+    if fmt == "nf4" and nf4_decode == "level":
+        out = np.empty((N, K), np.float64)
+        _core().e4bref_nf4_decode_level(_p(codes), _p(scales), N, K, _p(nf4_codebook()), _p(out))
+        return out
+    if fmt == "nf4" and nf4_decode != "product":
+        raise ValueError(nf4_decode)
+    out = np.empty((N, K), np.float32)
     if fmt == "nf4":
         cb = nf4_codebook()
         _core().e4bref_nf4_decode(_p(codes), _p(scales), N, K, _p(cb), _p(out))
@@ -88,31 +97,36 @@ def decode(fmt: str, codes, scales, N: int, K: int) -> np.ndarray:
 
 
 def matvec(W: np.ndarray, X: np.ndarray) -> np.ndarray:
-    """fp64 X @ W^T for W fp32 [rows, K], X fp64 [n, K]."""
-    W = np.ascontiguousarray(W, np.float32)
+    """fp64 X @ W^T for W fp32 or fp64 [rows, K], X fp64 [n, K]."""
     X = np.ascontiguousarray(X, np.float64)
     rows, K = W.shape
     n = X.shape[0]
     Y = np.empty((n, rows), np.float64)
-    _core().e4bref_matvec_f64(_p(W), rows, K, _p(X), n, _p(Y))
+    if W.dtype == np.float64:
+        W = np.ascontiguousarray(W)
+        _core().e4bref_matvec_f64w(_p(W), rows, K, _p(X), n, _p(Y))
+    else:
+        W = np.ascontiguousarray(W, np.float32)
+        _core().e4bref_matvec_f64(_p(W), rows, K, _p(X), n, _p(Y))
     return Y
 
 
-def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=None):
+def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=None, nf4_decode="product"):
     """One expert's contribution for the rows X (bf16 values, [n, H]):
     decode gate_up -> fp64 matmul (+ bias) -> bf16(activation(gate, up)) ->
     decode down -> fp64 matmul (+ bias). ``variant``: dict of moe_forward_ref's
     expert-variant arguments (layout, act, alpha, limit, gu_bias, dn_bias),
-    the biases indexed by expert ``e``. Returns (O fp64 [n, len(cols)], h)."""
+    the biases indexed by expert ``e``. ``nf4_decode`` as in moe_forward_ref
+    ("product" or "level"). Returns (O fp64 [n, len(cols)], h)."""
     v = variant or {}
-    Wgu = decode(fmt, *packed_gu, 2 * I, H)
+    Wgu = decode(fmt, *packed_gu, 2 * I, H, nf4_decode)
     GU = matvec(Wgu, np.asarray(X, np.float64))
     del Wgu
     if v.get("gu_bias") is not None:
         GU = GU + np.asarray(v["gu_bias"][e], np.float64)
     G, U = split_gate_up(GU, v.get("layout", "halves"))
     h = bf16_round(activation_ref(G, U, v.get("act", "swiglu"), v.get("alpha", 1.702), v.get("limit", 7.0)))
-    Wd = decode(fmt, *packed_dn, H, I)
+    Wd = decode(fmt, *packed_dn, H, I, nf4_decode)
     if cols is not None:
         Wd = np.ascontiguousarray(Wd[cols])
     O = matvec(Wd, h)
@@ -123,11 +137,12 @@ def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=N
 
 
 def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_rows=None,
-                        packed_fn=None, variant=None):
+                        packed_fn=None, variant=None, nf4_decode="product"):
     """Outputs y[t, n] for the given tokens (and optionally only the given
     output columns n) of the layer whose fp32 expert weights weight_fn(which,
     e) returns ("gate_up" [2I, H], "down" [H, I]); with packed_fn(which, e)
     given instead, the experts arrive already packed (codes, scales).
+    nf4_decode: the NF4 weight value as in moe_forward_ref.
 
     Returns (y fp64 holding bf16 values [len(tokens), len(cols)], cols,
     packed) where packed[(which, e)] = (codes, scales) this function used.
@@ -147,7 +162,7 @@ def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_row
                 packed[(which, e)] = quantize(fmt, weight_fn(which, e))
         X = x[[t for _, t in pairs]]
         O, _ = expert_term(fmt, X, packed[("gate_up", e)], packed[("down", e)], H, I,
-                           None if down_rows is None else cols, variant, e)
+                           None if down_rows is None else cols, variant, e, nf4_decode)
         for r, (slot, _) in enumerate(pairs):
             O_slot[slot] = O[r]
     y = np.zeros((len(tokens), len(cols)), np.float64)

@@ -22,10 +22,17 @@ per-expert fp32 absmax):
     distance; ties go to the lower index). ``a == 0`` gives code 7 (the zero
     level) for the whole block. Pack two codes per byte, the first element of
     each pair in the HIGH nibble.
-  * decode: ``dequant_ref`` returns the parity-contract weight value
-    ``bf16_rne(fp32(c[code]) * a)`` (the product rounded to fp32, then once to
-    bf16). ``dequant_ref_exact`` returns ``c[code] * a`` in fp64, used for
-    fidelity reports only.
+  * decode (the README's kernel decodes to fp32 in registers and applies the
+    blockwise scale; the tensor cores take bf16 operands, so the reading
+    fixes where the one bf16 rounding falls -- two ways, both within 2^-8
+    relative of ``c[code] * a``):
+      - ``dequant_ref`` ("product"): ``bf16_rne(fp32(c[code]) * a)`` (the
+        product rounded to fp32, then once to bf16);
+      - ``dequant_ref_level`` ("level"): ``bf16_rne(c[code]) * a``, the exact
+        product of the bf16-rounded level and the fp32 absmax (the operand is
+        the rounded level; the scale multiplies the block's partial sum).
+    ``dequant_ref_exact`` returns ``c[code] * a`` in fp64, used for fidelity
+    reports only.
 
 MXFP4 (README intro: "MXFP4 (OCP e2m1 + e8m0)"; CPU block 2:
 ``quantize_pack_mxfp4(w) -> blocks [N, K/32, 16] u8, scales [N, K/32] u8``;
@@ -193,6 +200,15 @@ def dequant_ref(packed, absmax, N: int, K: int, blocksize: int = NF4_BLOCK) -> n
     a = _expand_blocks(np.asarray(absmax, np.float32), K, blocksize)
     prod = (cb[codes] * a).astype(np.float32)  # one fp32 rounding of the product
     return bf16_round(prod).astype(np.float32)
+
+
+def dequant_ref_level(packed, absmax, N: int, K: int, blocksize: int = NF4_BLOCK) -> np.ndarray:
+    """Decode NF4 as bf16_rne(c[code]) * absmax, the exact product (fp64)."""
+    codes = unpack_nf4_codes(packed)
+    assert codes.shape[-2:] == (N, K)
+    cb = bf16_round(nf4_codebook()).astype(np.float64)
+    a = _expand_blocks(np.asarray(absmax, np.float64), K, blocksize)
+    return cb[codes] * a
 
 
 def dequant_ref_exact(packed, absmax, N: int, K: int, blocksize: int = NF4_BLOCK) -> np.ndarray:

@@ -52,6 +52,7 @@ from .formats import (
     bf16_round,
     dequant_ref,
     dequant_ref_exact,
+    dequant_ref_level,
     dequant_mxfp4,
 )
 
@@ -106,11 +107,18 @@ def activation_ref(G, U, act: str, alpha: float = 1.702, limit: float = 7.0):
     raise ValueError(act)
 
 
-def _decode(fmt, codes, scales, N, K, exact=False):
+NF4_DECODES = ("product", "level", "exact")
+
+
+def _decode(fmt, codes, scales, N, K, nf4_decode="product"):
     if fmt == "nf4":
-        if exact:
+        if nf4_decode == "exact":
             return dequant_ref_exact(codes, scales, N, K)
-        return dequant_ref(codes, scales, N, K).astype(np.float64)
+        if nf4_decode == "level":
+            return dequant_ref_level(codes, scales, N, K)
+        if nf4_decode == "product":
+            return dequant_ref(codes, scales, N, K).astype(np.float64)
+        raise ValueError(nf4_decode)
     if fmt == "mxfp4":
         return dequant_mxfp4(codes, scales).reshape(N, K).astype(np.float64)
     raise ValueError(fmt)
@@ -134,7 +142,7 @@ def expert_tokens(ids, tokens=None):
 def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales,
                     E, H, I, tokens=None, exact_decode=False, return_h=False,
                     layout="halves", act="swiglu", alpha=1.702, limit=7.0,
-                    gu_bias=None, dn_bias=None):
+                    gu_bias=None, dn_bias=None, nf4_decode="product"):
     """The MoE layer forward (per-expert dequantise-then-matmul loop).
 
     x: bf16 values as any float array [T, H]; ids int [T, k]; gates fp32
@@ -150,6 +158,11 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
     Expert variant: ``layout`` "halves" | "interleaved", ``act`` "swiglu" |
     "clamped_glu" (alpha, limit), ``gu_bias`` [E, 2I] and ``dn_bias`` [E, H]
     fp32 or None.
+
+    nf4_decode: the NF4 weight value, "product" (bf16_rne(fp32(level *
+    absmax)), dequant_ref), "level" (bf16_rne(level) * absmax exactly,
+    dequant_ref_level) or "exact" (level * absmax, fidelity only; also
+    selected by exact_decode=True).
     """
     x = np.asarray(x, dtype=np.float64)
     ids = np.asarray(ids)
@@ -162,8 +175,9 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
     O_slot = {}
     h_slot = {}
     for e, pairs in sorted(expert_tokens(ids, sel).items()):
-        Wgu = _decode(fmt, gu_codes[e], gu_scales[e], 2 * I, H, exact_decode)
-        Wd = _decode(fmt, dn_codes[e], dn_scales[e], H, I, exact_decode)
+        mode = "exact" if exact_decode else nf4_decode
+        Wgu = _decode(fmt, gu_codes[e], gu_scales[e], 2 * I, H, mode)
+        Wd = _decode(fmt, dn_codes[e], dn_scales[e], H, I, mode)
         X = x[[t for _, t in pairs]]
         GU = X @ Wgu.T
         if gu_bias is not None:

@@ -8,7 +8,8 @@
  *     absmax per 64-weight block, s = fp32(w / absmax), nearest level with
  *     ties to the lower index (decided exactly: 2s > c[i] + c[i+1] in double),
  *     zero block -> level 7; packed with the earlier weight in the high nibble;
- *     decoded value bf16_rne(fp32(c[code] * absmax)).
+ *     decoded value bf16_rne(fp32(c[code] * absmax)) ("product"), or
+ *     bf16_rne(c[code]) * absmax as the exact double product ("level").
  *   MXFP4 (README intro, CPU block 2; OCP MX v1.0): e = floor(log2 amax) - 2
  *     clamped to [-127, 127], elements rounded to e2m1 with ties to even,
  *     sign bit copied, earlier weight in the low nibble.
@@ -80,6 +81,18 @@ void e4bref_nf4_decode(const uint8_t* codes, const float* absmax, int64_t rows, 
   }
 }
 
+void e4bref_nf4_decode_level(const uint8_t* codes, const float* absmax, int64_t rows, int64_t K,
+                             const float* cb, double* out) {
+  const int64_t nb = K / 64;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      const uint8_t byte = codes[r * (K / 2) + k / 2];
+      const int c = (k & 1) ? (byte & 15) : (byte >> 4);
+      out[r * K + k] = (double)bf16_rne_f32(cb[c]) * (double)absmax[r * nb + k / 64];
+    }
+  }
+}
+
 static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 
 static int e2m1_nearest(double m) {
@@ -144,6 +157,19 @@ void e4bref_mxfp4_decode(const uint8_t* blocks, const uint8_t* scales, int64_t r
 }
 
 /* y[i, r] = sum_k W[r, k] * x[i, k] in fp64, for n vectors x. */
+void e4bref_matvec_f64w(const double* W, int64_t rows, int64_t K, const double* x, int64_t n,
+                        double* y) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double* xi = x + i * K;
+    for (int64_t r = 0; r < rows; ++r) {
+      const double* wr = W + r * K;
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += wr[k] * xi[k];
+      y[i * rows + r] = acc;
+    }
+  }
+}
+
 void e4bref_matvec_f64(const float* W, int64_t rows, int64_t K, const double* x, int64_t n,
                        double* y) {
   for (int64_t i = 0; i < n; ++i) {

@@ -18,11 +18,18 @@ def scaled_err(y, y_ref) -> float:
     return float(np.max(np.abs(y - y_ref) / (1.0 + np.abs(y_ref)))) if y.size else 0.0
 
 
-def assert_close(y, y_ref, what=""):
+def assert_close(y, y_ref, what="", tol=TOL):
     err = scaled_err(y, y_ref)
     assert np.all(np.isfinite(y)), what
-    assert err <= TOL, f"{what}: max scaled error {err:.4g} > {TOL}"
+    assert err <= tol, f"{what}: max scaled error {err:.4g} > {tol}"
     return err
+
+
+# Between the two kernel paths on NF4: their decode readings ("level" on
+# small-M, "product" on tcgen05) differ by up to one bf16 rounding of every
+# weight, which at full size moves outputs by a few 1e-2 of the scale; each
+# path matches its own reading within TOL.
+TOL_NF4_ACROSS_PATHS = 5e-2
 
 
 def oracle_quantize(fmt, w: np.ndarray):
@@ -59,6 +66,18 @@ def small_layer(fmt, E, H, I, seed, std=0.02, spread=False):
     return layer, (gc, gs, dc, ds)
 
 
+_last = {"flags": 0}
+
+
+def last_nf4_decode() -> str:
+    """The NF4 decode reading the last layer call used: the small-M path's
+    default "level" (bf16(level), absmax after the block's MMA) unless the
+    product flag was given; "product" (bf16(fp32(level * absmax))) on tcgen05."""
+    if e4b.e4b_last_path() == e4b.E4B_PATH_GEMV and not (_last["flags"] & e4b.FLAG_NF4_PRODUCT_DECODE):
+        return "level"
+    return "product"
+
+
 def run_layer(layer, x_bf16: torch.Tensor, ids: np.ndarray, gates: np.ndarray, flags=0, staged=True):
     """staged=False hands the layer a workspace without room for the staging
     copy of the routed rows (the last [T*k, H] bf16 region), so the large-M
@@ -69,12 +88,16 @@ def run_layer(layer, x_bf16: torch.Tensor, ids: np.ndarray, gates: np.ndarray, f
     ws = e4b.workspace(layer, ids.shape[0], ids.shape[1])
     if not staged:
         ws = ws[: ws.numel() - (ids.size * layer.H * 2 + 255) // 256 * 256]
+    _last["flags"] = flags
     y = e4b.moe_forward(layer, x_d, ids_d, g_d, ws=ws, flags=flags)
     status = e4b.e4b_read_device_status(ws)
     return y.float().cpu().numpy(), status, ws
 
 
-def oracle_layer(fmt, x_bf16: torch.Tensor, ids, gates, ref, E, H, I, tokens=None):
+def oracle_layer(fmt, x_bf16: torch.Tensor, ids, gates, ref, E, H, I, tokens=None, nf4_decode="last"):
+    """The oracle's layer forward; nf4_decode "last" = the reading the last
+    layer call used (last_nf4_decode)."""
     gc, gs, dc, ds = ref
+    mode = last_nf4_decode() if nf4_decode == "last" else nf4_decode
     return oracle.moe_forward_ref(fmt, x_bf16.float().numpy(), ids, gates, gc, gs, dc, ds, E, H, I,
-                                  tokens=tokens)
+                                  tokens=tokens, nf4_decode=mode)

@@ -9,12 +9,14 @@ import torch
 import oracle
 from bit_grouped_moe_e4b_b200 import e4b, synth
 from bit_grouped_moe_e4b_b200.configs import TINY
-from gpu_util import assert_close, oracle_layer, run_layer, small_layer
+from gpu_util import assert_close, last_nf4_decode, oracle_layer, run_layer, scaled_err, small_layer
 
 pytestmark = pytest.mark.gpu
 
 PATHS = {"gemv": e4b.FLAG_FORCE_GEMV, "tcgen05": e4b.FLAG_FORCE_TCGEN05,
-         "tcgen05_gather": e4b.FLAG_FORCE_TCGEN05}
+         "tcgen05_gather": e4b.FLAG_FORCE_TCGEN05,
+         # small-M with the NF4 product decode (the tcgen05 path's operands)
+         "gemv_product": e4b.FLAG_FORCE_GEMV | e4b.FLAG_NF4_PRODUCT_DECODE}
 
 
 def _run(layer, x, ids, gates, path):
@@ -90,15 +92,18 @@ def test_many_tiles_per_cta(path):
         _many["layer"] = small_layer(fmt, E, H, I, seed=64)
         x = _x(T, H, seed=5)
         ids, gates = synth.random_ids(np.random.default_rng(6), T, k, E)
-        _many["case"] = (x, ids, gates, oracle_layer(fmt, x, ids, gates, _many["layer"][1], E, H, I))
-    layer, _ = _many["layer"]
-    x, ids, gates, y_ref = _many["case"]
+        _many["case"] = (x, ids, gates)
+    layer, ref = _many["layer"]
+    x, ids, gates = _many["case"]
     y, status, _ = _run(layer, x, ids, gates, path)
     assert status == 0
-    assert_close(y, y_ref, f"{fmt} {E}x{H}x{I} T={T} {path}")
+    key = ("ref", last_nf4_decode())
+    if key not in _many:
+        _many[key] = oracle_layer(fmt, x, ids, gates, ref, E, H, I)
+    assert_close(y, _many[key], f"{fmt} {E}x{H}x{I} T={T} {path}")
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("path", ["gemv", "gemv_product", "tcgen05"])
 @pytest.mark.parametrize("fmt,E,H,I,T,k", [("nf4", 3, 256, 320, 40, 2), ("mxfp4", 3, 288, 224, 40, 2),
                                            ("mxfp4", 2, 96, 160, 9, 1)])
 def test_block_scales_and_large_outputs(fmt, E, H, I, T, k, path):
@@ -111,9 +116,15 @@ def test_block_scales_and_large_outputs(fmt, E, H, I, T, k, path):
     rng = np.random.default_rng(4)
     ids, gates = synth.random_ids(rng, T, k, E)
     y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    mode = last_nf4_decode()
     y_ref = oracle_layer(fmt, x, ids, gates, ref, E, H, I)
     assert status == 0 and 3.0 < np.abs(y_ref).max() < 100.0
     assert_close(y, y_ref, f"{fmt} spread {E}x{H}x{I} {path}")
+    if fmt == "nf4":
+        # the two NF4 readings differ visibly on this data: the kernel follows
+        # the reading of its path, not the other one
+        other = oracle_layer(fmt, x, ids, gates, ref, E, H, I, nf4_decode="product" if mode == "level" else "level")
+        assert scaled_err(y, y_ref) < scaled_err(y, other), (path, mode)
 
 
 EDGE = {

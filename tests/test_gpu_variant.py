@@ -14,7 +14,7 @@ import oracle
 from oracle import fast
 from bit_grouped_moe_e4b_b200 import e4b, synth
 from bit_grouped_moe_e4b_b200.configs import MXFP4
-from gpu_util import assert_close, run_layer, small_layer
+from gpu_util import assert_close, last_nf4_decode, run_layer, small_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -63,7 +63,8 @@ def test_clamped_glu_with_biases(fmt, E, H, I, T, k, layout, path):
     y, status, _ = run_layer(vl, x, ids, gates, PATHS[path], staged=path != "tcgen05_gather")
     assert status == 0
     y_ref = oracle.moe_forward_ref(fmt, x.float().numpy(), ids, gates, *ref, E, H, I, layout=layout,
-                                   act="clamped_glu", alpha=ALPHA, limit=LIMIT, gu_bias=bgu, dn_bias=bd)
+                                   act="clamped_glu", alpha=ALPHA, limit=LIMIT, gu_bias=bgu, dn_bias=bd,
+                                   nf4_decode=last_nf4_decode())
     assert_close(y, y_ref, f"{fmt} {layout} {path}")
 
 
@@ -84,7 +85,7 @@ def test_variant_parts(which, path):
     y, status, _ = run_layer(vl, x, ids, gates, PATHS[path])
     assert status == 0
     y_ref = oracle.moe_forward_ref(fmt, x.float().numpy(), ids, gates, *ref, E, H, I, layout=layout,
-                                   act="swiglu", gu_bias=gb, dn_bias=db)
+                                   act="swiglu", gu_bias=gb, dn_bias=db, nf4_decode=last_nf4_decode())
     assert_close(y, y_ref, f"{which} {path}")
 
 
@@ -100,7 +101,8 @@ def test_down_bias_counted_once_across_k_slices():
     for path in ("gemv", "tcgen05"):
         y, status, _ = run_layer(vl, x, ids, gates, PATHS[path])
         assert status == 0
-        y_ref = oracle.moe_forward_ref(fmt, x.float().numpy(), ids, gates, *ref, E, H, I, dn_bias=bd)
+        y_ref = oracle.moe_forward_ref(fmt, x.float().numpy(), ids, gates, *ref, E, H, I, dn_bias=bd,
+                                       nf4_decode=last_nf4_decode())
         assert_close(y, y_ref, f"down bias, K split, {path}")
 
 
