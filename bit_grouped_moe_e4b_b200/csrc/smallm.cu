@@ -193,25 +193,30 @@ struct StageInfo {
 //    tcgen05 path decodes (an 8-byte entry of two fp32 levels per code byte,
 //    twice the shared-memory traffic of the lookups).
 
-// Fills the byte table (whole CTA). The earlier weight of a byte is the high
-// nibble for NF4 and the low nibble for MXFP4; it goes first in the entry.
+// Fills the byte table (whole CTA; ends with a barrier). The earlier weight of
+// a byte is the high nibble for NF4 and the low nibble for MXFP4; it goes
+// first in the entry. The 16 values of a nibble are staged in shared memory
+// first: indexing the constant level arrays with a per-thread value would
+// rebuild them in local memory at every call.
 template <int FMT, bool SA>
-E4B_DEV void build_lut(uint8_t* lut) {
+E4B_DEV void build_lut(uint8_t* lut, float* s_val) {
+  if (threadIdx.x < 16) {
+    const int n = threadIdx.x;
+    s_val[n] = FMT == E4B_FMT_NF4 ? nf4_level(n) : ((n & 8) ? -e2m1_magnitude(n & 7) : e2m1_magnitude(n & 7));
+  }
+  __syncthreads();
   if constexpr (!SA) {
     for (int i = threadIdx.x; i < 256 * 16; i += blockDim.x)
-      reinterpret_cast<float2*>(lut)[i] = make_float2(nf4_level(i >> 8), nf4_level((i >> 4) & 15));
+      reinterpret_cast<float2*>(lut)[i] = make_float2(s_val[i >> 8], s_val[(i >> 4) & 15]);
   } else {
     for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
       const int v = i >> 5, lo = v & 15, hi = v >> 4;
-      float a = (lo & 8) ? -e2m1_magnitude(lo & 7) : e2m1_magnitude(lo & 7);
-      float b = (hi & 8) ? -e2m1_magnitude(hi & 7) : e2m1_magnitude(hi & 7);
-      if (FMT == E4B_FMT_NF4) {
-        a = nf4_level(hi);
-        b = nf4_level(lo);
-      }
-      reinterpret_cast<uint32_t*>(lut)[i] = pack_bf16x2(a, b);
+      const float first = FMT == E4B_FMT_NF4 ? s_val[hi] : s_val[lo];
+      const float second = FMT == E4B_FMT_NF4 ? s_val[lo] : s_val[hi];
+      reinterpret_cast<uint32_t*>(lut)[i] = pack_bf16x2(first, second);
     }
   }
+  __syncthreads();
 }
 
 // 8 codes (one 32-bit word, weights in byte order) -> 4 bf16x2 weight pairs,
@@ -746,7 +751,8 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   volatile int* s_abort = reinterpret_cast<volatile int*>(info + kStages);
 
   // The byte table (made visible by the barriers of the clearing loop below).
-  build_lut<FMT, SA>(smem);
+  __shared__ float s_val[16];
+  build_lut<FMT, SA>(smem, s_val);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 33);                  // 32 producer lanes' copies + the stage info
