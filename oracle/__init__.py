@@ -47,7 +47,7 @@ from .formats import (
     packed_bytes_per_weight,
 )
 from .moe import (route_ref, moe_forward_ref, swiglu_ref, expert_tokens, clamped_glu_ref,
-                  split_gate_up, activation_ref)
+                  split_gate_up, activation_ref, grouped_projection_ref, grouped_dgrad_ref)
 
 __all__ = [
     "NF4_BLOCK", "MXFP4_BLOCK", "E2M1_MAGNITUDES",
@@ -56,5 +56,5 @@ __all__ = [
     "dequant_ref_exact", "dequant_ref_level", "quantize_pack_mxfp4", "unpack_mxfp4_codes",
     "dequant_mxfp4", "packed_bytes_per_weight",
     "route_ref", "moe_forward_ref", "swiglu_ref", "expert_tokens", "clamped_glu_ref", "split_gate_up",
-    "activation_ref",
+    "activation_ref", "grouped_projection_ref", "grouped_dgrad_ref",
 ]

@@ -36,12 +36,22 @@ Definitions followed
   and 7). Bias rows follow the weight rows (gate_up bias [E, 2I] in the
   gate_up row order, down bias [E, H]).
 
+* Grouped projection and its input gradient ("grouped-nf4-gemm" README,
+  intro and entry table: the grouped GEMM and, for training, its backward
+  ``dgrad_4bit_grouped``): for routed row p of expert e,
+      out[p] = a[p] . D(W_e)^T        (grouped_projection_ref)
+      dx[p]  = dy[p] . D(W_e)         (grouped_dgrad_ref, the contraction over
+                                       the weight's rows: its adjoint)
+  fp64, rounded once to bf16.
+
 Parity pins (tests): routing invariants and a brute-force loop; the E=1, k=1,
 gate=1 case reduces to a dense SwiGLU MLP checked against torch on CPU; a
 pure-Python loop agrees with this module on tiny shapes. Variant: interleaved
 rows equal the halves layout after a row permutation; the clamped GLU with
 alpha = 1 and no clamp reduces to (U + 1) * silu(G) (checked against torch's
 silu); saturation beyond the limit; biases shift the output linearly.
+Projection and dgrad: the adjoint identity <dgrad(dy), a> = <dy, proj(a)>
+before rounding, a brute-force loop on tiny shapes, and empty experts.
 """
 
 from __future__ import annotations
@@ -199,3 +209,34 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
     if return_h:
         return y, h_slot
     return y
+
+
+def grouped_projection_ref(fmt, a, offsets, codes, scales, N, K, nf4_decode="product"):
+    """The grouped projection ("grouped-nf4-gemm" README, intro): routed row p
+    of expert e (offsets[e] <= p < offsets[e+1]) times the decoded weight
+    W_e [N, K]: out[p] = a[p] . W_e^T (a [R, K] -> out [R, N]), fp64 holding
+    the bf16-rounded result."""
+    a = np.asarray(a, np.float64)
+    offsets = np.asarray(offsets)
+    out = np.zeros((a.shape[0], N), np.float64)
+    for e in range(len(offsets) - 1):
+        p0, p1 = int(offsets[e]), int(offsets[e + 1])
+        if p1 > p0:
+            out[p0:p1] = a[p0:p1] @ _decode(fmt, codes[e], scales[e], N, K, nf4_decode).T
+    return bf16_round(out)
+
+
+def grouped_dgrad_ref(fmt, dy, offsets, codes, scales, N, K, nf4_decode="product"):
+    """The input gradient through the packed weights ("grouped-nf4-gemm"
+    README, entry table: the NF4 grouped GEMM's backward, dgrad_4bit_grouped):
+    for routed row p of expert e, dx[p] = dy[p] . W_e, the contraction over the
+    weight's rows (dy [R, N] -> dx [R, K]) -- the adjoint of
+    grouped_projection_ref. fp64 holding the bf16-rounded result."""
+    dy = np.asarray(dy, np.float64)
+    offsets = np.asarray(offsets)
+    out = np.zeros((dy.shape[0], K), np.float64)
+    for e in range(len(offsets) - 1):
+        p0, p1 = int(offsets[e]), int(offsets[e + 1])
+        if p1 > p0:
+            out[p0:p1] = dy[p0:p1] @ _decode(fmt, codes[e], scales[e], N, K, nf4_decode)
+    return bf16_round(out)
