@@ -252,6 +252,40 @@ e4b_status e4b_grouped_gemm(const e4b_gemm_args* a, uint32_t flags, void* stream
   return run_projection(p, gemv, static_cast<cudaStream_t>(stream));
 }
 
+e4b_status e4b_grouped_dgrad(const e4b_dgrad_args* a, uint32_t flags, void* stream) {
+  if (!a) return E4B_ERR_INVALID_ARG;
+  if (a->E <= 0 || a->R_max < 0) return E4B_ERR_INVALID_ARG;
+  if (a->fmt != E4B_FMT_NF4 && a->fmt != E4B_FMT_MXFP4) return E4B_ERR_INVALID_ARG;
+  if (a->N <= 0 || a->K <= 0) return E4B_ERR_INVALID_ARG;
+  if (a->fmt == E4B_FMT_NF4 && a->K % E4B_NF4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (a->fmt == E4B_FMT_MXFP4 && a->K % E4B_MXFP4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (a->E > 256 || (flags & E4B_FLAG_FORCE_GEMV)) return E4B_ERR_UNSUPPORTED;
+  if (!a->codes || !a->scales || !a->dy || !a->offsets || !a->dx) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(a->codes) || !aligned16(a->dy) || !aligned16(a->dx) || a->ld_dy % 8 || a->ld_dx % 8)
+    return E4B_ERR_MISALIGNED;
+  if (a->ld_dy < a->N || a->ld_dx < a->K) return E4B_ERR_INVALID_ARG;
+  if (a->R_max == 0) return E4B_OK;
+  GemmProblem p{};
+  p.fmt = a->fmt;
+  p.epilogue = kEpiDgrad;
+  p.E = a->E;
+  p.top_k = 1;
+  p.N = a->N;
+  p.K = a->K;
+  p.R_max = a->R_max;
+  p.codes = a->codes;
+  p.scales = a->scales;
+  p.a = a->dy;
+  p.lda = a->ld_dy;
+  p.offsets = a->offsets;
+  p.out = a->dx;
+  p.ldo = a->ld_dx;
+  p.flags = flags;
+  g_last_path = E4B_PATH_TCGEN05;
+  g_last_launches = 1;
+  return cuda_status(launch_tc_gemm(p, static_cast<cudaStream_t>(stream), sm_count()));
+}
+
 e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
                                   size_t* bytes) {
   if (!w || !bytes || T < 0 || top_k <= 0 || w->E <= 0 || w->H <= 0 || w->I <= 0)

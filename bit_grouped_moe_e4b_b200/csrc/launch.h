@@ -29,6 +29,10 @@ cudaError_t launch_gather_rows(const uint16_t* x, int64_t H, const int32_t* perm
 // routed rows that e4b_moe_workspace_size includes).
 size_t moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k);
 
+// GemmProblem::epilogue for the input gradient through the weights
+// (e4b_grouped_dgrad): out [R, K] bf16, row p = a_p . W_e, a [R, N].
+constexpr int kEpiDgrad = 3;
+
 // Description of one grouped projection as the kernels see it.
 struct GemmProblem {
   int fmt;          // e4b_format

@@ -179,6 +179,20 @@ E4B_DEV uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major bf16 tile with the 128B
+// swizzle: atoms of 8 K-rows x 128 bytes (64 consecutive M or N elements per
+// row, 1024 bytes per atom); lbo = bytes between atoms along M/N, sbo = bytes
+// between atoms along K. Each atom starts on a 1024-byte boundary.
+E4B_DEV uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;                  // descriptor version for sm_100
+  d |= uint64_t(2) << 61;                  // layout: 128B swizzle
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 D, both
 // operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {

@@ -125,6 +125,7 @@ template <int FMT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                const __grid_constant__ CUtensorMap tmap_act, GemmProblem p) {
+  constexpr bool DG = EPI == kEpiDgrad;
   constexpr int NMAT = (EPI == E4B_EPI_SWIGLU) ? 2 : 1;
   using C = Cfg<NMAT>;
   constexpr int CS = C::CS;
@@ -156,8 +157,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   const int64_t N = p.N;
   const int64_t K = p.K;
   const int64_t rows_per_mat = NMAT == 2 ? N / 2 : N;
-  const int64_t MT = (rows_per_mat + BM - 1) / BM;
-  const int KB = int((K + BK - 1) / BK);
+  // dgrad: the MMA's M runs over the weight's columns, its reduction over the
+  // weight's rows
+  const int64_t Mdim = DG ? K : rows_per_mat;
+  const int64_t Kred = DG ? N : K;
+  const int64_t MT = (Mdim + BM - 1) / BM;
+  const int KB = int((Kred + BK - 1) / BK);
   const bool il = NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED;
   const uint32_t limit = (p.flags & E4B_FLAG_TEST_TIMEOUT) ? 0u : kWaitPolls;
 
@@ -254,7 +259,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             uint8_t* dst = smem + C::kC + (s * NMAT + m) * kCTileBytes;
-            if (il) {
+            if (DG) {
+              // 64 weight rows x 128 weight columns (64 bytes)
+              tma_load_2d(dst, &tmap_codes, &c_full[s], int32_t(T.mt * (BM / 2)),
+                          int32_t(int64_t(T.e) * N + int64_t(kb) * BK));
+            } else if (il) {
               tma_load_3d(dst, &tmap_codes, &c_full[s], kb * (BK / 2), m,
                           int32_t(int64_t(T.e) * rows_per_mat + T.mt * BM));
             } else {
@@ -271,7 +280,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      // dgrad: A is MN-major (bit 15, "transpose A")
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN) | (DG ? (1u << 15) : 0u);
       int64_t i = 0;
       uint64_t* last_bar = nullptr;
       uint32_t last_ph = 0;
@@ -300,8 +310,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
             const uint32_t abase = smem_u32(smem + C::kA + (as * NMAT + m) * kATileBytes);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              mma_bf16_ss(dcol + uint32_t(m * BN), sw128_kmajor_desc(abase + kk * 32),
-                          sw128_kmajor_desc(bbase + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+              const uint64_t adesc = DG ? sw128_mnmajor_desc(abase + kk * 2048, 8192, 1024)
+                                        : sw128_kmajor_desc(abase + kk * 32);
+              mma_bf16_ss(dcol + uint32_t(m * BN), adesc, sw128_kmajor_desc(bbase + kk * 32), idesc,
+                          (kb | kk) ? 1u : 0u);
             }
           }
           mma_commit(&a_empty[as]);
@@ -366,6 +378,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const int d = tid - 128;                  // 0..255
     const int m = NMAT == 2 ? (d >> 7) : 0;   // matrix (gate / up)
     const int r = d & 127;                    // row within the tile
+    // dgrad: weight row dr of the job's 64, columns 64 db .. 64 db + 63 of the tile
+    const int dr = r & 63, db = r >> 6;
     const int grp = NMAT == 2 ? 0 : (d >> 7); // NMAT == 1: two groups take alternate jobs
     constexpr int step = NMAT == 2 ? 1 : 2;
     const uint8_t* scales = static_cast<const uint8_t*>(p.scales);
@@ -379,6 +393,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       if (q >= njobs) return 0u;
       const int j = int(q / KB);
       const int kb = int(q % KB);
+      if constexpr (DG) {
+        // the absmax (or the two scale bytes) of weight row kb*64 + dr at
+        // columns 128 mt + 64 db ..; zero past the expert's rows or columns
+        // (those products meet zero-filled dy columns or unstored outputs)
+        if (j != cached_j) {
+          cached_j = j;
+          const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
+          const int64_t col0 = T.mt * BM + 64 * db;
+          srow = col0 < K ? scales + int64_t(T.e) * N * sstride + (FMT == E4B_FMT_NF4 ? (col0 / 64) * 4 : col0 / 32)
+                          : nullptr;
+        }
+        const int64_t wr = int64_t(kb) * BK + dr;
+        if (!srow || wr >= N) return 0u;
+        if constexpr (FMT == E4B_FMT_NF4) {
+          return __float_as_uint(__ldg(reinterpret_cast<const float*>(srow + wr * sstride)));
+        } else {
+          const uint8_t* sb = srow + wr * sstride;
+          return uint32_t(__ldg(sb)) | (uint32_t(__ldg(sb + 1)) << 8);
+        }
+      }
       if (j != cached_j) {
         cached_j = j;
         const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
@@ -414,8 +448,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           aborted = true;
           break;
         }
-        const uint4* crow =
-            reinterpret_cast<const uint4*>(smem + C::kC + (cs * NMAT + m) * kCTileBytes + r * 32);
+        const uint4* crow = reinterpret_cast<const uint4*>(
+            smem + C::kC + (cs * NMAT + m) * kCTileBytes + (DG ? dr * 64 + db * 32 : r * 32));
         const uint4 c0 = crow[0];
         const uint4 c1 = crow[1];
         // The slot's next fill is a TMA write (async proxy); without this
@@ -429,7 +463,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           break;
         }
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        uint8_t* arow = smem + C::kA + (as * NMAT + m) * kATileBytes + r * 128;
+        // K-major: the 128-byte row r of the tile. dgrad, MN-major: the
+        // 128-byte row of K index dr (8-row atoms of 1024 bytes) in the atom
+        // column db (8 KB apart); the same 128B swizzle by row within the atom.
+        const int sw = DG ? (dr & 7) : (r & 7);
+        uint8_t* arow = smem + C::kA + (as * NMAT + m) * kATileBytes +
+                        (DG ? db * 8192 + (dr >> 3) * 1024 + (dr & 7) * 128 : r * 128);
         Lut L;
         lut_build<FMT>(L, __uint_as_float(cur), cur & 0xFFu);
 #pragma unroll
@@ -437,7 +476,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           if (FMT == E4B_FMT_MXFP4 && c == 4) lut_build<FMT>(L, 0.f, (cur >> 8) & 0xFFu);
           uint32_t o[4];
           lut_decode8<FMT>(L, words[c], o);
-          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(arow + ((c ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(&a_full[as]);
@@ -456,7 +495,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       tc_fence_after();
       const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
       const int64_t n = T.mt * BM + rloc;
-      const bool nvalid = n < rows_per_mat;
+      const bool nvalid = n < Mdim;
       // bias of this thread's row(s): gate and up, or the single output row
       float b0 = 0.f, b1 = 0.f;
       if (p.bias && nvalid) {
@@ -483,7 +522,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           if constexpr (EPI == E4B_EPI_SWIGLU) {
             const float hv = glu_act(p.act, gv, __uint_as_float(u[t]) + b1, p.alpha, p.limit);
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(hv);
-          } else if constexpr (EPI == E4B_EPI_STORE) {
+          } else if constexpr (EPI == E4B_EPI_STORE || DG) {
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(gv);
           } else {
             const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
@@ -528,10 +567,22 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
   using C = Cfg<NMAT>;
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return cudaErrorInitializationError;
-  // Packed codes viewed as a 2-D byte tensor [E*N rows, K/2 bytes], or for
-  // interleaved gate/up rows as [E*I, 2, K/2] (boxes of 128 gate or up rows).
+  constexpr bool DG = EPI == kEpiDgrad;
+  // Packed codes viewed as a 2-D byte tensor [E*N rows, K/2 bytes] (dgrad:
+  // boxes of 64 rows x 128 weight columns), or for interleaved gate/up rows as
+  // [E*I, 2, K/2] (boxes of 128 gate or up rows).
   CUtensorMap tmap_codes;
-  if (NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED) {
+  if (DG) {
+    const cuuint64_t gdim[2] = {cuuint64_t(p.K / 2), cuuint64_t(int64_t(p.E) * p.N)};
+    const cuuint64_t gstride[1] = {cuuint64_t(p.K / 2)};
+    const cuuint32_t box[2] = {BM / 2, BK};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = enc(&tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.codes),
+                      gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  } else if (NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED) {
     const cuuint64_t gdim[3] = {cuuint64_t(p.K / 2), 2, cuuint64_t(int64_t(p.E) * (p.N / 2))};
     const cuuint64_t gstride[2] = {cuuint64_t(p.K / 2), cuuint64_t(p.K)};
     const cuuint32_t box[3] = {BK / 2, 1, BM};
@@ -554,11 +605,12 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
   }
   // Activations [rows, K] bf16 with row stride lda, landing 128B-swizzled:
   // single rows for the four-row gather, 256-row tiles for contiguous rows.
+  // dgrad: dy [rows, N], the reduction running over the weight's rows.
   CUtensorMap tmap_act;
   {
     const bool gather = p.row_slot != nullptr;
     const int64_t rows = gather ? (p.R_max + p.top_k - 1) / p.top_k : p.R_max;
-    const cuuint64_t gdim[2] = {cuuint64_t(p.K), cuuint64_t(rows)};
+    const cuuint64_t gdim[2] = {cuuint64_t(DG ? p.N : p.K), cuuint64_t(rows)};
     const cuuint64_t gstride[1] = {cuuint64_t(p.lda) * 2};
     const cuuint32_t box[2] = {BK, gather ? 1u : cuuint32_t(BN)};
     const cuuint32_t estride[2] = {1, 1};
@@ -580,7 +632,7 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
     configured_dev = dev;
   }
   const int64_t rows_per_mat = NMAT == 2 ? p.N / 2 : p.N;
-  const int64_t MT = (rows_per_mat + BM - 1) / BM;
+  const int64_t MT = ((DG ? p.K : rows_per_mat) + BM - 1) / BM;
   const int64_t max_tiles = MT * ((p.R_max + BN - 1) / BN + p.E);
   int grid = int(max_tiles < sms ? max_tiles : sms);
   if (grid < 1) grid = 1;
@@ -592,6 +644,11 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
 
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms) {
   if (p.E > kMaxE) return cudaErrorInvalidValue;
+  if (p.epilogue == kEpiDgrad) {
+    if (p.row_slot) return cudaErrorInvalidValue;  // dy rows are expert-ordered
+    return p.fmt == E4B_FMT_NF4 ? launch_t<E4B_FMT_NF4, kEpiDgrad>(p, st, sms)
+                                : launch_t<E4B_FMT_MXFP4, kEpiDgrad>(p, st, sms);
+  }
   if (p.fmt == E4B_FMT_NF4) {
     if (p.epilogue == E4B_EPI_SWIGLU) return launch_t<E4B_FMT_NF4, E4B_EPI_SWIGLU>(p, st, sms);
     if (p.epilogue == E4B_EPI_COMBINE) return launch_t<E4B_FMT_NF4, E4B_EPI_COMBINE>(p, st, sms);

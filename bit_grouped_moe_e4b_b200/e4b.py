@@ -36,7 +36,7 @@ FMT = {"nf4": E4B_FMT_NF4, "mxfp4": E4B_FMT_MXFP4}
 # Every symbol include/e4b.h declares.
 EXPORTED = [
     "e4b_quantize_nf4", "e4b_quantize_mxfp4", "e4b_dequantize", "e4b_nf4_codebook",
-    "e4b_route_workspace_size", "e4b_route", "e4b_grouped_gemm", "e4b_moe_workspace_size",
+    "e4b_route_workspace_size", "e4b_route", "e4b_grouped_gemm", "e4b_grouped_dgrad", "e4b_moe_workspace_size",
     "e4b_moe_forward", "e4b_moe_forward_noalloc", "e4b_read_device_status", "e4b_set_timing_events", "e4b_last_path",
     "e4b_last_launch_count",
     "e4b_status_string", "e4b_version",
@@ -73,6 +73,15 @@ class GemmArgs(ctypes.Structure):
     ]
 
 
+class DgradArgs(ctypes.Structure):
+    _fields_ = [
+        ("fmt", ctypes.c_int32), ("E", ctypes.c_int32), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("R_max", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("dy", ctypes.c_void_p), ("ld_dy", ctypes.c_int64), ("offsets", ctypes.c_void_p),
+        ("dx", ctypes.c_void_p), ("ld_dx", ctypes.c_int64),
+    ]
+
+
 # expert-variant codes (include/e4b.h)
 LAYOUT = {"halves": 0, "interleaved": 1}
 ACT = {"swiglu": 0, "clamped_glu": 1}
@@ -99,6 +108,7 @@ def lib() -> ctypes.CDLL:
         "e4b_route_workspace_size": [i64, i32, i32, ctypes.POINTER(sz)],
         "e4b_route": [vp, i64, i32, i32, vp, vp, vp, vp, vp, sz, vp],
         "e4b_grouped_gemm": [ctypes.POINTER(GemmArgs), ctypes.c_uint32, vp],
+        "e4b_grouped_dgrad": [ctypes.POINTER(DgradArgs), ctypes.c_uint32, vp],
         "e4b_moe_workspace_size": [ctypes.POINTER(MoeWeights), i64, i32, ctypes.POINTER(sz)],
         "e4b_moe_forward": [ctypes.POINTER(MoeWeights), vp, i64, i32, vp, vp, vp, vp, sz,
                             ctypes.c_uint32, vp],
@@ -220,6 +230,16 @@ def route(ids: torch.Tensor, E: int):
 
 
 # --------------------------------------------------------------- grouped GEMM
+def e4b_grouped_dgrad(fmt, codes, scales, dy, offsets, dx, *, E, N, K, R_max, flags=0, stream=None):
+    """dx[p] = dy[p] . W_e for the routed rows p of each expert (dy [R, N],
+    dx [R, K], bf16, rows in expert order)."""
+    _dev(codes, scales, dy, offsets, dx)
+    args = DgradArgs(FMT.get(fmt, fmt), E, N, K, R_max, _ptr(codes), _ptr(scales), _ptr(dy), dy.shape[-1],
+                     _ptr(offsets), _ptr(dx), dx.shape[-1])
+    _check(lib().e4b_grouped_dgrad(ctypes.byref(args), flags, _stream(stream)), "e4b_grouped_dgrad")
+
+
+
 def e4b_grouped_gemm(fmt, epilogue, codes, scales, a, offsets, out, *, E, N, K, R_max, top_k=1,
                      a_row_slot=None, out_row_slot=None, gates=None, flags=0, stream=None,
                      layout="halves", act="swiglu", alpha=1.702, limit=7.0, bias=None):

@@ -249,6 +249,34 @@ typedef struct {
 
 e4b_status e4b_grouped_gemm(const e4b_gemm_args* args, uint32_t flags, void* stream);
 
+/*
+ * e4b_grouped_dgrad -- [G] entry table (the NF4 grouped GEMM's backward,
+ * dgrad_4bit_grouped): the input gradient through the packed weights, in one
+ * launch over all active experts. For routed row p of expert e (offsets[e] <=
+ * p < offsets[e+1]):  dx[p] = dy[p] . W_e  (the contraction over the weight's
+ * rows), fp32 accumulation, bf16 output. W_e is decoded as in e4b_grouped_gemm
+ * (NF4 bf16_rne(fp32(level * absmax)), MXFP4 exact); no bf16 weight tensor is
+ * stored. Runs on the tcgen05 path (E <= 256); flags: 0 (E4B_FLAG_FORCE_GEMV
+ * returns E4B_ERR_UNSUPPORTED). Shapes: K % 64 == 0 (NF4) or K % 32 == 0
+ * (MXFP4); N any. dy, codes, dx 16-byte aligned; ld_dy >= N and ld_dx >= K,
+ * both multiples of 8. Rows p >= offsets[E] of dx are not written.
+ */
+typedef struct {
+  int32_t fmt; /* e4b_format */
+  int32_t E;
+  int64_t N, K;          /* each expert's weight W_e is [N, K], packed along K (as the forward) */
+  int64_t R_max;         /* bound on offsets[E] (rows of dy and dx) */
+  const uint8_t* codes;  /* the packed stack [E, N, ...] as in e4b_gemm_args */
+  const void* scales;
+  const uint16_t* dy;    /* bf16 [R, N], rows in expert order */
+  int64_t ld_dy;         /* elements between rows of dy */
+  const int64_t* offsets; /* [E+1] */
+  uint16_t* dx;          /* bf16 [R, K] */
+  int64_t ld_dx;         /* elements between rows of dx */
+} e4b_dgrad_args;
+
+e4b_status e4b_grouped_dgrad(const e4b_dgrad_args* args, uint32_t flags, void* stream);
+
 /* ---------------------------------------------------------- whole layer */
 
 /* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots.

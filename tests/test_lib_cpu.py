@@ -123,7 +123,7 @@ def test_variant_argument_checks():
 def test_binding_structs_match_the_header(tmp_path):
     # sizes and field offsets of the two argument structs, as a C compiler
     # lays them out from include/e4b.h, against the ctypes mirrors
-    structs = {"e4b_moe_weights": e4b.MoeWeights, "e4b_gemm_args": e4b.GemmArgs}
+    structs = {"e4b_moe_weights": e4b.MoeWeights, "e4b_gemm_args": e4b.GemmArgs, "e4b_dgrad_args": e4b.DgradArgs}
     src = ["#include <stdio.h>", "#include <stddef.h>", '#include "e4b.h"', "int main(void) {"]
     for cname, py in structs.items():
         src.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
@@ -143,3 +143,26 @@ def test_binding_structs_match_the_header(tmp_path):
         assert got[(cname, "sizeof")] == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
             assert got[(cname, f)] == getattr(py, f).offset, (cname, f)
+
+
+def test_dgrad_argument_checks():
+    L = e4b.lib()
+    p = 4096
+
+    def call(**kw):
+        a = e4b.DgradArgs(0, 4, 256, 128, 64, p, p, p, 256, p, p, 128)
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return L.e4b_grouped_dgrad(ctypes.byref(a), 0, None)
+
+    assert call(fmt=7) == 1
+    assert call(K=96) == 2            # NF4 needs K % 64
+    assert call(E=300) == 2           # tcgen05 table holds 256 experts
+    assert call(dy=4100) == 7
+    assert call(ld_dy=200) == 1       # ld_dy < N
+    assert call(ld_dx=100) == 7       # not a multiple of 8
+    assert call(dx=None) == 1
+    a = e4b.DgradArgs(0, 4, 256, 128, 0, p, p, p, 256, p, p, 128)
+    assert L.e4b_grouped_dgrad(ctypes.byref(a), 0, None) == 0  # no rows: nothing to do
+    a = e4b.DgradArgs(0, 4, 256, 128, 64, p, p, p, 256, p, p, 128)
+    assert L.e4b_grouped_dgrad(ctypes.byref(a), e4b.FLAG_FORCE_GEMV, None) == 2
