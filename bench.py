@@ -51,6 +51,9 @@ def _args():
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per workload and token count (no cpu baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["forward", "dgrad"], default="forward",
+                    help="dgrad: time e4b_grouped_dgrad, the input gradients of both projections "
+                         "(one JSON line, TFLOP/s)")
     return ap.parse_args()
 
 
@@ -315,6 +318,76 @@ def oracle_sample(wl, T, ids, gates, x_h, slots):
     return time.perf_counter() - t
 
 
+def run_dgrad(wl, T, steps, warmup, bf16, bf16_sus, peak_src):
+    """Times the input gradients through the packed weights of both
+    projections of the workload's layer on its routed rows (expert order):
+    gate_up: dx [R, H] = dGU [R, 2I] . W_gu;  down: dh [R, I] = dO [R, H] . W_d.
+    dy values are N(0, 1) rounded to bf16. Returns one JSON-ready dict."""
+    import torch
+    from bit_grouped_moe_e4b_b200 import e4b, synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layer = build_layer(wl, dev)
+    ids_h, _ = synth.routing(wl, T)
+    _, offsets, _, _, _ = e4b.route(torch.from_numpy(ids_h).to(dev), wl.E)
+    R = ids_h.size
+    g = torch.Generator(device=dev).manual_seed(wl.seed + 7)
+    d_gu = torch.randn((R, 2 * wl.I), generator=g, device=dev).to(torch.bfloat16)
+    d_dn = torch.randn((R, wl.H), generator=g, device=dev).to(torch.bfloat16)
+    dx = torch.empty((R, wl.H), dtype=torch.bfloat16, device=dev)
+    dh = torch.empty((R, wl.I), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        e4b.e4b_grouped_dgrad(wl.fmt, layer.gate_up_codes, layer.gate_up_scales, d_gu, offsets, dx, E=wl.E,
+                              N=2 * wl.I, K=wl.H, R_max=R)
+        if ev:
+            ev[1].record(stream)
+        e4b.e4b_grouped_dgrad(wl.fmt, layer.down_codes, layer.down_scales, d_dn, offsets, dh, E=wl.E,
+                              N=wl.H, K=wl.I, R_max=R)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / steps
+    gu_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    dn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    f_gu = 2.0 * R * 2 * wl.I * wl.H
+    f_dn = 2.0 * R * wl.H * wl.I
+    dom, dom_ms, dom_f = ("gate_up_dgrad", gu_ms, f_gu) if gu_ms >= dn_ms else ("down_dgrad", dn_ms, f_dn)
+    achieved = dom_f / (dom_ms * 1e-3) / 1e12
+    return {
+        "metric": "grouped dgrad TFLOP/s (input gradients of both projections, packed weights)",
+        "value": (f_gu + f_dn) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "T": T, "routed_rows": R, "format": wl.fmt, "E": wl.E, "H": wl.H,
+                   "I": wl.I, "op": "dgrad", "l2": "no flush: packed weights exceed the 126 MB L2"},
+        "phases_ms": {"gate_up_dgrad": gu_ms, "down_dgrad": dn_ms},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                     "frac": achieved / bf16, "peak_source": peak_src + " (burst)", "peak_sustained": bf16_sus,
+                     "traffic": None, "algorithmic_flops": dom_f},
+        "clocks": clk,
+        "gpu_launches": 2 * steps,
+    }
+
+
 def run_reference(args, wl, T):
     from bit_grouped_moe_e4b_b200 import synth
 
@@ -372,6 +445,12 @@ def main():
                                  device_id=torch.device("cuda", local))
         dist = tdist
     hbm, bf16, bf16_sus, peak_src = _peaks()
+
+    if args.op == "dgrad":
+        line = run_dgrad(wl, T, args.steps, args.warmup, bf16, bf16_sus, peak_src)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
 
     cases = [(wl, T)]
     if args.sweep:
