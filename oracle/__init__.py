@@ -22,6 +22,10 @@ Sources (page titles; sections):
   * bitsandbytes PR #1984 "Experts4bit", Summary / Design / Benchmark Results:
     per-expert quantisation with per-expert absmax, the per-expert dequantise
     loop, the gated SiLU (SwiGLU) activation, MAE / RMSE of NF4.
+  * "How do I run a single-token INT4 decode GEMV over routed MoE experts, and
+    pack calibrated (GPTQ) weights for it?" (grouped-nf4-gemm solutions page):
+    the int4-b32 decode GEMV with exact integer accumulation and the GPTQ
+    packer (module ``int4b32``).
   * "experts4bit-qlora" README: fused ``gate_up_proj [E, 2I, H]`` and
     ``down_proj [E, H, I]`` expert stacks (transformers v5 layout).
 
@@ -48,6 +52,7 @@ from .formats import (
 )
 from .moe import (route_ref, moe_forward_ref, swiglu_ref, expert_tokens, clamped_glu_ref,
                   split_gate_up, activation_ref, grouped_projection_ref, grouped_dgrad_ref)
+from . import int4b32
 
 __all__ = [
     "NF4_BLOCK", "MXFP4_BLOCK", "E2M1_MAGNITUDES",
@@ -56,5 +61,5 @@ __all__ = [
     "dequant_ref_exact", "dequant_ref_level", "quantize_pack_mxfp4", "unpack_mxfp4_codes",
     "dequant_mxfp4", "packed_bytes_per_weight",
     "route_ref", "moe_forward_ref", "swiglu_ref", "expert_tokens", "clamped_glu_ref", "split_gate_up",
-    "activation_ref", "grouped_projection_ref", "grouped_dgrad_ref",
+    "activation_ref", "grouped_projection_ref", "grouped_dgrad_ref", "int4b32",
 ]
