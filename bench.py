@@ -51,9 +51,10 @@ def _args():
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per workload and token count (no cpu baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["forward", "dgrad"], default="forward",
+    ap.add_argument("--op", choices=["forward", "dgrad", "int4"], default="forward",
                     help="dgrad: time e4b_grouped_dgrad, the input gradients of both projections "
-                         "(one JSON line, TFLOP/s)")
+                         "(one JSON line, TFLOP/s); int4: the int4-b32 decode GEMVs of one token "
+                         "through the workload's layer (one JSON line, packed-weight GB/s)")
     return ap.parse_args()
 
 
@@ -388,6 +389,149 @@ def run_dgrad(wl, T, steps, warmup, bf16, bf16_sus, peak_src):
     }
 
 
+def run_int4(wl, steps, warmup, hbm, peak_src, cpu_baseline=True):
+    """Times one token through the workload's layer on int4-b32 stacks (the
+    same N(0, 0.02) fp32 weights, packed by e4b_quantize_int4_b32): the gate_up
+    GEMV with the SwiGLU epilogue, then the down GEMV with the combine. Step i
+    routes the token to the i-th of four disjoint expert pairs, so consecutive
+    steps read different weights (no L2 reuse across steps). Returns one
+    JSON-ready dict."""
+    import torch
+    from bit_grouped_moe_e4b_b200 import e4b, synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    E, H, I = wl.E, wl.H, wl.I
+    stacks = []
+    for which in ("gate_up", "down"):
+        w = synth.layer_weights(wl, which, dev)
+        stacks += list(e4b.quantize_int4_b32(w))
+        del w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    gc, gs, dc, ds = stacks
+    x_h = synth.tokens_bf16(wl, 1)[0].contiguous()
+    pairs = [[(2 * i + 1) % E, (2 * i) % E] for i in range(E // 2)]
+    gates_h = np.array([0.62, 0.38], np.float32)
+    ids_d = [torch.tensor(p, dtype=torch.int32, device=dev) for p in pairs]
+    g_d = torch.from_numpy(gates_h).to(dev)
+    x = x_h.to(dev)
+    h = torch.empty((2, I), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((H,), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None, xin=x, ids=None):
+        ids = ids_d[i % len(ids_d)] if ids is None else ids
+        if ev:
+            ev[0].record(stream)
+        e4b.e4b_gemv_int4_b32("swiglu", gc, gs, ids, xin, h, E=E, N=2 * I, K=H, ld_y=I)
+        if ev:
+            ev[1].record(stream)
+        e4b.e4b_gemv_int4_b32("combine", dc, ds, ids, h, y, E=E, N=H, K=I, gates=g_d, ld_x=I)
+        if ev:
+            ev[2].record(stream)
+
+    for i in range(max(warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for row in ev:
+        for e_ in row:
+            e_.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    # a step takes less GPU time than its two host calls: a sleep kernel ahead
+    # of the timed region lets the host queue every step first, so the events
+    # time the GPU, not the host (the e2e number below keeps the host in)
+    torch.cuda._sleep(int(5e7))
+    t0.record(stream)
+    for i in range(steps):
+        step(i, ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / steps
+    gu_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    dn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    bpw = 0.5 + 2.0 / 32
+    gu_bytes = 2 * 2 * I * H * bpw + 2 * H + 2 * 2 * I      # two experts' gate_up, x in, h out
+    dn_bytes = 2 * H * I * bpw + 2 * 2 * I + 2 * H          # two experts' down, h in, y out
+    dom, dom_ms, dom_b = ("int4_gemv_gate_up", gu_ms, gu_bytes) if gu_ms >= dn_ms else \
+        ("int4_gemv_down", dn_ms, dn_bytes)
+    achieved = dom_b / (dom_ms * 1e-3) / 1e9
+
+    # end to end through the public call with host buffers: x, ids and gates
+    # in from pinned memory, y out, every step
+    x_pin = x_h.pin_memory()
+    ids_pin = [torch.tensor(p, dtype=torch.int32).pin_memory() for p in pairs]
+    g_pin = torch.from_numpy(gates_h).pin_memory()
+    y_pin = torch.empty((H,), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x)
+    idd = torch.empty(2, dtype=torch.int32, device=dev)
+
+    def e2e_step(i):
+        xd.copy_(x_pin, non_blocking=True)
+        idd.copy_(ids_pin[i % len(ids_pin)], non_blocking=True)
+        g_d.copy_(g_pin, non_blocking=True)
+        step(i, xin=xd, ids=idd)
+        y_pin.copy_(y, non_blocking=True)
+
+    for i in range(max(warmup, 3)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / steps
+    line = {
+        "metric": "int4-b32 decode: packed-weight HBM GB/s of one token through the MoE layer (GEMVs)",
+        "value": (gu_bytes + dn_bytes) / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": steps,
+        "warmup": max(warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8xint4->int32", "data": "synthetic",
+        "tokens_per_s": 1.0 / (ms * 1e-3),
+        "config": {"workload": wl.name + "_int4b32_T1", "format": "int4-b32 (fp16 scale per 32)", "E": E, "H": H,
+                   "I": I, "top_k": 2, "op": "int4",
+                   "routing": "step i: the i-th of four disjoint expert pairs, gates 0.62/0.38",
+                   "l2": "no flush: each step reads two experts not read by the step before "
+                         f"({(gu_bytes + dn_bytes) / 2 ** 20:.0f} MiB a step, 4 steps before a pair repeats)"},
+        "phases_ms": {"int4_gemv_gate_up": gu_ms, "int4_gemv_down": dn_ms},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": peak_src, "traffic": _traffic(wl.name + "_int4", dom),
+                     "algorithmic_bytes": dom_b},
+        "clocks": clk,
+        "e2e": {"value": (gu_bytes + dn_bytes) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "tokens_per_s": 1.0 / (e2e_ms * 1e-3),
+                "h2d_bytes_per_step": x_h.numel() * 2 + 8 + 8, "d2h_bytes_per_step": H * 2},
+        "gpu_launches": 2 * steps,
+    }
+    if cpu_baseline:
+        from oracle import int4b32 as q4
+
+        e_pair = pairs[0]
+        gcs, gss, dcs, dss = [], [], [], []
+        for e in e_pair:
+            a, b = q4.quantize_int4b32(synth.expert_weight(wl, "gate_up", e, dev).cpu().numpy())
+            gcs.append(a), gss.append(b)
+            a, b = q4.quantize_int4b32(synth.expert_weight(wl, "down", e, dev).cpu().numpy())
+            dcs.append(a), dss.append(b)
+        gcs, gss, dcs, dss = np.stack(gcs), np.stack(gss), np.stack(dcs), np.stack(dss)
+        tc = time.perf_counter()
+        q4.int4b32_decode_layer_ref(x_h.float().numpy(), [0, 1], gates_h, gcs, gss, dcs, dss)
+        secs = time.perf_counter() - tc
+        line["cpu_baseline"] = {"value": (gu_bytes + dn_bytes) / secs / 1e9, "unit": "GB/s",
+                                "tokens_per_s": 1.0 / secs, "cores": 1, "kind": "oracle",
+                                "sample": "one token through the layer on one expert pair (numpy oracle, "
+                                          "weights packed before timing)"}
+    return line
+
+
 def run_reference(args, wl, T):
     from bit_grouped_moe_e4b_b200 import synth
 
@@ -448,6 +592,12 @@ def main():
 
     if args.op == "dgrad":
         line = run_dgrad(wl, T, args.steps, args.warmup, bf16, bf16_sus, peak_src)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
+    if args.op == "int4":
+        line = run_int4(wl, args.steps, args.warmup, hbm, peak_src,
+                        cpu_baseline=not args.no_cpu_baseline and rank == 0)
         if rank == 0:
             print(json.dumps(line), flush=True)
         return

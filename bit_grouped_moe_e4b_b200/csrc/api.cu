@@ -286,6 +286,82 @@ e4b_status e4b_grouped_dgrad(const e4b_dgrad_args* a, uint32_t flags, void* stre
   return cuda_status(launch_tc_gemm(p, static_cast<cudaStream_t>(stream), sm_count()));
 }
 
+e4b_status e4b_quantize_int4_b32(const float* w, int64_t E, int64_t N, int64_t K, uint8_t* codes,
+                                 uint16_t* scales, void* stream) {
+  if (E < 0 || N < 0 || K < 0) return E4B_ERR_INVALID_ARG;
+  if (K % E4B_INT4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  const int64_t nblocks = E * N * (K / E4B_INT4_BLOCK);
+  g_last_launches = 0;
+  if (nblocks == 0) return E4B_OK;
+  if (!w || !codes || !scales) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u)) return E4B_ERR_MISALIGNED;
+  g_last_launches = 1;
+  return cuda_status(launch_quantize_int4(w, nblocks, codes, scales, static_cast<cudaStream_t>(stream),
+                                          sm_count()));
+}
+
+e4b_status e4b_gptq_pack_int4_b32(const int32_t* qweight, const uint16_t* gptq_scales, int64_t E,
+                                  int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                                  void* stream) {
+  if (E < 0 || N < 0 || K < 0) return E4B_ERR_INVALID_ARG;
+  if (K % E4B_INT4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (E > 65535 || (N + 31) / 32 > 0x7FFFFFFF || K / 256 + 1 > 65535) return E4B_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (E == 0 || N == 0 || K == 0) return E4B_OK;
+  if (!qweight || !gptq_scales || !codes || !scales) return E4B_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(qweight) & 3u) || (reinterpret_cast<uintptr_t>(codes) & 3u) ||
+      (reinterpret_cast<uintptr_t>(gptq_scales) & 1u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return E4B_ERR_MISALIGNED;
+  g_last_launches = 2;
+  return cuda_status(launch_gptq_repack(qweight, gptq_scales, E, N, K, codes, scales,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+e4b_status e4b_gemv_int4_b32(const e4b_int4_gemv_args* a, uint32_t flags, void* stream) {
+  if (!a || (flags & ~E4B_FLAG_TEST_TIMEOUT)) return E4B_ERR_INVALID_ARG;
+  if (a->epilogue != E4B_EPI_STORE && a->epilogue != E4B_EPI_SWIGLU && a->epilogue != E4B_EPI_COMBINE)
+    return E4B_ERR_INVALID_ARG;
+  if (a->E <= 0 || a->N <= 0 || a->K <= 0 || a->n_slots <= 0 || a->ld_x < 0) return E4B_ERR_INVALID_ARG;
+  if (a->n_slots > int4_gemv_max_slots()) return E4B_ERR_UNSUPPORTED;
+  if (a->K % E4B_INT4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  if (a->epilogue == E4B_EPI_SWIGLU && a->N % 2) return E4B_ERR_INVALID_ARG;
+  if (!a->codes || !a->scales || !a->expert_ids || !a->x || !a->y) return E4B_ERR_INVALID_ARG;
+  if (a->epilogue == E4B_EPI_COMBINE && !a->gates) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(a->codes) || !aligned16(a->x) || (reinterpret_cast<uintptr_t>(a->y) & 1u) ||
+      (reinterpret_cast<uintptr_t>(a->scales) & 1u) || a->ld_x % 8)
+    return E4B_ERR_MISALIGNED;
+  if (a->ld_x != 0 && a->ld_x < a->K) return E4B_ERR_INVALID_ARG;
+  if (a->epilogue == E4B_EPI_STORE && a->ld_y < a->N) return E4B_ERR_INVALID_ARG;
+  if (a->epilogue == E4B_EPI_SWIGLU && a->ld_y < a->N / 2) return E4B_ERR_INVALID_ARG;
+  const int nx = a->ld_x == 0 ? 1 : a->n_slots;
+  if (int64_t(nx) * a->K > 200 * 1024) return E4B_ERR_UNSUPPORTED;
+  // outputs and items are counted in 32 bits
+  const int64_t outputs = a->epilogue == E4B_EPI_COMBINE ? a->N : int64_t(a->n_slots) * ((a->N + 1) / 2);
+  if (outputs * ((a->n_slots + 1) / 2) * ((a->K / E4B_INT4_BLOCK + 127) / 128) >= (int64_t(1) << 31))
+    return E4B_ERR_UNSUPPORTED;
+  Int4Gemv p{};
+  p.epilogue = a->epilogue;
+  p.E = a->E;
+  p.n_slots = a->n_slots;
+  p.nx = nx;
+  p.N = a->N;
+  p.K = a->K;
+  p.codes = a->codes;
+  p.scales = a->scales;
+  p.ids = a->expert_ids;
+  p.gates = a->gates;
+  p.x = a->x;
+  p.ld_x = a->ld_x;
+  p.y = a->y;
+  p.ld_y = a->ld_y;
+  p.status = a->status;
+  p.flags = flags;
+  if (int4_gemv_warps(nx, a->K) <= 0) return E4B_ERR_UNSUPPORTED;
+  g_last_path = E4B_PATH_INT4_GEMV;
+  g_last_launches = 1;
+  return cuda_status(launch_int4_gemv(p, static_cast<cudaStream_t>(stream), sm_count()));
+}
+
 e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
                                   size_t* bytes) {
   if (!w || !bytes || T < 0 || top_k <= 0 || w->E <= 0 || w->H <= 0 || w->I <= 0)

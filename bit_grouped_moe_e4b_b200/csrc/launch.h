@@ -91,4 +91,41 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms);
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms);
 cudaError_t launch_finalize(const float* acc, int64_t n, uint16_t* y, cudaStream_t st, int sms);
 
+// The int4-b32 decode GEMV (csrc/int4.cu): one token against n_slots routed
+// experts of a stack [E, N, K] (codes [E, N, K/2], fp16 scales [E, N, K/32]).
+// nx activation rows: 1 (every slot reads x) or n_slots (slot j reads row j).
+struct Int4Gemv {
+  int epilogue;  // E4B_EPI_STORE / E4B_EPI_SWIGLU / E4B_EPI_COMBINE
+  int E, n_slots, nx;
+  int64_t N, K;
+  const uint8_t* codes;
+  const uint16_t* scales;
+  const int32_t* ids;
+  const float* gates;
+  const uint16_t* x;
+  int64_t ld_x;
+  uint16_t* y;
+  int64_t ld_y;
+  int32_t* status;
+  uint32_t flags;
+};
+// Launch plan of the GEMV (csrc/int4.cu), made on the host.
+struct Int4Plan {
+  int warps;         // streaming warps per CTA
+  uint32_t nch;      // chunks of 128 blocks per weight row
+  uint32_t np;       // tasks per output (COMBINE: slot pairs)
+  int64_t outputs;
+  uint32_t acc_off, ring_off;  // shared-memory offsets
+  uint32_t polls;    // bound of every wait
+  uint32_t sbulk;    // 1: scales travel with the codes in the bulk copies (K % 256 == 0, aligned)
+};
+size_t int4_gemv_smem_bytes(int nx, int64_t K, int warps);
+int int4_gemv_warps(int nx, int64_t K);
+int int4_gemv_max_slots();
+cudaError_t launch_int4_gemv(const Int4Gemv& p, cudaStream_t st, int sms);
+cudaError_t launch_quantize_int4(const float* w, int64_t nblocks, uint8_t* codes, uint16_t* scales,
+                                 cudaStream_t st, int sms);
+cudaError_t launch_gptq_repack(const int32_t* qweight, const uint16_t* gscales, int64_t E, int64_t N, int64_t K,
+                               uint8_t* codes, uint16_t* scales, cudaStream_t st);
+
 }  // namespace e4b

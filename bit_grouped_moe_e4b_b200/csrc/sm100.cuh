@@ -66,6 +66,18 @@ E4B_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit,
   }
 }
 
+// Non-tensor bulk copy of `bytes` contiguous bytes, global -> this CTA's shared
+// memory, completing on `bar` (both addresses 16-byte aligned, bytes % 16 == 0).
+E4B_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+E4B_DEV void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // ------------------------------------------------------------------ TMA
 E4B_DEV void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y) {
   asm volatile(

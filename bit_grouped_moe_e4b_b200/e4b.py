@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libe4b.so")
 E4B_OK = 0
 E4B_FMT_NF4, E4B_FMT_MXFP4 = 0, 1
 E4B_EPI_STORE, E4B_EPI_SWIGLU, E4B_EPI_COMBINE = 0, 1, 2
-E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05 = 0, 1, 2
+E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05, E4B_PATH_INT4_GEMV = 0, 1, 2, 3
 FLAG_FORCE_GEMV = 0x1
 FLAG_FORCE_TCGEN05 = 0x2
 FLAG_TEST_TIMEOUT = 0x4
@@ -40,7 +40,9 @@ EXPORTED = [
     "e4b_moe_forward", "e4b_moe_forward_noalloc", "e4b_read_device_status", "e4b_set_timing_events", "e4b_last_path",
     "e4b_last_launch_count",
     "e4b_status_string", "e4b_version",
+    "e4b_quantize_int4_b32", "e4b_gptq_pack_int4_b32", "e4b_gemv_int4_b32",
 ]
+EPI = {"store": E4B_EPI_STORE, "swiglu": E4B_EPI_SWIGLU, "combine": E4B_EPI_COMBINE}
 
 
 class E4BError(RuntimeError):
@@ -82,6 +84,15 @@ class DgradArgs(ctypes.Structure):
     ]
 
 
+class Int4GemvArgs(ctypes.Structure):
+    _fields_ = [
+        ("epilogue", ctypes.c_int32), ("E", ctypes.c_int32), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("n_slots", ctypes.c_int32), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("expert_ids", ctypes.c_void_p), ("gates", ctypes.c_void_p), ("x", ctypes.c_void_p),
+        ("ld_x", ctypes.c_int64), ("y", ctypes.c_void_p), ("ld_y", ctypes.c_int64), ("status", ctypes.c_void_p),
+    ]
+
+
 # expert-variant codes (include/e4b.h)
 LAYOUT = {"halves": 0, "interleaved": 1}
 ACT = {"swiglu": 0, "clamped_glu": 1}
@@ -120,6 +131,9 @@ def lib() -> ctypes.CDLL:
         "e4b_last_launch_count": [],
         "e4b_status_string": [i32],
         "e4b_version": [],
+        "e4b_quantize_int4_b32": [vp, i64, i64, i64, vp, vp, vp],
+        "e4b_gptq_pack_int4_b32": [vp, vp, i64, i64, i64, vp, vp, vp],
+        "e4b_gemv_int4_b32": [ctypes.POINTER(Int4GemvArgs), ctypes.c_uint32, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -203,6 +217,59 @@ def dequantize(fmt: str, codes, scales, E, N, K):
 
 
 # ------------------------------------------------------------------ routing
+# ------------------------------------------------------------- int4-b32
+def e4b_quantize_int4_b32(w, codes, scales, stream=None):
+    """fp32 w [E, N, K] -> codes uint8 [E, N, K/2], scales fp16 [E, N, K/32]."""
+    _dev(w, codes, scales)
+    E, N, K = w.shape
+    _check(lib().e4b_quantize_int4_b32(_ptr(w), E, N, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "e4b_quantize_int4_b32")
+
+
+def e4b_gptq_pack_int4_b32(qweight, gptq_scales, codes, scales, *, E, N, K, stream=None):
+    """GPTQ qweight int32 [E, K/8, N] + scales fp16 [E, K/32, N] -> int4-b32 codes/scales."""
+    _dev(qweight, gptq_scales, codes, scales)
+    _check(lib().e4b_gptq_pack_int4_b32(_ptr(qweight), _ptr(gptq_scales), E, N, K, _ptr(codes), _ptr(scales),
+                                        _stream(stream)), "e4b_gptq_pack_int4_b32")
+
+
+def e4b_gemv_int4_b32(epilogue, codes, scales, expert_ids, x, y, *, E, N, K, gates=None, ld_x=0, ld_y=None,
+                      status=None, flags=0, stream=None):
+    """The int4-b32 decode GEMV of one token over its routed experts (include/e4b.h)."""
+    _dev(codes, scales, expert_ids, x, y, gates, status)
+    epi = EPI.get(epilogue, epilogue)
+    n_slots = expert_ids.numel()
+    if ld_y is None:
+        ld_y = N // 2 if epi == E4B_EPI_SWIGLU else N
+    a = Int4GemvArgs(epi, E, N, K, n_slots, codes.data_ptr(), scales.data_ptr(), expert_ids.data_ptr(),
+                     None if gates is None else gates.data_ptr(), x.data_ptr(), ld_x, y.data_ptr(), ld_y,
+                     None if status is None else status.data_ptr())
+    _check(lib().e4b_gemv_int4_b32(ctypes.byref(a), flags, _stream(stream)), "e4b_gemv_int4_b32")
+
+
+def quantize_int4_b32(w: torch.Tensor):
+    """Packs fp32 weights [E, N, K] into int4-b32 on the GPU; returns (codes, scales)."""
+    E, N, K = w.shape
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((E, N, K // 32), dtype=torch.float16, device=w.device)
+    e4b_quantize_int4_b32(w, codes, scales)
+    return codes, scales
+
+
+def int4_decode_layer(x, expert_ids, gates, gu_codes, gu_scales, dn_codes, dn_scales, *, E, H, I, h=None, y=None):
+    """One token through the MoE layer on int4-b32 stacks: the gate_up GEMV
+    with the SwiGLU epilogue (h [k, I]), then the down GEMV with the combine
+    epilogue (y [H]). Two launches; returns y."""
+    k = expert_ids.numel()
+    if h is None:
+        h = torch.empty((k, I), dtype=torch.bfloat16, device=x.device)
+    if y is None:
+        y = torch.empty((H,), dtype=torch.bfloat16, device=x.device)
+    e4b_gemv_int4_b32("swiglu", gu_codes, gu_scales, expert_ids, x, h, E=E, N=2 * I, K=H, ld_y=I)
+    e4b_gemv_int4_b32("combine", dn_codes, dn_scales, expert_ids, h, y, E=E, N=H, K=I, gates=gates, ld_x=I)
+    return y
+
+
 def e4b_route_workspace_size(T, top_k, E) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().e4b_route_workspace_size(T, top_k, E, ctypes.byref(n)), "e4b_route_workspace_size")

@@ -22,6 +22,9 @@
  *        gated SiLU / SwiGLU activation).
  *   [Q]  "experts4bit-qlora" README: fused gate_up_proj / down_proj stacks
  *        (transformers v5 layout).
+ *   [S]  "How do I run a single-token INT4 decode GEMV over routed MoE
+ *        experts, and pack calibrated (GPTQ) weights for it?" (grouped-nf4-gemm
+ *        solutions page): the int4-b32 decode GEMV and the GPTQ packer.
  *
  * Conventions for every entry point
  *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
@@ -68,7 +71,8 @@ typedef enum { E4B_FMT_NF4 = 0, E4B_FMT_MXFP4 = 1 } e4b_format;
 typedef enum {
   E4B_PATH_NONE = 0,
   E4B_PATH_GEMV = 1,   /* small-M: register-fed mma.sync streaming the packed bytes */
-  E4B_PATH_TCGEN05 = 2 /* large-M: TMA + on-the-fly decode + tcgen05 MMA into TMEM */
+  E4B_PATH_TCGEN05 = 2, /* large-M: TMA + on-the-fly decode + tcgen05 MMA into TMEM */
+  E4B_PATH_INT4_GEMV = 3 /* the int4-b32 decode GEMV (dp4a, exact integer block sums) */
 } e4b_path;
 
 /* Flags for e4b_moe_forward / e4b_grouped_gemm. */
@@ -276,6 +280,87 @@ typedef struct {
 } e4b_dgrad_args;
 
 e4b_status e4b_grouped_dgrad(const e4b_dgrad_args* args, uint32_t flags, void* stream);
+
+/* ---------------------------------------------------- int4-b32 (decode) */
+/*
+ * [S] "How do I run a single-token INT4 decode GEMV over routed MoE experts,
+ * and pack calibrated (GPTQ) weights for it?" (grouped-nf4-gemm solutions
+ * page): the batch-1 int4-b32 decode GEMV with exact integer accumulation and
+ * the packer of calibrated weights onto the same bytes; [G] README table row
+ * "int4-b32 decode GEMV, dense M=1". The pages do not print the encoding;
+ * the library's reading:
+ *   stack [E, N, K] as codes uint8 [E, N, K/2] (signed 4-bit q in [-8, 7],
+ *   two's complement, the earlier weight in the LOW nibble) and scales fp16
+ *   (bit patterns, uint16_t) [E, N, K/32]; weight = s * q. K % 32 == 0.
+ */
+#define E4B_INT4_BLOCK 32
+#define E4B_INT4_MAX_SLOTS 64
+
+/*
+ * e4b_quantize_int4_b32 -- fp32 w [E, N, K] (16-byte aligned, K % 32 == 0)
+ * -> codes [E, N, K/2] (16-byte aligned) and scales [E, N, K/32]: per 32
+ * weights along K, s = fp16_rne(fp32(absmax / 7)) and q = clamp(rint(fp32(w /
+ * s)), -8, 7), ties to even (q = 0 where s is 0). Weights must be finite.
+ */
+e4b_status e4b_quantize_int4_b32(const float* w, int64_t E, int64_t N, int64_t K, uint8_t* codes,
+                                 uint16_t* scales, void* stream);
+
+/*
+ * e4b_gptq_pack_int4_b32 -- [S] the GPTQ packer. Input: symmetric GPTQ tensors
+ * of each expert's W [N, K], group size 32, no act-order: qweight int32
+ * [E, K/8, N] (eight unsigned 4-bit values u along K per word, value i in bits
+ * 4i..4i+3, zero point 8: q = u - 8) and scales fp16 [E, K/32, N]. Output: the
+ * int4-b32 stack above (codes [E, N, K/2], scales [E, N, K/32]), the same
+ * values moved into row-major bytes. qweight and codes 4-byte aligned; buffers
+ * must not overlap. Asymmetric zero points and act-order (g_idx) are not
+ * accepted inputs.
+ */
+e4b_status e4b_gptq_pack_int4_b32(const int32_t* qweight, const uint16_t* gptq_scales, int64_t E,
+                                  int64_t N, int64_t K, uint8_t* codes, uint16_t* scales,
+                                  void* stream);
+
+/*
+ * e4b_gemv_int4_b32 -- [S] the decode GEMV: one token against its n_slots
+ * routed experts e_j = expert_ids[j] of an int4-b32 stack, in one launch.
+ * Every CTA quantises the token row(s) to int8 with one fp32 scale per row
+ * (sx = fp32(max|x|) / 127, xq = clamp(rint(fp32(x / sx)), -127, 127)); per
+ * 32-weight block the products q * xq are summed exactly in int32; then
+ *   acc[j, n] = sx_j * sum_b s[e_j, n, b] * D[e_j, n, b]   (fp32)
+ * and the epilogue writes bf16:
+ *   E4B_EPI_STORE    y [n_slots, N] (row stride ld_y >= N):  bf16(acc[j, n])
+ *   E4B_EPI_SWIGLU   y [n_slots, N/2] (ld_y >= N/2, N even): bf16(silu(acc[j, i])
+ *                    * acc[j, N/2 + i]) -- gate rows first, up rows second
+ *   E4B_EPI_COMBINE  y [N]: bf16(sum_j gates[j] * acc[j, n]) -- no accumulator,
+ *                    one warp owns a row across all slots
+ * x: bf16 rows of K values (16-byte aligned). ld_x == 0: every slot reads the
+ * one row x (the gate_up GEMV); ld_x > 0 (>= K, multiple of 8): slot j reads
+ * x + j * ld_x (the down GEMV, h of each slot), each row with its own sx.
+ * 1 <= n_slots <= 64; the rows of x (ld_x == 0: 1, else n_slots) times K must
+ * fit in shared memory (<= 200 KiB), else E4B_ERR_UNSUPPORTED. An expert id
+ * outside [0, E) drops that slot (its STORE/SWIGLU rows are written as 0) and
+ * records E4B_ERR_BAD_EXPERT_ID in *status when status is not NULL. x must
+ * be finite. Weight rows stream through shared memory in bulk copies whose
+ * waits are bounded; a wait that gives up records E4B_ERR_DEVICE_TIMEOUT in
+ * *status and leaves y unwritten. flags: 0, or E4B_FLAG_TEST_TIMEOUT (every
+ * wait gives up at once: tests that error path).
+ */
+typedef struct {
+  int32_t epilogue;           /* E4B_EPI_STORE, E4B_EPI_SWIGLU or E4B_EPI_COMBINE */
+  int32_t E;
+  int64_t N, K;               /* each expert's W is [N, K] */
+  int32_t n_slots;
+  const uint8_t* codes;       /* [E, N, K/2], 16-byte aligned */
+  const uint16_t* scales;     /* fp16 [E, N, K/32] */
+  const int32_t* expert_ids;  /* [n_slots] */
+  const float* gates;         /* [n_slots], COMBINE only (else may be NULL) */
+  const uint16_t* x;          /* bf16, see ld_x */
+  int64_t ld_x;               /* 0 = one row for every slot, else elements between slot rows */
+  uint16_t* y;                /* bf16 output, see epilogue */
+  int64_t ld_y;               /* elements between output rows (STORE / SWIGLU) */
+  int32_t* status;            /* optional device int32 that records a bad expert id */
+} e4b_int4_gemv_args;
+
+e4b_status e4b_gemv_int4_b32(const e4b_int4_gemv_args* args, uint32_t flags, void* stream);
 
 /* ---------------------------------------------------------- whole layer */
 

@@ -123,7 +123,8 @@ def test_variant_argument_checks():
 def test_binding_structs_match_the_header(tmp_path):
     # sizes and field offsets of the two argument structs, as a C compiler
     # lays them out from include/e4b.h, against the ctypes mirrors
-    structs = {"e4b_moe_weights": e4b.MoeWeights, "e4b_gemm_args": e4b.GemmArgs, "e4b_dgrad_args": e4b.DgradArgs}
+    structs = {"e4b_moe_weights": e4b.MoeWeights, "e4b_gemm_args": e4b.GemmArgs, "e4b_dgrad_args": e4b.DgradArgs,
+               "e4b_int4_gemv_args": e4b.Int4GemvArgs}
     src = ["#include <stdio.h>", "#include <stddef.h>", '#include "e4b.h"', "int main(void) {"]
     for cname, py in structs.items():
         src.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
@@ -166,3 +167,42 @@ def test_dgrad_argument_checks():
     assert L.e4b_grouped_dgrad(ctypes.byref(a), 0, None) == 0  # no rows: nothing to do
     a = e4b.DgradArgs(0, 4, 256, 128, 64, p, p, p, 256, p, p, 128)
     assert L.e4b_grouped_dgrad(ctypes.byref(a), e4b.FLAG_FORCE_GEMV, None) == 2
+
+
+def test_int4_argument_checks():
+    L = e4b.lib()
+    p = 4096
+
+    def gemv(**kw):
+        a = e4b.Int4GemvArgs(e4b.E4B_EPI_STORE, 8, 256, 512, 2, p, p, p, p, p, 0, p, 256, None)
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return L.e4b_gemv_int4_b32(ctypes.byref(a), 0, None)
+
+    assert gemv(epilogue=5) == 1
+    assert gemv(K=48) == 2                       # blocks of 32 along K
+    assert gemv(n_slots=0) == 1
+    assert gemv(n_slots=65) == 2                 # at most 64 routed slots
+    assert gemv(epilogue=e4b.E4B_EPI_SWIGLU, N=255, ld_y=200) == 1  # SwiGLU needs N even
+    assert gemv(epilogue=e4b.E4B_EPI_COMBINE, gates=None) == 1
+    assert gemv(codes=p + 8) == 7
+    assert gemv(x=p + 2) == 7
+    assert gemv(ld_x=12) == 7                    # row stride not a multiple of 8
+    assert gemv(ld_x=256) == 1                   # row stride below K
+    assert gemv(ld_y=100) == 1                   # STORE rows need N
+    assert gemv(x=None) == 1
+    assert gemv(K=256 * 1024) == 2               # activation row beyond shared memory
+    assert gemv(ld_x=64 * 1024, K=64 * 1024, n_slots=4) == 2
+    a = e4b.Int4GemvArgs(0, 8, 256, 512, 2, p, p, p, p, p, 0, p, 256, None)
+    assert L.e4b_gemv_int4_b32(ctypes.byref(a), 1, None) == 1  # only E4B_FLAG_TEST_TIMEOUT is defined
+    q = L.e4b_quantize_int4_b32
+    assert q(p, 2, 4, 48, p, p, None) == 2
+    assert q(p, -1, 4, 64, p, p, None) == 1
+    assert q(None, 2, 4, 64, p, p, None) == 1
+    assert q(p + 4, 2, 4, 64, p, p, None) == 7
+    assert q(None, 0, 4, 64, None, None, None) == 0   # nothing to pack
+    g = L.e4b_gptq_pack_int4_b32
+    assert g(p, p, 2, 4, 48, p, p, None) == 2
+    assert g(p + 2, p, 2, 4, 64, p, p, None) == 7
+    assert g(None, p, 2, 4, 64, p, p, None) == 1
+    assert g(None, None, 0, 4, 64, None, None, None) == 0
