@@ -14,9 +14,12 @@ that give exact integer accumulation):
   s * q. Quantising an fp32 row: s = fp16(absmax / 7) (absmax / 7 in fp32, then
   rounded to fp16); q = clamp(round_half_even(fp32(w / float(s))), -8, 7); an
   all-zero block (or one whose scale rounds to 0) gets s = 0 and q = 0.
-* Activation (one token): one fp32 scale sx = fp32(max |x|) / 127 (IEEE fp32
-  division), xq = clamp(round_half_even(fp32(x / sx)), -127, 127) as int8; an
-  all-zero token has sx = 0 and xq = 0.
+* Activation (one token): amax = max |x|; the dequantisation scale is
+  sx = fp32(amax / 127) and the quantisation multiplier r = fp32(127 / amax)
+  (both IEEE fp32 divisions); xq = clamp(round_half_even(fp32(x * r)), -127,
+  127) as int8, so that every value is decided by one fp32 product. A token
+  whose r is not finite (amax = 0, or amax below 127 / FLT_MAX) has sx = 0 and
+  xq = 0.
 * Output, for weight row n: y[n] = sx * sum_b s[n, b] * D[n, b] with the block
   dot products D[n, b] = sum over the block of q * xq, exact integers. Here the
   sum over blocks is taken in fp64 and y is rounded once to bf16, after the
@@ -98,10 +101,12 @@ def quantize_token(x) -> tuple[np.ndarray, np.float32]:
     """One token (values as fp32 [K]) -> (xq int8 [K] as int64, sx fp32)."""
     x = np.asarray(x, np.float32)
     amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0.0)
-    sx = np.float32(amax / np.float32(127.0))
-    if sx == 0:
+    with np.errstate(divide="ignore", over="ignore"):
+        r = np.float32(np.float32(127.0) / amax) if amax > 0 else np.float32(np.inf)
+    if not np.isfinite(r):
         return np.zeros(x.shape, np.int64), np.float32(0.0)
-    xq = np.clip(_rne((x / sx).astype(np.float32)), -127, 127)
+    sx = np.float32(amax / np.float32(127.0))
+    xq = np.clip(_rne((x * r).astype(np.float32)), -127, 127)
     return xq, sx
 
 

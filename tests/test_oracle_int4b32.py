@@ -89,10 +89,29 @@ def test_quantize_token_within_half_a_step():
     rng = np.random.default_rng(12)
     x = bf16_round(rng.standard_normal(512)).astype(np.float32)
     xq, sx = q4.quantize_token(x)
-    assert sx == np.float32(np.max(np.abs(x)) / np.float32(127))
+    amax = np.float32(np.max(np.abs(x)))
+    assert sx == np.float32(amax / np.float32(127))
     assert np.max(np.abs(xq)) == 127 and np.min(xq) >= -127
-    assert np.all(np.abs(x - np.float64(sx) * xq) <= np.float64(sx) * (0.5 + 2.0 ** -16))
+    # x * fp32(127 / amax) is within 2^-21 relative of x / sx: half a step and a hair
+    assert np.all(np.abs(x - np.float64(sx) * xq) <= np.float64(sx) * (0.5 + 2.0 ** -12))
     assert xq[np.argmax(np.abs(x))] == 127 * np.sign(x[np.argmax(np.abs(x))])
+    # each value is decided by one fp32 product with r = fp32(127 / amax)
+    r = np.float32(np.float32(127) / amax)
+    for i in range(0, 512, 37):
+        t = float(np.float32(x[i] * r))
+        lo = np.floor(t)
+        want = lo + 1 if (t - lo > 0.5 or (t - lo == 0.5 and lo % 2 == 1)) else lo
+        assert xq[i] == int(want)
+
+
+def test_quantize_token_tiny_and_tie_values():
+    # a token so small that 127 / amax overflows is treated as zero
+    xq, sx = q4.quantize_token(np.array([1e-38, -2e-38], np.float32))
+    assert sx == 0 and np.all(xq == 0)
+    # exact ties of x * r round to even: amax = 127 gives r = 1
+    x = np.array([127.0, 0.5, 1.5, 2.5, -0.5, -1.5, -126.5], np.float32)
+    xq, sx = q4.quantize_token(x)
+    assert sx == 1.0 and xq.tolist() == [127, 0, 2, 2, 0, -2, -126]
 
 
 def test_block_dots_against_integer_loops():
