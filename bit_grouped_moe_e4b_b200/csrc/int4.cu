@@ -46,8 +46,7 @@ constexpr int kRows = 4;           // weight rows per item (two outputs)
 constexpr int kChunkBlocks = 128;  // blocks of one row per item (2 KiB of codes)
 constexpr int kLaneBlocks = kChunkBlocks / 32;
 constexpr int kRowBytes = kChunkBlocks * 16;
-constexpr int kScaleRowBytes = kChunkBlocks * 2;  // fp16 scales of one row's chunk
-constexpr int kStageBytes = kRows * (kRowBytes + kScaleRowBytes);
+constexpr int kStageBytes = kRows * kChunkBlocks * (16 + 2);  // codes, then the rows' fp16 scales
 constexpr int kRoundOutputs = 256;  // outputs whose fp32 sums sit in shared memory at once
 constexpr int kQuantGroups = 8;     // groups of 8 activations a thread keeps in registers
 constexpr int kMaxSlots = 64;       // routed experts of one token
@@ -103,18 +102,11 @@ E4B_DEV float warp_max(float v) {
   return v;
 }
 
-// clamp(rint(fl(v / sx)), -127, 127) with fl the IEEE quotient, taken without
-// a division when possible: t = fl(v * r), r = fl(1 / sx), is within 2^-15 of
-// fl(v / sx) for |v / sx| <= 127.01 (two roundings of relative size 2^-24 each
-// on r and t, one on the quotient), so rint(t) is the rounded quotient unless
-// t lies within 2^-15 of a half-integer; those (and a non-finite t) divide.
-E4B_DEV int quant_x(float v, float sx, float r) {
-  if (!(sx > 0.f)) return 0;
-  const float t = __fmul_rn(v, r);
-  float n = rintf(t);
-  if (!(fabsf(t - n) <= 0.499969482421875f)) n = rintf(__fdiv_rn(v, sx));
-  n = fminf(fmaxf(n, -127.f), 127.f);
-  return static_cast<int>(n);
+// clamp(rint(fl(v * r)), -127, 127), ties to even, with r = fl(127 / amax):
+// one fp32 product decides each int8 (r = 0 for a token treated as zero).
+E4B_DEV int quant_x(float v, float r) {
+  const int n = __float2int_rn(__fmul_rn(v, r));
+  return min(max(n, -127), 127);
 }
 
 E4B_DEV uint32_t pack4(int a, int b, int c, int d) {
@@ -139,16 +131,34 @@ E4B_DEV float group_absmax(const uint4 v) {
   return m;
 }
 
-E4B_DEV int quant_group(const uint4 v, float sx, float rcp, int (&q)[8]) {
+E4B_DEV int quant_group(const uint4 v, float r, int (&q)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   int sum = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    q[2 * i] = quant_x(bf16_bits_to_f32(w[i] & 0xFFFFu), sx, rcp);
-    q[2 * i + 1] = quant_x(bf16_bits_to_f32(w[i] >> 16), sx, rcp);
+    q[2 * i] = quant_x(__uint_as_float(w[i] << 16), r);
+    q[2 * i + 1] = quant_x(__uint_as_float(w[i] & 0xFFFF0000u), r);
     sum += q[2 * i] + q[2 * i + 1];
   }
   return sum;
+}
+
+// Quantises one group of 8 activations of row `row` (values v) and stores
+// them; returns their sum (0 for a group past the row).
+E4B_DEV int quant_store(uint8_t* row, int64_t K, int64_t g, bool valid, const uint4 v, float r) {
+  int q[8], sum = 0;
+  if (valid) {
+    sum = quant_group(v, r, q);
+    store_group(row, K, g, q);
+  }
+  return sum;
+}
+
+// Block sums: the 4 groups of a block sit in 4 neighbouring lanes.
+E4B_DEV void store_block_sum(uint8_t* row, int64_t K, int64_t g, bool valid, int sum) {
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+  sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+  if (valid && (g & 3) == 0) reinterpret_cast<int16_t*>(row + K)[g >> 2] = int16_t(-8 * sum);
 }
 
 // Quantises the nx activation rows into xs (row r at r * xrow_bytes(K): plane
@@ -161,66 +171,72 @@ E4B_DEV void quantize_rows(const Int4Gemv& p, uint8_t* xs, float* s_sx, float* s
   const int tid = threadIdx.x, nthreads = blockDim.x, nwarps = nthreads >> 5;
   const int64_t K = p.K, G = K / 8;  // groups of 8 values; 4 groups a block
   const bool cached = G <= int64_t(kQuantGroups) * nthreads;
+  const int passes = int((G + nthreads - 1) / nthreads);
   for (int r0 = 0; r0 < p.nx; r0 += 2) {
-    const int nr = min(2, p.nx - r0);
-    const uint16_t* xr[2] = {p.x + r0 * p.ld_x, p.x + (r0 + nr - 1) * p.ld_x};
-    uint4 v[2][kQuantGroups];
-    float m[2] = {0.f, 0.f};
+    const bool two = r0 + 1 < p.nx;
+    const uint16_t* xa = p.x + r0 * p.ld_x;
+    const uint16_t* xb = two ? xa + p.ld_x : xa;
+    uint4 va[kQuantGroups], vb[kQuantGroups];
+    float ma = 0.f, mb = 0.f;
     if (cached) {
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
+      for (int i = 0; i < kQuantGroups; ++i) {
+        const int64_t g = tid + int64_t(i) * nthreads;
+        const bool ok = g < G;
+        va[i] = ok ? *reinterpret_cast<const uint4*>(xa + 8 * g) : make_uint4(0, 0, 0, 0);
+        vb[i] = (ok && two) ? *reinterpret_cast<const uint4*>(xb + 8 * g) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-        for (int i = 0; i < kQuantGroups; ++i) {
-          const int64_t g = tid + int64_t(i) * nthreads;
-          v[rr][i] = (rr < nr && g < G) ? *reinterpret_cast<const uint4*>(xr[rr] + 8 * g) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-        for (int i = 0; i < kQuantGroups; ++i) m[rr] = fmaxf(m[rr], group_absmax(v[rr][i]));
+      for (int i = 0; i < kQuantGroups; ++i) {
+        ma = fmaxf(ma, group_absmax(va[i]));
+        mb = fmaxf(mb, group_absmax(vb[i]));
+      }
     } else {
-      for (int rr = 0; rr < nr; ++rr)
-        for (int64_t g = tid; g < G; g += nthreads)
-          m[rr] = fmaxf(m[rr], group_absmax(*reinterpret_cast<const uint4*>(xr[rr] + 8 * g)));
+      for (int64_t g = tid; g < G; g += nthreads) {
+        ma = fmaxf(ma, group_absmax(*reinterpret_cast<const uint4*>(xa + 8 * g)));
+        if (two) mb = fmaxf(mb, group_absmax(*reinterpret_cast<const uint4*>(xb + 8 * g)));
+      }
     }
-    m[0] = warp_max(m[0]);
-    m[1] = warp_max(m[1]);
-    if ((tid & 31) == 0) s_red[2 * (tid >> 5)] = m[0], s_red[2 * (tid >> 5) + 1] = m[1];
+    ma = warp_max(ma);
+    mb = warp_max(mb);
+    if ((tid & 31) == 0) s_red[2 * (tid >> 5)] = ma, s_red[2 * (tid >> 5) + 1] = mb;
     __syncthreads();
-    float sx[2], rcp[2];
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      float amax = 0.f;
-      for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, s_red[2 * w + rr]);
-      sx[rr] = __fdiv_rn(amax, 127.f);
-      rcp[rr] = sx[rr] > 0.f ? __fdiv_rn(1.f, sx[rr]) : 0.f;
-      if (tid == 0 && rr < nr) s_sx[r0 + rr] = sx[rr];
+    float amax_a = 0.f, amax_b = 0.f;
+    for (int w = 0; w < nwarps; ++w) amax_a = fmaxf(amax_a, s_red[2 * w]), amax_b = fmaxf(amax_b, s_red[2 * w + 1]);
+    // r = fl(127 / amax); a token whose r is not finite is treated as zero
+    float ra = __fdiv_rn(127.f, amax_a), rb = __fdiv_rn(127.f, amax_b);
+    const bool za = !(amax_a > 0.f) || isinf(ra), zb = !(amax_b > 0.f) || isinf(rb);
+    const float sxa = za ? 0.f : __fdiv_rn(amax_a, 127.f), sxb = zb ? 0.f : __fdiv_rn(amax_b, 127.f);
+    ra = za ? 0.f : ra;
+    rb = zb ? 0.f : rb;
+    if (tid == 0) {
+      s_sx[r0] = sxa;
+      if (two) s_sx[r0 + 1] = sxb;
     }
-    // quantise; every thread runs the same passes so the block sums reduce
-    // over the 4 lanes of a block with full-warp shuffles
-    for (int rr = 0; rr < nr; ++rr) {
-      uint8_t* row = xs + (r0 + rr) * xrow_bytes(K);
-      int16_t* bsum = reinterpret_cast<int16_t*>(row + K);
-      const int passes = int((G + nthreads - 1) / nthreads);
+    uint8_t* rowa = xs + r0 * xrow_bytes(K);
+    uint8_t* rowb = rowa + xrow_bytes(K);
+    // every thread runs the same passes: the block sums reduce over 4 lanes
+    // with full-warp shuffles
+    if (cached) {
+#pragma unroll
+      for (int i = 0; i < kQuantGroups; ++i) {
+        if (i < passes) {
+          const int64_t g = tid + int64_t(i) * nthreads;
+          const bool ok = g < G;
+          store_block_sum(rowa, K, g, ok, quant_store(rowa, K, g, ok, va[i], ra));
+          if (two) store_block_sum(rowb, K, g, ok, quant_store(rowb, K, g, ok, vb[i], rb));
+        }
+      }
+    } else {
       for (int i = 0; i < passes; ++i) {
         const int64_t g = tid + int64_t(i) * nthreads;
-        int q[8], sum = 0;
-        if (g < G) {
-          uint4 val;
-          if (cached) {
-            val = v[0][0];
-#pragma unroll
-            for (int k = 0; k < kQuantGroups; ++k)
-              if (k == i) val = rr == 0 ? v[0][k] : v[1][k];
-          } else {
-            val = *reinterpret_cast<const uint4*>(xr[rr] + 8 * g);
-          }
-          sum = quant_group(val, sx[rr], rcp[rr], q);
-          store_group(row, K, g, q);
+        const bool ok = g < G;
+        const uint4 v0 = ok ? *reinterpret_cast<const uint4*>(xa + 8 * g) : make_uint4(0, 0, 0, 0);
+        store_block_sum(rowa, K, g, ok, quant_store(rowa, K, g, ok, v0, ra));
+        if (two) {
+          const uint4 v1 = ok ? *reinterpret_cast<const uint4*>(xb + 8 * g) : make_uint4(0, 0, 0, 0);
+          store_block_sum(rowb, K, g, ok, quant_store(rowb, K, g, ok, v1, rb));
         }
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
-        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-        if (g < G && (g & 3) == 0) bsum[g >> 2] = int16_t(-8 * sum);
       }
     }
     __syncthreads();  // s_red is reused by the next row pair
@@ -245,6 +261,15 @@ struct __align__(16) ItemDesc {
   uint32_t ja, jb;           // COMBINE: slots a and b (jb == n_slots: none)
 };
 static_assert(sizeof(ItemDesc) == 64, "descriptor slot is 64 bytes");
+
+// Stage position of row r: rows that are neighbours in memory (same expert,
+// consecutive weight rows) sit in neighbouring positions, so that when a
+// chunk is a whole row they arrive in one copy. STORE: rows n, n+1, n', n'+1;
+// SWIGLU: gate i, gate i', up i, up i'; COMBINE: (a, n), (a, n+1), (b, n), (b, n+1).
+template <int EPI>
+__host__ __device__ constexpr int row_pos(int r) {
+  return EPI == E4B_EPI_STORE ? r : (r == 1 ? 2 : r == 2 ? 1 : r);
+}
 
 struct Cursor {
   uint32_t c, pp, ol;  // chunk, slot pair, first output of the item within the round
@@ -296,88 +321,114 @@ E4B_DEV void cursor_next(Cursor& k, const Int4Gemv& p, const Int4Plan& q) {
   out_next<EPI>(k.j, k.n, p);
 }
 
-// Lane 0: writes the descriptor of the item at cursor k into d, starts the
-// bulk copies of its code chunks into the stage (row r at r * kRowBytes) and
-// prefetches its scales into L2. `nout` = outputs of the round.
+E4B_DEV int64_t pick4(int i, int64_t v0, int64_t v1, int64_t v2, int64_t v3) {
+  return i == 0 ? v0 : i == 1 ? v1 : i == 2 ? v2 : v3;
+}
+
+// The whole warp starts item k into a stage: lane 0 writes the descriptor and
+// posts the expected bytes on the stage's barrier; lanes 0-3 then take one
+// stage position each and copy its row chunk (two neighbouring rows in one
+// copy when the chunk is the whole row and the rows are consecutive rows of
+// one expert), and prefetch the row's scales into L2. `nout` = outputs of
+// the round. Ends with every lane past a __syncwarp.
 template <int EPI>
 E4B_DEV void issue_item(const Cursor& k, uint32_t nout, const Int4Gemv& p, const Int4Plan& q,
-                        const int32_t* s_ids, ItemDesc* d, uint8_t* stage, uint64_t* bar) {
+                        const int32_t* s_ids, ItemDesc* d, uint8_t* stage, uint64_t* bar, int lane) {
   const int64_t N = p.N, NB = p.K / kI4Block, halfK = p.K / 2;
   const int64_t coff = int64_t(k.c) * kChunkBlocks;
   const uint32_t nb = uint32_t(min(int64_t(kChunkBlocks), NB - coff));
   const bool two = k.ol + 1 < nout;
-  int e[kRows];
-  int64_t row[kRows];
-  uint32_t xj[2];
-  uint32_t xsel = 0;
   uint32_t j2 = k.j, n2 = k.n;
   out_next<EPI>(j2, n2, p);
+  // expert (-1: none) and weight row of logical rows 0..3
+  int e0, e1, e2, e3;
+  int64_t w0, w1, w2, w3;
+  uint32_t xj0, xj1, ja = 0, jb = 0;
   if constexpr (EPI == E4B_EPI_STORE) {
-    const int ea = s_ids[k.j];
-    const int eb = two ? s_ids[j2] : -1;
-    e[0] = ea, row[0] = k.n;
-    e[1] = k.n + 1 < uint32_t(N) ? ea : -1, row[1] = k.n + 1;
-    e[2] = eb, row[2] = n2;
-    e[3] = (two && n2 + 1 < uint32_t(N)) ? eb : -1, row[3] = n2 + 1;
-    xj[0] = k.j, xj[1] = two ? j2 : k.j;
-    xsel = 0xC;
+    const int ea = s_ids[k.j], eb = two ? s_ids[j2] : -1;
+    e0 = ea, w0 = k.n;
+    e1 = k.n + 1 < uint32_t(N) ? ea : -1, w1 = k.n + 1;
+    e2 = eb, w2 = n2;
+    e3 = (two && n2 + 1 < uint32_t(N)) ? eb : -1, w3 = n2 + 1;
+    xj0 = k.j, xj1 = two ? j2 : k.j;
   } else if constexpr (EPI == E4B_EPI_SWIGLU) {
     const int64_t I = N / 2;
-    const int ea = s_ids[k.j];
-    const int eb = two ? s_ids[j2] : -1;
-    e[0] = ea, row[0] = k.n;
-    e[1] = ea, row[1] = k.n + I;
-    e[2] = eb, row[2] = n2;
-    e[3] = eb, row[3] = n2 + I;
-    xj[0] = k.j, xj[1] = two ? j2 : k.j;
-    xsel = 0xC;
+    const int ea = s_ids[k.j], eb = two ? s_ids[j2] : -1;
+    e0 = ea, w0 = k.n;
+    e1 = ea, w1 = k.n + I;
+    e2 = eb, w2 = n2;
+    e3 = eb, w3 = n2 + I;
+    xj0 = k.j, xj1 = two ? j2 : k.j;
   } else {
-    const uint32_t a = 2 * k.pp, b = a + 1;
-    const int ea = s_ids[a];
-    const int eb = b < uint32_t(p.n_slots) ? s_ids[b] : -1;
-    e[0] = ea, row[0] = k.n;
-    e[1] = eb, row[1] = k.n;
-    e[2] = two ? ea : -1, row[2] = k.n + 1;
-    e[3] = two ? eb : -1, row[3] = k.n + 1;
-    xj[0] = a, xj[1] = b < uint32_t(p.n_slots) ? b : a;
-    xsel = 0xA;
-    d->ja = a;
-    d->jb = b;
+    ja = 2 * k.pp, jb = ja + 1;
+    const int ea = s_ids[ja], eb = jb < uint32_t(p.n_slots) ? s_ids[jb] : -1;
+    e0 = ea, w0 = k.n;
+    e1 = eb, w1 = k.n;
+    e2 = two ? ea : -1, w2 = k.n + 1;
+    e3 = two ? eb : -1, w3 = k.n + 1;
+    xj0 = ja, xj1 = jb < uint32_t(p.n_slots) ? jb : ja;
   }
-  const uint32_t xrb = uint32_t(xrow_bytes(p.K));
-  d->x0 = (p.nx == 1 ? 0 : xj[0]) * xrb;
-  d->x1 = (p.nx == 1 ? 0 : xj[1]) * xrb;
-  d->xsel = xsel;
-  d->nb = nb;
-  d->acc = 2 * k.ol;
-  uint32_t flags = two ? 16u : 0u;
-  uint32_t total = 0;
-  const uint8_t* src[kRows];
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) {
-    const int64_t er = int64_t(e[r]) * N + row[r];
-    d->s[r] = e[r] >= 0 ? p.scales + er * NB + coff : nullptr;
-    src[r] = e[r] >= 0 ? p.codes + er * halfK + coff * 16 : nullptr;
-    total += e[r] >= 0 ? nb * 16 : 0;
-    flags |= e[r] >= 0 ? 1u << r : 0u;
+  const uint32_t flags = (two ? 16u : 0u) | (e0 >= 0 ? 1u : 0u) | (e1 >= 0 ? 2u : 0u) | (e2 >= 0 ? 4u : 0u) |
+                         (e3 >= 0 ? 8u : 0u);
+  if (lane == 0) {
+    const uint32_t xrb = uint32_t(xrow_bytes(p.K));
+    d->s[0] = e0 >= 0 ? p.scales + (int64_t(e0) * N + w0) * NB + coff : nullptr;
+    d->s[1] = e1 >= 0 ? p.scales + (int64_t(e1) * N + w1) * NB + coff : nullptr;
+    d->s[2] = e2 >= 0 ? p.scales + (int64_t(e2) * N + w2) * NB + coff : nullptr;
+    d->s[3] = e3 >= 0 ? p.scales + (int64_t(e3) * N + w3) * NB + coff : nullptr;
+    d->x0 = (p.nx == 1 ? 0 : xj0) * xrb;
+    d->x1 = (p.nx == 1 ? 0 : xj1) * xrb;
+    d->nb = nb;
+    d->acc = 2 * k.ol;
+    d->flags = flags;
+    d->ja = ja;
+    d->jb = jb;
+    mbar_arrive_expect_tx(bar, uint32_t(__popc(flags & 15u)) * nb * (q.sbulk ? 18u : 16u));
   }
-  d->flags = flags;
-  // scales come with the codes when every row's chunk of them is 16-byte
-  // aligned (K % 256 == 0), else the lanes load them (after an L2 prefetch)
-  if (q.sbulk) total += __popc(flags & 15u) * nb * 2;
-  mbar_arrive_expect_tx(bar, total);  // releases the descriptor stores to the waiting lanes
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) {
-    if (src[r]) {
-      bulk_load(stage + r * kRowBytes, src[r], nb * 16, bar);
+  __syncwarp();  // the expected bytes are posted before any copy lands
+  if (lane < kRows) {
+    // logical row at this position and at the next one
+    const int r = row_pos<EPI>(lane);  // the position map is its own inverse
+    const int rn = row_pos<EPI>((lane + 1) & 3);
+    const int64_t e = pick4(r, e0, e1, e2, e3), w = pick4(r, w0, w1, w2, w3);
+    const int64_t en = pick4(rn, e0, e1, e2, e3), wn = pick4(rn, w0, w1, w2, w3);
+    const int rp = row_pos<EPI>((lane + 3) & 3);  // the previous position's row
+    const int64_t ep = pick4(rp, e0, e1, e2, e3), wp = pick4(rp, w0, w1, w2, w3);
+    // positions pair up as (0, 1) and (2, 3)
+    const bool whole = q.nch == 1;
+    const bool joins_next = whole && (lane & 1) == 0 && e >= 0 && en == e && wn == w + 1;
+    const bool joined = whole && (lane & 1) == 1 && e >= 0 && ep == e && w == wp + 1;
+    if (e >= 0 && !joined) {
+      const int64_t er = e * N + w;
+      const uint32_t rows = joins_next ? 2u : 1u;
+      bulk_load(stage + lane * nb * 16, p.codes + er * halfK + coff * 16, rows * nb * 16, bar);
+      const uint16_t* sc = p.scales + er * NB + coff;
       if (q.sbulk) {
-        bulk_load(stage + kRows * kRowBytes + r * kScaleRowBytes, d->s[r], nb * 2, bar);
+        // scales ride with the codes (every row's chunk of them is 16-byte aligned)
+        bulk_load(stage + kRows * nb * 16 + lane * nb * 2, sc, rows * nb * 2, bar);
       } else {
-        prefetch_l2(d->s[r]);
-        if (nb > 64) prefetch_l2(d->s[r] + 64);
+        prefetch_l2(sc);
+        if (nb > 64) prefetch_l2(sc + 64);
+        if (joins_next) {
+          prefetch_l2(sc + NB);
+          if (nb > 64) prefetch_l2(sc + NB + 64);
+        }
       }
     }
   }
+  __syncwarp();
+}
+
+// The lane's scales of an item: row r, lane block u (0 where the row is
+// absent or the block is past the chunk).
+E4B_DEV void load_scales(const ItemDesc& d, int lane, uint32_t (&h)[kRows][kLaneBlocks]) {
+#pragma unroll
+  for (int r = 0; r < kRows; ++r)
+#pragma unroll
+    for (int u = 0; u < kLaneBlocks; ++u) {
+      const uint32_t lb = lane + 32 * u;
+      h[r][u] = (((d.flags >> r) & 1u) && lb < d.nb) ? ldg_nc_u16(d.s[r] + lb) : 0u;
+    }
 }
 
 template <int EPI>
@@ -425,8 +476,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     const uint32_t i0 = streams ? uint32_t(uint64_t(warp) * items / q.warps) : 0;
     const uint32_t i1 = streams ? uint32_t(uint64_t(warp + 1) * items / q.warps) : 0;
     for (uint32_t i = tid; i < 2 * nout; i += blockDim.x) s_acc[i] = 0.f;
-    // the first stages start before the activation rows are quantised: the
-    // copies do not depend on them
+    // the first stages (and the first item's scales) are on their way while
+    // the activation rows are quantised: they do not depend on them
     Cursor ki{}, kc{};
     if (i0 < i1) {
       cursor_init<EPI>(ki, i0, p, q, r0);
@@ -434,11 +485,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     }
     uint32_t issued = i0, waited = i0;
     for (int s = 0; s < kStages && issued < i1; ++s, ++issued) {
-      if (lane == 0) issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + s, my_ring + s * kStageBytes, my_bar + s);
+      issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + s, my_ring + s * kStageBytes, my_bar + s, lane);
       cursor_next<EPI>(ki, p, q);
     }
+    uint32_t hn[kRows][kLaneBlocks];  // scales of the next item (when they are not copied)
+    if (!q.sbulk && i0 < i1) load_scales(my_desc[0], lane, hn);
     if (first) {
-      quantize_rows(p, xs, s_sx, s_red);  // ends with __syncthreads
+      quantize_rows(p, xs, s_sx, s_red);  // ends with __syncthreads (s_acc cleared too)
       first = false;
     } else {
       __syncthreads();  // s_acc cleared
@@ -446,20 +499,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     bool ok = true;
     for (uint32_t it = i0; it < i1; ++it) {
       const int s = int((it - i0) % kStages);
-      // the descriptor was written at least two __syncwarp (or a
-      // __syncthreads) ago, so it is read, and the scales fetched, before
-      // the wait on the codes
+      // the descriptor was written before at least one __syncwarp
       const ItemDesc d = my_desc[s];
+      // the inner loop has no branches, so the 16 block dot products of an
+      // item overlap: a row that is absent, or a block past the chunk, gets
+      // scale 0 (its reads stay inside this CTA's stage and activation rows).
+      // The scales of the next item are loaded now (L2 hits after the
+      // prefetch at issue time) and used one item later.
       uint32_t h[kRows][kLaneBlocks];
-      if (!q.sbulk) {
 #pragma unroll
-        for (int r = 0; r < kRows; ++r)
+      for (int r = 0; r < kRows; ++r)
 #pragma unroll
-          for (int u = 0; u < kLaneBlocks; ++u) {
-            const uint32_t lb = lane + 32 * u;
-            h[r][u] = (((d.flags >> r) & 1u) && lb < d.nb) ? ldg_nc_u16(d.s[r] + lb) : 0u;
-          }
-      }
+        for (int u = 0; u < kLaneBlocks; ++u) h[r][u] = hn[r][u];
+      if (!q.sbulk && it + 1 < i1) load_scales(my_desc[(s + 1) % kStages], lane, hn);
       // polls == 0 (E4B_FLAG_TEST_TIMEOUT): give up at the first wait
       if (q.polls == 0 || !mbar_wait_bounded(my_bar + s, (parity >> s) & 1u, q.polls, s_abort)) {
         ok = false;
@@ -469,41 +521,35 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
       ++waited;
       const uint8_t* st = my_ring + s * kStageBytes;
       if (q.sbulk) {
-        const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + kRows * kRowBytes);
+        const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + kRows * d.nb * 16);
 #pragma unroll
         for (int r = 0; r < kRows; ++r)
 #pragma unroll
-          for (int u = 0; u < kLaneBlocks; ++u) h[r][u] = ss[r * kChunkBlocks + lane + 32 * u];
+          for (int u = 0; u < kLaneBlocks; ++u) {
+            const uint32_t lb = lane + 32 * u;
+            const uint32_t v = ss[row_pos<EPI>(r) * d.nb + lb];
+            h[r][u] = (((d.flags >> r) & 1u) && lb < d.nb) ? v : 0u;
+          }
       }
-      const uint8_t* x0 = xs + d.x0;
-      const uint8_t* x1 = xs + d.x1;
-      const int64_t boff = int64_t(p.K) + int64_t(kChunkBlocks) * 2 * kc.c;  // block sums of the chunk
+      const uint8_t* x0 = xs + d.x0 + kc.c * kChunkBlocks * 16;
+      const uint8_t* x1 = xs + d.x1 + kc.c * kChunkBlocks * 16;
+      const int16_t* b0 = reinterpret_cast<const int16_t*>(xs + d.x0 + p.K) + kc.c * kChunkBlocks;
+      const int16_t* b1 = reinterpret_cast<const int16_t*>(xs + d.x1 + p.K) + kc.c * kChunkBlocks;
       float a[kRows] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int u = 0; u < kLaneBlocks; ++u) {
         const uint32_t lb = lane + 32 * u;
-        if (lb < d.nb) {
-          const uint32_t xo = (kc.c * kChunkBlocks + lb) * 16;
-          const uint4 xa0 = lds_v4(x0 + xo), xb0 = lds_v4(x0 + halfK + xo);
-          const int s0 = reinterpret_cast<const int16_t*>(x0 + boff)[lb];
-          uint4 xa1 = xa0, xb1 = xb0;
-          int s1 = s0;
-          if (d.x1 != d.x0) {
-            xa1 = lds_v4(x1 + xo);
-            xb1 = lds_v4(x1 + halfK + xo);
-            s1 = reinterpret_cast<const int16_t*>(x1 + boff)[lb];
-          }
+        const uint4 xa0 = lds_v4(x0 + lb * 16), xb0 = lds_v4(x0 + halfK + lb * 16);
+        const uint4 xa1 = lds_v4(x1 + lb * 16), xb1 = lds_v4(x1 + halfK + lb * 16);
+        const int s0 = b0[lb], s1 = b1[lb];
 #pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            // the activation row of row r is fixed by the epilogue: rows 2, 3
-            // (STORE / SWIGLU) or 1, 3 (COMBINE) read x1
-            constexpr uint32_t kSel = EPI == E4B_EPI_COMBINE ? 0xAu : 0xCu;
-            if ((d.flags >> r) & 1u) {
-              const uint4 w = lds_v4(st + r * kRowBytes + lb * 16);
-              const int v = ((kSel >> r) & 1u) ? block_dot16(w, xa1, xb1, s1) : block_dot16(w, xa0, xb0, s0);
-              a[r] = fmaf(half_bits_to_f32(h[r][u]), float(v), a[r]);
-            }
-          }
+        for (int r = 0; r < kRows; ++r) {
+          // the activation row of row r is fixed by the epilogue: rows 2, 3
+          // (STORE / SWIGLU) or 1, 3 (COMBINE) read x1
+          constexpr uint32_t kSel = EPI == E4B_EPI_COMBINE ? 0xAu : 0xCu;
+          const uint4 w = lds_v4(st + (row_pos<EPI>(r) * d.nb + lb) * 16);
+          const int v = ((kSel >> r) & 1u) ? block_dot16(w, xa1, xb1, s1) : block_dot16(w, xa0, xb0, s0);
+          a[r] = fmaf(half_bits_to_f32(h[r][u]), float(v), a[r]);
         }
       }
       // four row sums leave the warp in one butterfly: after it, lane 8 m
@@ -532,7 +578,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
       }
       __syncwarp();  // every lane has read the stage and its descriptor before the refill
       if (issued < i1) {
-        if (lane == 0) issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + s, my_ring + s * kStageBytes, my_bar + s);
+        issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + s, my_ring + s * kStageBytes, my_bar + s, lane);
         cursor_next<EPI>(ki, p, q);
         ++issued;
       }
