@@ -476,17 +476,19 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     const uint32_t i0 = streams ? uint32_t(uint64_t(warp) * items / q.warps) : 0;
     const uint32_t i1 = streams ? uint32_t(uint64_t(warp + 1) * items / q.warps) : 0;
     for (uint32_t i = tid; i < 2 * nout; i += blockDim.x) s_acc[i] = 0.f;
-    // the first stages (and the first item's scales) are on their way while
-    // the activation rows are quantised: they do not depend on them
+    // the first item (and its scales) is on its way while the activation rows
+    // are quantised; the other stages start at the top of the item loop (a
+    // burst of copies at the start would hold up the quantisation's loads)
     Cursor ki{}, kc{};
     if (i0 < i1) {
       cursor_init<EPI>(ki, i0, p, q, r0);
       kc = ki;
     }
     uint32_t issued = i0, waited = i0;
-    for (int s = 0; s < kStages && issued < i1; ++s, ++issued) {
-      issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + s, my_ring + s * kStageBytes, my_bar + s, lane);
+    if (issued < i1) {
+      issue_item<EPI>(ki, nout, p, q, s_ids, my_desc, my_ring, my_bar, lane);
       cursor_next<EPI>(ki, p, q);
+      ++issued;
     }
     uint32_t hn[kRows][kLaneBlocks];  // scales of the next item (when they are not copied)
     if (!q.sbulk && i0 < i1) load_scales(my_desc[0], lane, hn);
@@ -498,6 +500,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     }
     bool ok = true;
     for (uint32_t it = i0; it < i1; ++it) {
+      // keep kStages items in flight: the stages of items before `it` are free
+      while (issued < i1 && issued < it + kStages) {
+        const int sn = int((issued - i0) % kStages);
+        issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + sn, my_ring + sn * kStageBytes, my_bar + sn, lane);
+        cursor_next<EPI>(ki, p, q);
+        ++issued;
+      }
       const int s = int((it - i0) % kStages);
       // the descriptor was written before at least one __syncwarp
       const ItemDesc d = my_desc[s];
@@ -576,12 +585,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
         const int m = lane >> 3;  // value index held by lanes 8m..8m+7
         if ((lane & 7) == 0 && ((d.flags >> m) & 1u)) atomicAdd(s_acc + d.acc + m, v);
       }
-      __syncwarp();  // every lane has read the stage and its descriptor before the refill
-      if (issued < i1) {
-        issue_item<EPI>(ki, nout, p, q, s_ids, my_desc + s, my_ring + s * kStageBytes, my_bar + s, lane);
-        cursor_next<EPI>(ki, p, q);
-        ++issued;
-      }
+      __syncwarp();  // every lane has read the stage and its descriptor before its refill
       cursor_next<EPI>(kc, p, q);
     }
     if (!ok) {
