@@ -318,7 +318,7 @@ e4b_status e4b_gptq_pack_int4_b32(const int32_t* qweight, const uint16_t* gptq_s
 }
 
 e4b_status e4b_gemv_int4_b32(const e4b_int4_gemv_args* a, uint32_t flags, void* stream) {
-  if (!a || (flags & ~E4B_FLAG_TEST_TIMEOUT)) return E4B_ERR_INVALID_ARG;
+  if (!a || (flags & ~(E4B_FLAG_TEST_TIMEOUT | E4B_FLAG_IDS_READY))) return E4B_ERR_INVALID_ARG;
   if (a->epilogue != E4B_EPI_STORE && a->epilogue != E4B_EPI_SWIGLU && a->epilogue != E4B_EPI_COMBINE)
     return E4B_ERR_INVALID_ARG;
   if (a->E <= 0 || a->N <= 0 || a->K <= 0 || a->n_slots <= 0 || a->ld_x < 0) return E4B_ERR_INVALID_ARG;

@@ -451,6 +451,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
   ItemDesc* my_desc = s_desc + warp * kStages;
   const int64_t halfK = p.K / 2;
 
+  // programmatic dependent launch: x, and unless the caller says otherwise
+  // the ids and gates, may come from the kernel before this one in the
+  // stream, and y may still be read by it
+  const bool ids_ready = (p.flags & E4B_FLAG_IDS_READY) != 0;
+  if (!ids_ready) grid_dependency_wait();
   if (tid < p.n_slots) {
     const int e = p.ids[tid];
     const bool bad = e < 0 || e >= p.E;
@@ -493,6 +498,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     uint32_t hn[kRows][kLaneBlocks];  // scales of the next item (when they are not copied)
     if (!q.sbulk && i0 < i1) load_scales(my_desc[0], lane, hn);
     if (first) {
+      // with the ids ready the first weight copies are already on their way
+      if (ids_ready) grid_dependency_wait();
       quantize_rows(p, xs, s_sx, s_red);  // ends with __syncthreads (s_acc cleared too)
       first = false;
     } else {
@@ -601,6 +608,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
         parity ^= 1u << s;
       }
     }
+    // every copy of this CTA has been issued: the next grid may start
+    // launching (its CTAs take SMs as this grid's CTAs leave)
+    if (r0 + kRoundOutputs >= o1) grid_launch_dependents();
     __syncthreads();  // all sums of the round are in s_acc
     const bool aborted = *reinterpret_cast<volatile int32_t*>(s_abort) != 0;
     for (uint32_t ol = tid; ol < nout && !aborted; ol += blockDim.x) {
@@ -735,8 +745,19 @@ cudaError_t launch_int4_gemv(const Int4Gemv& p, cudaStream_t st, int sms) {
   auto launch = [&](auto kernel) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kGemvThreads, smem, st>>>(p, q);
-    return cudaGetLastError();
+    // programmatic dependent launch: the kernel waits on its predecessor in
+    // the stream itself (griddepcontrol.wait) before it reads x or writes y
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kGemvThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p, q);
   };
   switch (p.epilogue) {
     case E4B_EPI_STORE: return launch(int4_gemv_kernel<E4B_EPI_STORE>);

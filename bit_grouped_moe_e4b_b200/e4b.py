@@ -25,6 +25,7 @@ E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05, E4B_PATH_INT4_GEMV = 0, 1, 2, 3
 FLAG_FORCE_GEMV = 0x1
 FLAG_FORCE_TCGEN05 = 0x2
 FLAG_TEST_TIMEOUT = 0x4
+FLAG_IDS_READY = 0x10  # e4b_gemv_int4_b32: ids and gates not written by the preceding work on the stream
 FLAG_NF4_PRODUCT_DECODE = 0x8  # small-M NF4: bf16(level * absmax) operands (the default is bf16(level), absmax after the block MMA)
 STATUS_NAMES = {
     0: "E4B_OK", 1: "E4B_ERR_INVALID_ARG", 2: "E4B_ERR_UNSUPPORTED",
@@ -259,14 +260,18 @@ def quantize_int4_b32(w: torch.Tensor):
 def int4_decode_layer(x, expert_ids, gates, gu_codes, gu_scales, dn_codes, dn_scales, *, E, H, I, h=None, y=None):
     """One token through the MoE layer on int4-b32 stacks: the gate_up GEMV
     with the SwiGLU epilogue (h [k, I]), then the down GEMV with the combine
-    epilogue (y [H]). Two launches; returns y."""
+    epilogue (y [H]). Two launches (the second a programmatic dependent of the
+    first); returns y."""
     k = expert_ids.numel()
     if h is None:
         h = torch.empty((k, I), dtype=torch.bfloat16, device=x.device)
     if y is None:
         y = torch.empty((H,), dtype=torch.bfloat16, device=x.device)
     e4b_gemv_int4_b32("swiglu", gu_codes, gu_scales, expert_ids, x, h, E=E, N=2 * I, K=H, ld_y=I)
-    e4b_gemv_int4_b32("combine", dn_codes, dn_scales, expert_ids, h, y, E=E, N=H, K=I, gates=gates, ld_x=I)
+    # the ids and gates were read by the gate_up launch: the down launch may
+    # start streaming its experts' weights while gate_up finishes
+    e4b_gemv_int4_b32("combine", dn_codes, dn_scales, expert_ids, h, y, E=E, N=H, K=I, gates=gates, ld_x=I,
+                      flags=FLAG_IDS_READY)
     return y
 
 

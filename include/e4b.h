@@ -88,6 +88,11 @@ typedef enum {
  * 2^-8 relative of level * absmax); the default needs half the shared-memory
  * table traffic and is the faster one. */
 #define E4B_FLAG_NF4_PRODUCT_DECODE 0x8u
+/* e4b_gemv_int4_b32: the expert ids and gates are not written by the work
+ * queued just before the call on the stream (they are ready when the call is
+ * enqueued), so the kernel may start streaming the routed experts' weights
+ * before that work completes. It still waits for it before reading x. */
+#define E4B_FLAG_IDS_READY 0x10u
 
 /* NF4 block size (weights per absmax) and MXFP4 block size (weights per scale). */
 #define E4B_NF4_BLOCK 64
@@ -341,8 +346,11 @@ e4b_status e4b_gptq_pack_int4_b32(const int32_t* qweight, const uint16_t* gptq_s
  * records E4B_ERR_BAD_EXPERT_ID in *status when status is not NULL. x must
  * be finite. Weight rows stream through shared memory in bulk copies whose
  * waits are bounded; a wait that gives up records E4B_ERR_DEVICE_TIMEOUT in
- * *status and leaves y unwritten. flags: 0, or E4B_FLAG_TEST_TIMEOUT (every
- * wait gives up at once: tests that error path).
+ * *status and leaves y unwritten. The kernel is launched as a programmatic
+ * dependent of the work before it on the stream: it waits for that work to
+ * complete before it reads x (and, without E4B_FLAG_IDS_READY, the ids and
+ * gates) or writes y. flags: any of E4B_FLAG_IDS_READY (see above) and
+ * E4B_FLAG_TEST_TIMEOUT (every wait gives up at once: tests that error path).
  */
 typedef struct {
   int32_t epilogue;           /* E4B_EPI_STORE, E4B_EPI_SWIGLU or E4B_EPI_COMBINE */

@@ -194,7 +194,7 @@ def test_int4_argument_checks():
     assert gemv(K=256 * 1024) == 2               # activation row beyond shared memory
     assert gemv(ld_x=64 * 1024, K=64 * 1024, n_slots=4) == 2
     a = e4b.Int4GemvArgs(0, 8, 256, 512, 2, p, p, p, p, p, 0, p, 256, None)
-    assert L.e4b_gemv_int4_b32(ctypes.byref(a), 1, None) == 1  # only E4B_FLAG_TEST_TIMEOUT is defined
+    assert L.e4b_gemv_int4_b32(ctypes.byref(a), 1, None) == 1  # only E4B_FLAG_TEST_TIMEOUT and E4B_FLAG_IDS_READY
     q = L.e4b_quantize_int4_b32
     assert q(p, 2, 4, 48, p, p, None) == 2
     assert q(p, -1, 4, 64, p, p, None) == 1
