@@ -24,6 +24,31 @@ E4B_DEV void record_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Programmatic dependent launch: wait until the grid this one depends on has
+// completed and its memory is visible (returns at once when there is none);
+// allow the grid that depends on this one to start launching.
+E4B_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+E4B_DEV void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launches `kernel` as a programmatic dependent of the work before it on the
+// stream: it may start before that work completes and must call
+// grid_dependency_wait() before touching memory that work writes or reads.
+template <typename Kernel, typename... Args>
+inline cudaError_t launch_dependent(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                    Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------------ bf16
 E4B_DEV uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -747,17 +747,7 @@ cudaError_t launch_int4_gemv(const Int4Gemv& p, cudaStream_t st, int sms) {
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: the kernel waits on its predecessor in
     // the stream itself (griddepcontrol.wait) before it reads x or writes y
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kGemvThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, p, q);
+    return launch_dependent(kernel, dim3(grid), dim3(kGemvThreads), smem, st, p, q);
   };
   switch (p.epilogue) {
     case E4B_EPI_STORE: return launch(int4_gemv_kernel<E4B_EPI_STORE>);

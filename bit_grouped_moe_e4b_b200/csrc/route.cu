@@ -30,6 +30,11 @@ route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __r
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
+  // launched as a programmatic dependent: the work before it may still read
+  // what this kernel writes; the layer kernel after it may start launching
+  // (it waits for this kernel before reading the routing)
+  grid_dependency_wait();
+  grid_launch_dependents();
   for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) wcnt[i] = 0;
   // counters the following layer kernels expect at zero
   for (int i = tid; i < nclear; i += kRouteThreads) clear[i] = 0;
@@ -143,9 +148,8 @@ cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* coun
     if (err != cudaSuccess) return err;
     configured = dev;
   }
-  route_kernel<<<1, kRouteThreads, smem, st>>>(ids, R, E, counts, offsets, perm, inv, active, status,
-                                                clear, nclear);
-  return cudaGetLastError();
+  return launch_dependent(route_kernel, dim3(1), dim3(kRouteThreads), smem, st, ids, R, E, counts, offsets, perm, inv,
+                          active, status, clear, nclear);
 }
 
 // The routed activation rows in expert order, xs[p] = x[perm[p] / top_k] for

@@ -64,12 +64,6 @@ E4B_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Programmatic dependent launch: wait until the grid this one depends on has
-// completed and its memory is visible (returns at once when there is none);
-// allow the grid that depends on this one to start launching.
-E4B_DEV void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-E4B_DEV void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // Barrier `id` over the first `nthreads` threads that also returns, to every
 // one of them, the OR of their `v`.
 E4B_DEV bool named_bar_or(int id, int nthreads, bool v) {

@@ -761,6 +761,10 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
     *s_abort = 0;
     mbar_init_fence();
   }
+  // launched as a programmatic dependent of the routing pass: the table and
+  // barriers above are set up while it runs; everything below reads its
+  // output or the counters it clears
+  grid_dependency_wait();
 
   // Clear the fp32 accumulator in chunks handed out by a counter, so that
   // waiting on the cleared count only depends on CTAs that are running.
@@ -895,13 +899,13 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
   // persistent: one CTA per SM, all resident at once
   if (L.fmt == E4B_FMT_NF4) {
     if (L.flags & E4B_FLAG_NF4_PRODUCT_DECODE)
-      smallm_layer_kernel<E4B_FMT_NF4, false><<<sms, kThreads, Geo<E4B_FMT_NF4>::kSmemBytes, st>>>(m, p);
-    else
-      smallm_layer_kernel<E4B_FMT_NF4, true><<<sms, kThreads, Geo<E4B_FMT_NF4>::kSmemBytes, st>>>(m, p);
-  } else {
-    smallm_layer_kernel<E4B_FMT_MXFP4, true><<<sms, kThreads, Geo<E4B_FMT_MXFP4>::kSmemBytes, st>>>(m, p);
+      return launch_dependent(smallm_layer_kernel<E4B_FMT_NF4, false>, dim3(sms), dim3(kThreads),
+                              Geo<E4B_FMT_NF4>::kSmemBytes, st, m, p);
+    return launch_dependent(smallm_layer_kernel<E4B_FMT_NF4, true>, dim3(sms), dim3(kThreads),
+                            Geo<E4B_FMT_NF4>::kSmemBytes, st, m, p);
   }
-  return cudaGetLastError();
+  return launch_dependent(smallm_layer_kernel<E4B_FMT_MXFP4, true>, dim3(sms), dim3(kThreads),
+                          Geo<E4B_FMT_MXFP4>::kSmemBytes, st, m, p);
 }
 
 }  // namespace e4b
