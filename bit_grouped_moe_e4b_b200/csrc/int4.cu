@@ -8,25 +8,32 @@
 // grouped-nf4-gemm README).
 //
 // GEMV design (HBM-bound: 0.5625 bytes per weight, read once):
-//   * one CTA per SM; it quantises the token (or each routed slot's row) to
-//     int8 with one fp32 scale per row into shared memory, laid out so a
-//     16-byte load pairs with the nibbles of one 4-byte code word: per
-//     32-weight block two 16-byte planes (word i holds the bytes of the even
-//     or odd positions of weights 8i..8i+7), plus -8 * (block sum) as int16;
+//   * one CTA of 8 warps per SM; it quantises the token (or each routed
+//     slot's row) to int8 in shared memory, one fp32 product per value,
+//     laid out so a 16-byte load pairs with the nibbles of one 4-byte code
+//     word: per 32-weight block two 16-byte planes (word i holds the bytes of
+//     the even or odd positions of weights 8i..8i+7), plus -8 * (block sum)
+//     as int16;
 //   * an item is four weight rows (two outputs) over a chunk of up to 128
-//     blocks (2 KiB of codes a row); every streaming warp owns a contiguous
-//     run of items and pipelines them through kStages shared-memory stages
-//     that bulk copies fill; lane 0 issues the copies and writes the item's
-//     descriptor next to the stage, so the other lanes only read it;
+//     blocks; every warp owns a contiguous run of items and keeps kStages of
+//     them in flight in its own shared-memory stages, filled by bulk copies
+//     that the whole warp starts (lane 0 writes the item's descriptor and
+//     posts the bytes; lanes 0-3 copy one row position each, two
+//     neighbouring rows of one expert in one copy when the chunk is the
+//     whole row; the scales ride along when 16-byte aligned);
 //   * a code word w gives (w ^ 0x88888888) & 0x0F0F0F0F = q + 8 of the even
 //     positions and (w ^ 0x88888888) & 0xF0F0F0F0 = 16 (q + 8) of the odd
 //     ones as unsigned bytes, so two LOP3 and two unsigned x signed dp4a per
 //     word, with the chains seeded by the block's -8 * sum(xq), give exactly
 //     16 * sum(q * xq) = 16 D (|16 D| < 2^20);
-//   * per row and block the warp accumulates s * 16 D in fp32; four row sums
-//     leave the warp in one butterfly and are added to the round's fp32
-//     accumulators in shared memory, which the epilogue (store / SwiGLU /
-//     gate-weighted combine over the routed slots) turns into bf16.
+//   * the 16 block dot products of an item run without branches; the four
+//     row sums leave the warp in one butterfly and are added to the round's
+//     fp32 accumulators in shared memory, which the epilogue (store / SwiGLU
+//     / gate-weighted combine over the routed slots) turns into bf16;
+//   * the kernel is a programmatic dependent of the work before it on the
+//     stream: it waits (griddepcontrol.wait) only before it reads x, the ids
+//     and gates (or, with E4B_FLAG_IDS_READY, after its first copies), and
+//     lets the next kernel launch once its copies are all issued.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -45,7 +52,6 @@ constexpr int kStages = 3;         // per-warp stages in flight
 constexpr int kRows = 4;           // weight rows per item (two outputs)
 constexpr int kChunkBlocks = 128;  // blocks of one row per item (2 KiB of codes)
 constexpr int kLaneBlocks = kChunkBlocks / 32;
-constexpr int kRowBytes = kChunkBlocks * 16;
 constexpr int kStageBytes = kRows * kChunkBlocks * (16 + 2);  // codes, then the rows' fp16 scales
 constexpr int kRoundOutputs = 256;  // outputs whose fp32 sums sit in shared memory at once
 constexpr int kQuantGroups = 8;     // groups of 8 activations a thread keeps in registers
@@ -254,7 +260,7 @@ E4B_DEV void quantize_rows(const Int4Gemv& p, uint8_t* xs, float* s_sx, float* s
 struct __align__(16) ItemDesc {
   const uint16_t* s[kRows];  // scales of the chunk of each row (null: no row)
   uint32_t x0, x1;           // activation rows (byte offsets into xs)
-  uint32_t xsel;             // bit r: row r reads x1
+  uint32_t pad;
   uint32_t nb;               // blocks in the chunk
   uint32_t acc;              // accumulator of the item's first output (2 floats an output)
   uint32_t flags;            // bits 0-3: row r present; bit 4: the item has its second output
