@@ -478,21 +478,26 @@ def run_int4(wl, steps, warmup, hbm, peak_src, cpu_baseline=True):
         ("int4_gemv_down", dn_ms, dn_bytes)
     achieved = dom_b / (dom_ms * 1e-3) / 1e9
 
-    # end to end through the public call with host buffers: x, ids and gates
-    # in from pinned memory, y out, every step
-    x_pin = x_h.pin_memory()
-    ids_pin = [torch.tensor(p, dtype=torch.int32).pin_memory() for p in pairs]
-    g_pin = torch.from_numpy(gates_h).pin_memory()
-    y_pin = torch.empty((H,), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(x)
-    idd = torch.empty(2, dtype=torch.int32, device=dev)
+    # end to end through the public layer call (e4b_moe_forward on the int4-b32
+    # stacks, one call a step) with host buffers: x, ids and gates in from
+    # pinned memory, y out, every step
+    layer = e4b.PackedLayer("int4b32", E, H, I, gc, gs, dc, ds)
+    ws = e4b.workspace(layer, 1, 2, dev)
+    x_pin = x_h.reshape(1, H).pin_memory()
+    ids_pin = [torch.tensor([p], dtype=torch.int32).pin_memory() for p in pairs]
+    g_pin = torch.from_numpy(gates_h.reshape(1, 2)).pin_memory()
+    y_pin = torch.empty((1, H), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty((1, H), dtype=torch.bfloat16, device=dev)
+    idd = torch.empty((1, 2), dtype=torch.int32, device=dev)
+    gd = torch.empty((1, 2), dtype=torch.float32, device=dev)
+    yd = torch.empty((1, H), dtype=torch.bfloat16, device=dev)
 
     def e2e_step(i):
         xd.copy_(x_pin, non_blocking=True)
         idd.copy_(ids_pin[i % len(ids_pin)], non_blocking=True)
-        g_d.copy_(g_pin, non_blocking=True)
-        step(i, xin=xd, ids=idd)
-        y_pin.copy_(y, non_blocking=True)
+        gd.copy_(g_pin, non_blocking=True)
+        e4b.e4b_moe_forward(layer, xd, idd, gd, yd, ws)
+        y_pin.copy_(yd, non_blocking=True)
 
     for i in range(max(warmup, 3)):
         e2e_step(i)
@@ -505,6 +510,8 @@ def run_int4(wl, steps, warmup, hbm, peak_src, cpu_baseline=True):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / steps
+    if e4b.e4b_read_device_status(ws) != 0:
+        raise RuntimeError("device status set during the end-to-end loop")
     line = {
         "metric": "int4-b32 decode: packed-weight HBM GB/s of one token through the MoE layer (GEMVs)",
         "value": (gu_bytes + dn_bytes) / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": steps,

@@ -362,11 +362,88 @@ e4b_status e4b_gemv_int4_b32(const e4b_int4_gemv_args* a, uint32_t flags, void* 
   return cuda_status(launch_int4_gemv(p, static_cast<cudaStream_t>(stream), sm_count()));
 }
 
+// Workspace of the int4-b32 decode path: the status words, then h [top_k, I].
+static size_t int4_layer_ws_bytes(int64_t I, int64_t top_k) {
+  return size_t(kStatusBytes) + align_up(size_t(top_k) * size_t(I) * 2, 256);
+}
+
 e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
                                   size_t* bytes) {
   if (!w || !bytes || T < 0 || top_k <= 0 || w->E <= 0 || w->H <= 0 || w->I <= 0)
     return E4B_ERR_INVALID_ARG;
-  *bytes = moe_ws_layout(w->E, w->H, w->I, T, top_k).total;
+  *bytes = w->fmt == E4B_FMT_INT4B32 ? int4_layer_ws_bytes(w->I, top_k)
+                                     : moe_ws_layout(w->E, w->H, w->I, T, top_k).total;
+  return E4B_OK;
+}
+
+// The layer on int4-b32 stacks: two decode GEMV launches a token.
+static e4b_status moe_forward_int4(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
+                            const int32_t* ids, const float* gates, uint16_t* y, void* ws, size_t ws_bytes,
+                            uint32_t flags, void* stream) {
+  const int64_t E = w->E, H = w->H, I = w->I;
+  if (H % E4B_INT4_BLOCK || I % E4B_INT4_BLOCK || top_k > int4_gemv_max_slots()) return E4B_ERR_UNSUPPORTED;
+  if (w->gate_up_layout != E4B_GATE_UP_HALVES || w->activation != E4B_ACT_SWIGLU || w->gate_up_bias ||
+      w->down_bias)
+    return E4B_ERR_UNSUPPORTED;
+  if (flags & ~E4B_FLAG_TEST_TIMEOUT) return E4B_ERR_UNSUPPORTED;
+  if (int64_t(top_k) * I > 200 * 1024 || int4_gemv_warps(top_k, I) <= 0 || int4_gemv_warps(1, H) <= 0)
+    return E4B_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (T == 0) return E4B_OK;
+  if (!x || !ids || !gates || !y || !ws || !w->gate_up_codes || !w->gate_up_scales || !w->down_codes ||
+      !w->down_scales)
+    return E4B_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || !aligned16(w->gate_up_codes) ||
+      !aligned16(w->down_codes) || (reinterpret_cast<uintptr_t>(w->gate_up_scales) & 1u) ||
+      (reinterpret_cast<uintptr_t>(w->down_scales) & 1u))
+    return E4B_ERR_MISALIGNED;
+  if (ws_bytes < int4_layer_ws_bytes(I, top_k)) return E4B_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* status = static_cast<int32_t*>(ws);
+  uint16_t* h = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  // the status words describe this call
+  if (cudaMemsetAsync(status, 0, kStatusBytes, s) != cudaSuccess) return E4B_ERR_CUDA;
+  mark(0, s);
+  const int sms = sm_count();
+  for (int64_t t = 0; t < T; ++t) {
+    Int4Gemv gu{};
+    gu.epilogue = E4B_EPI_SWIGLU;
+    gu.E = int(E);
+    gu.n_slots = top_k;
+    gu.nx = 1;
+    gu.N = 2 * I;
+    gu.K = H;
+    gu.codes = w->gate_up_codes;
+    gu.scales = static_cast<const uint16_t*>(w->gate_up_scales);
+    gu.ids = ids + t * top_k;
+    gu.x = x + t * H;
+    gu.ld_x = 0;
+    gu.y = h;
+    gu.ld_y = I;
+    gu.status = status;
+    gu.flags = flags;
+    if (launch_int4_gemv(gu, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+    Int4Gemv dn{};
+    dn.epilogue = E4B_EPI_COMBINE;
+    dn.E = int(E);
+    dn.n_slots = top_k;
+    dn.nx = top_k;
+    dn.N = H;
+    dn.K = I;
+    dn.codes = w->down_codes;
+    dn.scales = static_cast<const uint16_t*>(w->down_scales);
+    dn.ids = ids + t * top_k;
+    dn.gates = gates + t * top_k;
+    dn.x = h;
+    dn.ld_x = I;
+    dn.y = y + t * H;
+    dn.status = status;
+    dn.flags = flags | E4B_FLAG_IDS_READY;  // the gate_up launch has read this token's ids
+    if (launch_int4_gemv(dn, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+  }
+  mark(4, s);
+  g_last_path = E4B_PATH_INT4_GEMV;
+  g_last_launches = int32_t(2 * T);
   return E4B_OK;
 }
 
@@ -376,6 +453,8 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   if (!w || T < 0 || top_k <= 0) return E4B_ERR_INVALID_ARG;
   const int64_t E = w->E, H = w->H, I = w->I;
   if (E <= 0 || H <= 0 || I <= 0 || top_k > E) return E4B_ERR_INVALID_ARG;
+  if (w->fmt == E4B_FMT_INT4B32)
+    return moe_forward_int4(w, x, T, top_k, ids, gates, y, ws, ws_bytes, flags, stream);
   e4b_status st = check_projection(w->fmt, 2 * I, H, true);
   if (st != E4B_OK) return st;
   st = check_projection(w->fmt, H, I, false);

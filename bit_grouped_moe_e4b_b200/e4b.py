@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libe4b.so")
 
 E4B_OK = 0
-E4B_FMT_NF4, E4B_FMT_MXFP4 = 0, 1
+E4B_FMT_NF4, E4B_FMT_MXFP4, E4B_FMT_INT4B32 = 0, 1, 2
 E4B_EPI_STORE, E4B_EPI_SWIGLU, E4B_EPI_COMBINE = 0, 1, 2
 E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05, E4B_PATH_INT4_GEMV = 0, 1, 2, 3
 FLAG_FORCE_GEMV = 0x1
@@ -32,7 +32,7 @@ STATUS_NAMES = {
     3: "E4B_ERR_WORKSPACE_TOO_SMALL", 4: "E4B_ERR_CUDA", 5: "E4B_ERR_DEVICE_TIMEOUT",
     6: "E4B_ERR_BAD_EXPERT_ID", 7: "E4B_ERR_MISALIGNED", 8: "E4B_ERR_EXCEEDS_STATIC_SCRATCH",
 }
-FMT = {"nf4": E4B_FMT_NF4, "mxfp4": E4B_FMT_MXFP4}
+FMT = {"nf4": E4B_FMT_NF4, "mxfp4": E4B_FMT_MXFP4, "int4b32": E4B_FMT_INT4B32}
 
 # Every symbol include/e4b.h declares.
 EXPORTED = [

@@ -65,7 +65,9 @@ typedef enum {
                                         16 MiB static scratch */
 } e4b_status;
 
-typedef enum { E4B_FMT_NF4 = 0, E4B_FMT_MXFP4 = 1 } e4b_format;
+/* E4B_FMT_INT4B32: int4-b32 stacks (see e4b_gemv_int4_b32); only
+ * e4b_moe_forward / e4b_moe_workspace_size take it, as the batch-1 decode path. */
+typedef enum { E4B_FMT_NF4 = 0, E4B_FMT_MXFP4 = 1, E4B_FMT_INT4B32 = 2 } e4b_format;
 
 /* Which kernel family ran last (e4b_last_path). */
 typedef enum {
@@ -396,6 +398,14 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
  *   flags E4B_FLAG_* (0 = choose the path from the shape)
  * The path is chosen on the host from T*top_k/E with no device sync, so the
  * call is graph-capturable. T == 0 is a no-op.
+ * With w->fmt == E4B_FMT_INT4B32 (stacks as in e4b_gemv_int4_b32: scales fp16)
+ * the layer runs the batch-1 int4-b32 decode GEMVs token by token: for each
+ * token the gate_up GEMV with the SwiGLU epilogue into h [top_k, I] in ws,
+ * then the down GEMV with the combine epilogue into y[t] (2 launches a
+ * token; the intermediate h and the activations are quantised as described
+ * there). The expert variant must be the plain one (halves, SwiGLU, no
+ * biases), top_k <= 64, H % 32 == 0 and I % 32 == 0; flags: 0 or
+ * E4B_FLAG_TEST_TIMEOUT. Otherwise E4B_ERR_UNSUPPORTED.
  */
 e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
                            const int32_t* ids, const float* gates, uint16_t* y, void* ws,

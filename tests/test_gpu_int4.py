@@ -223,3 +223,21 @@ def test_timeout_path_records_status_and_returns():
     y2 = torch.empty((2, 64), dtype=torch.bfloat16, device="cuda")
     e4b.e4b_gemv_int4_b32("store", codes, scales, ids, x.cuda(), y2, E=2, N=64, K=1024)
     assert_close(y2.float().cpu().numpy(), q4.gemv_int4b32_ref(xf, [1, 0], rc, rs, "store"), "after a timeout")
+
+
+def test_layer_forward_int4_through_moe_forward():
+    # e4b_moe_forward on int4-b32 stacks: two decode GEMVs a token, in one call
+    rng = np.random.default_rng(21)
+    E, H, I, T, k = 8, 512, 1024, 3, 2
+    gc, gs, rgc, rgs = _stack(rng, E, 2 * I, H)
+    dc, ds, rdc, rds = _stack(rng, E, H, I)
+    layer = e4b.PackedLayer("int4b32", E, H, I, gc, gs, dc, ds)
+    x, xf = _bf16(rng, (T, H))
+    ids = np.array([[3, 5], [0, 0], [7, 2]], np.int32)  # a duplicate expert in token 1
+    gates = np.array([[0.6, 0.4], [0.5, 0.5], [0.9, 0.1]], np.float32)
+    y = e4b.moe_forward(layer, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(gates).cuda())
+    torch.cuda.synchronize()
+    assert e4b.e4b_last_path() == e4b.E4B_PATH_INT4_GEMV and e4b.e4b_last_launch_count() == 2 * T
+    for t in range(T):
+        ref = q4.int4b32_decode_layer_ref(xf[t], list(ids[t]), gates[t], rgc, rgs, rdc, rds)
+        assert_close(y[t].float().cpu().numpy(), ref, f"int4 layer token {t}")

@@ -206,3 +206,25 @@ def test_int4_argument_checks():
     assert g(p + 2, p, 2, 4, 64, p, p, None) == 7
     assert g(None, p, 2, 4, 64, p, p, None) == 1
     assert g(None, None, 0, 4, 64, None, None, None) == 0
+
+
+def test_int4_layer_argument_checks():
+    # e4b_moe_forward with the int4-b32 format: the batch-1 decode path
+    L = e4b.lib()
+    p = 4096
+    n = ctypes.c_size_t(0)
+    w = e4b.MoeWeights(e4b.E4B_FMT_INT4B32, 8, 256, 512, p, p, p, p)
+    assert L.e4b_moe_workspace_size(ctypes.byref(w), 3, 2, ctypes.byref(n)) == 0
+    assert n.value >= 256 + 2 * 512 * 2          # status words and h [top_k, I]
+    fwd = L.e4b_moe_forward
+    q = ctypes.c_void_p(p)
+    big = 1 << 20
+    assert fwd(ctypes.byref(w), None, 0, 2, None, None, None, None, 0, 0, None) == 0  # T == 0
+    assert fwd(ctypes.byref(w), q, 1, 2, q, q, None, q, big, 0, None) == 1            # null y
+    assert fwd(ctypes.byref(w), q, 1, 2, q, q, q, q, 16, 0, None) == 3                # workspace too small
+    assert fwd(ctypes.byref(w), q, 1, 2, q, q, q, q, big, e4b.FLAG_FORCE_GEMV, None) == 2
+    bad = e4b.MoeWeights(e4b.E4B_FMT_INT4B32, 8, 256, 496, p, p, p, p)              # I % 32
+    assert fwd(ctypes.byref(bad), q, 1, 2, q, q, q, q, big, 0, None) == 2
+    var = e4b.MoeWeights(e4b.E4B_FMT_INT4B32, 8, 256, 512, p, p, p, p, 1)            # interleaved
+    assert fwd(ctypes.byref(var), q, 1, 2, q, q, q, q, big, 0, None) == 2
+    assert fwd(ctypes.byref(w), ctypes.c_void_p(p + 2), 1, 2, q, q, q, q, big, 0, None) == 7
