@@ -140,6 +140,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's value (the slowest rank sets a multi-GPU
+    time); `value` itself without a process group."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ GPU arm
 def build_layer(wl, device):
     import torch
@@ -254,10 +266,7 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist):
     phases = {name: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(steps)]))
               for name, a, b in spans}
     phases["_note"] = "each launch alone (events between launches); the timed steps overlap them"
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
 
     # end-to-end through the C ABI with host buffers (pinned), copies inside
     x_pin = x_h.pin_memory()
@@ -287,10 +296,7 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if e4b.e4b_read_device_status(ws) != 0:
         raise RuntimeError("device status set during the timed loops")
     return {
