@@ -67,10 +67,18 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def _source_hash() -> str:
+# The sources a kernel is compiled from: its own file and the device headers.
+_KERNEL_SOURCES = {
+    "smallm_layer": "smallm.cu", "gate_up": "tc_gemm.cu", "down": "tc_gemm.cu",
+    "int4_gemv_gate_up": "int4.cu", "int4_gemv_down": "int4.cu",
+}
+_DEVICE_HEADERS = ("common.cuh", "sm100.cuh", "launch.h", "tmap.h")
+
+
+def _source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_grouped_moe_e4b_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in (_KERNEL_SOURCES[kernel],) + _DEVICE_HEADERS:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -79,13 +87,13 @@ def _source_hash() -> str:
 
 def _traffic(key: str, kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the kernel's current sources; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         rec = d[key][kernel]
-        if rec.get("source_hash") != _source_hash():
+        if rec.get("source_hash") != _source_hash(kernel):
             return None
         return float(rec["dram_bytes_per_launch"])
     except Exception:

@@ -4,6 +4,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "ep.h"
 #include "launch.h"
 
 namespace {
@@ -360,6 +361,41 @@ e4b_status e4b_gemv_int4_b32(const e4b_int4_gemv_args* a, uint32_t flags, void* 
   g_last_path = E4B_PATH_INT4_GEMV;
   g_last_launches = 1;
   return cuda_status(launch_int4_gemv(p, static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_ep_dest(const int32_t* ids, int64_t n, int32_t E, int32_t epr, int32_t* dest, void* stream) {
+  if (n < 0 || E <= 0 || epr <= 0 || E % epr) return E4B_ERR_INVALID_ARG;
+  g_last_launches = 0;
+  if (n == 0) return E4B_OK;
+  if (!ids || !dest) return E4B_ERR_INVALID_ARG;
+  g_last_launches = 1;
+  return cuda_status(launch_ep_dest(ids, n, E, epr, dest, static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_ep_pack(const uint16_t* x, int64_t H, const int32_t* ids, const float* gates, int32_t top_k,
+                       const int32_t* perm, const int64_t* offsets, int32_t G, int64_t R_max, int32_t epr,
+                       uint16_t* xs, int32_t* local_ids, float* local_gates, void* stream) {
+  if (H <= 0 || top_k <= 0 || G <= 0 || R_max < 0 || epr <= 0) return E4B_ERR_INVALID_ARG;
+  if (H % 8) return E4B_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (R_max == 0) return E4B_OK;
+  if (!x || !ids || !gates || !perm || !offsets || !xs || !local_ids || !local_gates) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xs)) return E4B_ERR_MISALIGNED;
+  g_last_launches = 1;
+  return cuda_status(launch_ep_pack(x, H, ids, gates, top_k, perm, offsets, G, R_max, epr, xs, local_ids,
+                                    local_gates, static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_ep_combine(const uint16_t* ys, int64_t H, const int32_t* inv_perm, int64_t T, int32_t top_k,
+                          uint16_t* y, void* stream) {
+  if (H <= 0 || T < 0 || top_k <= 0) return E4B_ERR_INVALID_ARG;
+  if (H % 8) return E4B_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (T == 0) return E4B_OK;
+  if (!inv_perm || !y || !ys) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(ys) || !aligned16(y)) return E4B_ERR_MISALIGNED;
+  g_last_launches = 1;
+  return cuda_status(launch_ep_combine(ys, H, inv_perm, T, top_k, y, static_cast<cudaStream_t>(stream), sm_count()));
 }
 
 // Workspace of the int4-b32 decode path: the status words, then h [top_k, I].

@@ -42,6 +42,7 @@ EXPORTED = [
     "e4b_last_launch_count",
     "e4b_status_string", "e4b_version",
     "e4b_quantize_int4_b32", "e4b_gptq_pack_int4_b32", "e4b_gemv_int4_b32",
+    "e4b_ep_dest", "e4b_ep_pack", "e4b_ep_combine",
 ]
 EPI = {"store": E4B_EPI_STORE, "swiglu": E4B_EPI_SWIGLU, "combine": E4B_EPI_COMBINE}
 
@@ -135,6 +136,9 @@ def lib() -> ctypes.CDLL:
         "e4b_quantize_int4_b32": [vp, i64, i64, i64, vp, vp, vp],
         "e4b_gptq_pack_int4_b32": [vp, vp, i64, i64, i64, vp, vp, vp],
         "e4b_gemv_int4_b32": [ctypes.POINTER(Int4GemvArgs), ctypes.c_uint32, vp],
+        "e4b_ep_dest": [vp, i64, i32, i32, vp, vp],
+        "e4b_ep_pack": [vp, i64, vp, vp, i32, vp, vp, i32, i64, i32, vp, vp, vp, vp],
+        "e4b_ep_combine": [vp, i64, vp, i64, i32, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -273,6 +277,25 @@ def int4_decode_layer(x, expert_ids, gates, gu_codes, gu_scales, dn_codes, dn_sc
     e4b_gemv_int4_b32("combine", dn_codes, dn_scales, expert_ids, h, y, E=E, N=H, K=I, gates=gates, ld_x=I,
                       flags=FLAG_IDS_READY)
     return y
+
+
+# ---------------------------------------------------------- expert parallel
+def e4b_ep_dest(ids, E, epr, dest, stream=None):
+    _dev(ids, dest)
+    _check(lib().e4b_ep_dest(_ptr(ids), ids.numel(), E, epr, _ptr(dest), _stream(stream)), "e4b_ep_dest")
+
+
+def e4b_ep_pack(x, ids, gates, perm, offsets, G, R_max, epr, xs, local_ids, local_gates, stream=None):
+    _dev(x, ids, gates, perm, offsets, xs, local_ids, local_gates)
+    _check(lib().e4b_ep_pack(_ptr(x), x.shape[1], _ptr(ids), _ptr(gates), ids.shape[1], _ptr(perm), _ptr(offsets),
+                             G, R_max, epr, _ptr(xs), _ptr(local_ids), _ptr(local_gates), _stream(stream)),
+           "e4b_ep_pack")
+
+
+def e4b_ep_combine(ys, inv_perm, T, top_k, y, stream=None):
+    _dev(ys, inv_perm, y)
+    _check(lib().e4b_ep_combine(_ptr(ys), y.shape[1], _ptr(inv_perm), T, top_k, _ptr(y), _stream(stream)),
+           "e4b_ep_combine")
 
 
 def e4b_route_workspace_size(T, top_k, E) -> int:

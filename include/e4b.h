@@ -372,6 +372,39 @@ typedef struct {
 
 e4b_status e4b_gemv_int4_b32(const e4b_int4_gemv_args* args, uint32_t flags, void* stream);
 
+/* ------------------------------------------------------ expert parallel */
+/*
+ * Expert parallelism over G ranks, one process per GPU (the pages describe one
+ * GPU; this split is the library's own): rank r holds the experts
+ * [r * epr, (r + 1) * epr) of the layer. A rank routes its tokens' slots by
+ * destination rank (e4b_ep_dest, then e4b_route with E = G), packs the routed
+ * rows in that order (e4b_ep_pack), exchanges them with an all-to-all (the
+ * caller's NCCL), runs its experts on the rows it received with
+ * e4b_moe_forward (one slot a row: ids = the local expert ids, gates = the
+ * slot gates), sends the outputs back and sums each token's rows
+ * (e4b_ep_combine). Every slot's output is rounded to bf16 before the sum, so
+ * y differs from the one-GPU layer by at most top_k bf16 roundings.
+ */
+
+/* dest[i] = ids[i] / epr for ids[i] in [0, E), else -1 (the routing pass then
+ * drops the slot and records E4B_ERR_BAD_EXPERT_ID). ids, dest: int32 [n]. */
+e4b_status e4b_ep_dest(const int32_t* ids, int64_t n, int32_t E, int32_t epr, int32_t* dest, void* stream);
+
+/* For every position p < offsets[G] of the destination order (perm and
+ * offsets from e4b_route over dest with E = G): xs[p] = x[perm[p] / top_k]
+ * (bf16 [R_max, H]), local_ids[p] = ids[perm[p]] % epr, local_gates[p] =
+ * gates[perm[p]]. x and xs 16-byte aligned, H % 8 == 0. Positions from
+ * offsets[G] to R_max are not written. */
+e4b_status e4b_ep_pack(const uint16_t* x, int64_t H, const int32_t* ids, const float* gates, int32_t top_k,
+                       const int32_t* perm, const int64_t* offsets, int32_t G, int64_t R_max, int32_t epr,
+                       uint16_t* xs, int32_t* local_ids, float* local_gates, void* stream);
+
+/* y[t] = bf16(sum_j ys[inv_perm[t * top_k + j]]) with fp32 sums; slots whose
+ * inv_perm is -1 are left out (a token with none gets 0). ys bf16 [R, H] in
+ * the destination order, y bf16 [T, H]; 16-byte aligned, H % 8 == 0. */
+e4b_status e4b_ep_combine(const uint16_t* ys, int64_t H, const int32_t* inv_perm, int64_t T, int32_t top_k,
+                          uint16_t* y, void* stream);
+
 /* ---------------------------------------------------------- whole layer */
 
 /* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots.
