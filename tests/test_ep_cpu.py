@@ -11,6 +11,7 @@ import sys
 from datetime import timedelta
 
 import numpy as np
+import pytest
 import torch
 
 from conftest import ROOT
@@ -71,7 +72,7 @@ def _layer(E, H, I):
     return gc, gs, dc, ds
 
 
-def _rank(rank, world, port, q):
+def _rank(rank, world, port, q, local_only=False):
     import torch.distributed as dist
 
     sys.path.insert(0, ROOT)
@@ -94,6 +95,8 @@ def _rank(rank, world, port, q):
     ids, gates = synth.random_ids(rng, T, k, E)
     if rank == 1:
         ids[2, 1] = ids[2, 0]  # a token sending both slots to one expert
+    if local_only:  # every slot stays on its own rank: the cross-rank exchanges are empty
+        ids = (ids % epr + rank * epr).astype(np.int32)
     y = ep.forward(torch.from_numpy(x), torch.from_numpy(ids), torch.from_numpy(gates)).numpy()
     ref = oracle.moe_forward_ref("nf4", x.astype(np.float64), ids, gates, gc, gs, dc, ds, E, H, I)
     err = float(np.max(np.abs(y - ref) / (1 + np.abs(ref))))
@@ -108,13 +111,14 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def test_expert_parallel_layer_on_two_gloo_ranks():
+@pytest.mark.parametrize("local_only", [False, True])
+def test_expert_parallel_layer_on_two_gloo_ranks(local_only):
     import torch.multiprocessing as mp
 
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q, local_only)) for r in range(2)]
     for p in procs:
         p.start()
     got = sorted(q.get(timeout=300) for _ in procs)
