@@ -228,3 +228,39 @@ def test_int4_layer_argument_checks():
     var = e4b.MoeWeights(e4b.E4B_FMT_INT4B32, 8, 256, 512, p, p, p, p, 1)            # interleaved
     assert fwd(ctypes.byref(var), q, 1, 2, q, q, q, q, big, 0, None) == 2
     assert fwd(ctypes.byref(w), ctypes.c_void_p(p + 2), 1, 2, q, q, q, q, big, 0, None) == 7
+
+
+def test_ep_argument_checks():
+    L = e4b.lib()
+    p = 4096
+    assert L.e4b_ep_dest(p, 10, 8, 3, p, None) == 1            # 8 experts do not split over ranks of 3
+    assert L.e4b_ep_dest(None, 0, 8, 4, None, None) == 0       # nothing to do
+    assert L.e4b_ep_dest(None, 4, 8, 4, p, None) == 1
+    pack = L.e4b_ep_pack
+    assert pack(p, 100, p, p, 2, p, p, 2, 8, 4, p, p, p, None) == 2        # H % 8
+    assert pack(p + 8, 128, p, p, 2, p, p, 2, 8, 4, p, p, p, None) == 7    # x not 16-byte aligned
+    assert pack(p, 128, p, p, 2, p, p, 2, 0, 4, None, None, None, None) == 0
+    assert pack(p, 128, None, p, 2, p, p, 2, 8, 4, p, p, p, None) == 1
+    comb = L.e4b_ep_combine
+    assert comb(p, 128, p, 4, 2, p + 4, None) == 7
+    assert comb(p, 100, p, 4, 2, p, None) == 2                 # H % 8
+    assert comb(None, 128, None, 0, 2, None, None) == 0
+
+
+def test_expert_parallel_layer_rejects_a_bad_split():
+    import torch.distributed as dist
+    from bit_grouped_moe_e4b_b200.ep import ExpertParallelLayer
+
+    class _L:
+        E = 3
+
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        with pytest.raises(ValueError):
+            ExpertParallelLayer(_L(), 8)   # 8 experts on one rank, but the local layer holds 3
+    finally:
+        dist.destroy_process_group()
