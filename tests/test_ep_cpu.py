@@ -1,4 +1,4 @@
-"""Expert parallelism on two CPU ranks (gloo): ExpertParallelLayer's routing by
+"""Expert parallelism on CPU ranks (gloo; 2 and 4 ranks): ExpertParallelLayer's routing by
 destination rank, the all-to-all exchanges of counts, rows, local ids and
 gates, the return of the outputs and the combine, with the device steps taken
 by a CPU double built on the oracle. Each rank's output must match the
@@ -111,20 +111,20 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("local_only", [False, True])
-def test_expert_parallel_layer_on_two_gloo_ranks(local_only):
+@pytest.mark.parametrize("world,local_only", [(2, False), (2, True), (4, False)])
+def test_expert_parallel_layer_on_gloo_ranks(world, local_only):
     import torch.multiprocessing as mp
 
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, q, local_only)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q, local_only)) for r in range(world)]
     for p in procs:
         p.start()
     got = sorted(q.get(timeout=300) for _ in procs)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert [g[2] for g in got] == [(5, 128), (8, 128)]
+    assert [g[2] for g in got] == [(5 + 3 * r, 128) for r in range(world)]
     for rank, err, _ in got:
         assert err <= 1e-2, f"rank {rank}: max scaled error {err}"
