@@ -329,9 +329,12 @@ e4b_status e4b_gptq_pack_int4_b32(const int32_t* qweight, const uint16_t* gptq_s
 /*
  * e4b_gemv_int4_b32 -- [S] the decode GEMV: one token against its n_slots
  * routed experts e_j = expert_ids[j] of an int4-b32 stack, in one launch.
- * Every CTA quantises the token row(s) to int8 with one fp32 scale per row
- * (sx = fp32(max|x|) / 127, xq = clamp(rint(fp32(x / sx)), -127, 127)); per
- * 32-weight block the products q * xq are summed exactly in int32; then
+ * Every CTA quantises the token row(s) to int8 with one fp32 scale per row:
+ * amax = max|x|, sx = fp32(amax / 127), r = fp32(127 / amax),
+ * xq = clamp(rint(fp32(x * r)), -127, 127), ties to even (a row whose r is
+ * not finite -- all zero, or amax below 127 / FLT_MAX -- gets sx = 0 and
+ * xq = 0); per 32-weight block the products q * xq are summed exactly in
+ * int32; then
  *   acc[j, n] = sx_j * sum_b s[e_j, n, b] * D[e_j, n, b]   (fp32)
  * and the epilogue writes bf16:
  *   E4B_EPI_STORE    y [n_slots, N] (row stride ld_y >= N):  bf16(acc[j, n])
