@@ -194,7 +194,8 @@ def _roofline(path, kernel, kb, dur_s, wl, ids, key, hbm, bf16, bf16_sus, peak_s
 
 
 def kernel_bytes(wl, T, ids):
-    """Algorithmic bytes per launch of each kernel."""
+    """Algorithmic bytes per launch of each kernel: the packed bytes of the active experts plus the
+    activation rows in and out, and the routing ids and gates."""
     # storage per weight: 4-bit code + fp32 absmax per 64 (NF4) or one e8m0 byte per 32 (MXFP4)
     bpw = 0.5 + (4.0 / 64 if wl.fmt == "nf4" else 1.0 / 32)
     active = len(np.unique(ids))

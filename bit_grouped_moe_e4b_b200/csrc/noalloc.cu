@@ -21,6 +21,9 @@ void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
 // Device address of the scratch array on the current device, looked up once
 // per device (the array's name in host code is only a host-side stand-in).
+// The cached address belongs to the device's current context: a
+// cudaDeviceReset (or any teardown of the primary context) invalidates it, so
+// the process must not call this entry point again on that device afterwards.
 e4b_status scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return E4B_ERR_CUDA;
@@ -44,10 +47,13 @@ extern "C" e4b_status e4b_moe_forward_noalloc(const e4b_moe_weights* w, const ui
   size_t full = 0;
   e4b_status st = e4b_moe_workspace_size(w, T, top_k, &full);
   if (st != E4B_OK) return st;
-  // The staging copy of the routed rows is optional: without room for it the
-  // large-M path gathers the rows inside its kernel.
-  if (e4b::moe_workspace_min_bytes(w->E, w->H, w->I, T, top_k) > kNoallocScratchBytes)
-    return E4B_ERR_EXCEEDS_STATIC_SCRATCH;
+  // int4-b32 stacks need only the status words and h [top_k, I], whatever T.
+  // For NF4 / MXFP4 the staging copy of the routed rows is optional: without
+  // room for it the large-M path gathers the rows inside its kernel.
+  const size_t need = w->fmt == E4B_FMT_INT4B32
+                          ? full
+                          : e4b::moe_workspace_min_bytes(w->E, w->H, w->I, T, top_k);
+  if (need > kNoallocScratchBytes) return E4B_ERR_EXCEEDS_STATIC_SCRATCH;
   if (T == 0) return e4b_moe_forward(w, x, T, top_k, ids, gates, y, nullptr, 0, flags, stream);
   void* scratch = nullptr;
   st = scratch_for_current_device(&scratch);

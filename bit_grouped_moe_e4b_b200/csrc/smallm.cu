@@ -15,7 +15,7 @@
 //    weight rows (two TMA tiles, 128B-swizzled), the chunk of each routed
 //    activation row (four-row TMA gathers from x, or TMA tiles of h) and the
 //    block scales into a shared-memory stage (four stages of 44 KB);
-//  * eight consumer warps take 32 weight rows each from a stage, decode the
+//  * sixteen consumer warps take 16 weight rows each from a stage, decode the
 //    codes through a 256-entry byte table (conflict-free shared loads) into
 //    the A fragments of mma.sync m16n8k16 (bf16 in, fp32 accumulate), with the
 //    activations of the stage as B, and release the stage;

@@ -433,7 +433,10 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
  *         the optional staging copy of the routed rows)
  *   flags E4B_FLAG_* (0 = choose the path from the shape)
  * The path is chosen on the host from T*top_k/E with no device sync, so the
- * call is graph-capturable. T == 0 is a no-op.
+ * call is graph-capturable. T == 0 is a no-op. Limits: E <= 1024 and
+ * T*top_k < 2^31; the large-M (tcgen05) path takes E <= 256, so with E > 256
+ * the small-M path runs whatever T (E4B_FLAG_FORCE_TCGEN05 then returns
+ * E4B_ERR_UNSUPPORTED).
  * With w->fmt == E4B_FMT_INT4B32 (stacks as in e4b_gemv_int4_b32: scales fp16)
  * the layer runs the batch-1 int4-b32 decode GEMVs token by token: for each
  * token the gate_up GEMV with the SwiGLU epilogue into h [top_k, I] in ws,
@@ -461,14 +464,18 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
  * scratch (routing arrays, bf16 intermediate, fp32 accumulator, status word)
  * lives in a 16 MiB array in the library's device memory, which every GPU
  * that loads the library keeps until the process exits. A call whose
- * required scratch (e4b_moe_workspace_size without the optional staging
- * copy) exceeds 16 MiB returns E4B_ERR_EXCEEDS_STATIC_SCRATCH and enqueues
- * nothing (a layer with H=4096, I=14336 and top-2 routing fits up to 227
- * tokens; the staging copy is used while it also fits). Nothing is allocated
- * or freed.
+ * required scratch exceeds 16 MiB returns E4B_ERR_EXCEEDS_STATIC_SCRATCH and
+ * enqueues nothing. The required scratch is, for NF4 and MXFP4 stacks,
+ * e4b_moe_workspace_size without the optional staging copy (a layer with
+ * H=4096, I=14336 and top-2 routing fits up to 227 tokens; the staging copy
+ * is used while it also fits), and for int4-b32 stacks
+ * e4b_moe_workspace_size itself, which does not grow with T. Nothing is
+ * allocated or freed.
  *   - The first call on each device looks up that device's copy of the
  *     array (set-up, once per device); make that first call before any stream
- *     capture begins.
+ *     capture begins. The address found belongs to the device's context as it
+ *     was then: after a cudaDeviceReset on that device, do not call this
+ *     entry point again in the same process.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents; each call re-clears what must start at zero. Calls whose GPU
  *     work overlaps (different streams, or graphs replayed concurrently) race

@@ -137,16 +137,24 @@ def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=N
 
 
 def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_rows=None,
-                        packed_fn=None, variant=None, nf4_decode="product"):
+                        packed_fn=None, variant=None, nf4_decode="product", workers=None):
     """Outputs y[t, n] for the given tokens (and optionally only the given
     output columns n) of the layer whose fp32 expert weights weight_fn(which,
     e) returns ("gate_up" [2I, H], "down" [H, I]); with packed_fn(which, e)
     given instead, the experts arrive already packed (codes, scales).
     nf4_decode: the NF4 weight value as in moe_forward_ref.
 
+    The experts are independent, so they are taken by `workers` threads
+    (default: one per host core, at most one per expert); the C loops run
+    without the interpreter lock. weight_fn / packed_fn are called under a
+    lock, one at a time. Every expert's arithmetic is the serial one.
+
     Returns (y fp64 holding bf16 values [len(tokens), len(cols)], cols,
     packed) where packed[(which, e)] = (codes, scales) this function used.
     """
+    import threading
+    from concurrent.futures import ThreadPoolExecutor
+
     x = np.asarray(x, np.float64)
     ids = np.asarray(ids)
     gates = np.asarray(gates, np.float32)
@@ -154,17 +162,29 @@ def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_row
     cols = np.arange(H) if down_rows is None else np.asarray(down_rows)
     O_slot = {}
     packed = {}
-    for e, pairs in sorted(expert_tokens(ids, tokens).items()):
+    lock = threading.Lock()
+    work = sorted(expert_tokens(ids, tokens).items())
+
+    def one(item):
+        e, pairs = item
+        mine = {}
         for which in ("gate_up", "down"):
-            if packed_fn is not None:
-                packed[(which, e)] = packed_fn(which, e)
-            else:
-                packed[(which, e)] = quantize(fmt, weight_fn(which, e))
+            with lock:
+                src = packed_fn(which, e) if packed_fn is not None else weight_fn(which, e)
+            mine[which] = src if packed_fn is not None else quantize(fmt, src)
+            del src
         X = x[[t for _, t in pairs]]
-        O, _ = expert_term(fmt, X, packed[("gate_up", e)], packed[("down", e)], H, I,
+        O, _ = expert_term(fmt, X, mine["gate_up"], mine["down"], H, I,
                            None if down_rows is None else cols, variant, e, nf4_decode)
-        for r, (slot, _) in enumerate(pairs):
-            O_slot[slot] = O[r]
+        return e, pairs, mine, O
+
+    n = workers or min(len(work), os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=max(1, n)) as ex:
+        for e, pairs, mine, O in ex.map(one, work):
+            for which in ("gate_up", "down"):
+                packed[(which, e)] = mine[which]
+            for r, (slot, _) in enumerate(pairs):
+                O_slot[slot] = O[r]
     y = np.zeros((len(tokens), len(cols)), np.float64)
     for i, t in enumerate(tokens):
         for j in range(k):

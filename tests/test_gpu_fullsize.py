@@ -2,7 +2,9 @@
 times (path chosen from the shape), plus the other kernel path: sampled
 tokens checked against the oracle, which quantises the experts those tokens
 use from the same fp32 weights and compares its codes with the GPU's bit for
-bit."""
+bit. The sample holds at least 32 tokens and covers every active expert's
+first and last routed row and the rows on both sides of each 256-row tile
+boundary of the large-M kernel."""
 
 import numpy as np
 import pytest
@@ -33,6 +35,35 @@ def _layer(wl):
 
 CASES = [(name, T) for name, wl in WORKLOADS.items() for T in wl.T]
 
+TILE_ROWS = 256  # routed rows per tile of the large-M kernel
+
+
+def sample_tokens(ids, E, n_min=32, seed=0):
+    """Tokens whose routed rows include, for every active expert, its first
+    and last row in expert order and the two rows on each side of every
+    TILE_ROWS boundary inside it; then tokens 0, T/2 and T-1, and random
+    tokens up to n_min (all tokens when T <= n_min)."""
+    T, k = ids.shape
+    flat = ids.ravel()
+    perm = np.argsort(flat, kind="stable")
+    counts = np.bincount(flat, minlength=E)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    rows = set()
+    for e in range(E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b == a:
+            continue
+        rows.update((a, b - 1))
+        for j in range(TILE_ROWS, b - a, TILE_ROWS):
+            rows.update((a + j - 1, a + j))
+    tokens = {int(perm[p]) // k for p in rows} | {0, T // 2, T - 1}
+    if T <= n_min:
+        return list(range(T))
+    rng = np.random.default_rng(seed)
+    while len(tokens) < n_min:
+        tokens.add(int(rng.integers(T)))
+    return sorted(tokens)
+
 
 @pytest.mark.parametrize("name,T", CASES)
 def test_workload_sampled_tokens(name, T):
@@ -52,7 +83,8 @@ def test_workload_sampled_tokens(name, T):
     y_other = e4b.moe_forward(layer, x_d, ids_d, g_d, ws=ws, flags=other)
     assert e4b.e4b_read_device_status(ws) == 0
 
-    tokens = sorted({0, T // 2, T - 1})
+    tokens = sample_tokens(ids, wl.E, seed=T)
+    assert len(tokens) >= min(32, T)
     weight_fn = lambda which, e: synth.expert_weight(wl, which, e, "cuda").cpu().numpy()
     # NF4: the small-M path takes the "level" reading, tcgen05 the "product" one
     mode = {e4b.E4B_PATH_GEMV: "level", e4b.E4B_PATH_TCGEN05: "product"}
@@ -72,7 +104,7 @@ def test_workload_sampled_tokens(name, T):
                                                      nf4_decode=other_mode)
     for y, ref, what in ((y_auto, y_ref, "auto"), (y_other, y_ref_other, "other path")):
         got = y.float().cpu().numpy()[tokens]
-        assert_close(got, ref, f"{name} T={T} {what}")
+        assert_close(got, ref, f"{name} T={T} {what}", min_rms=0.1)
     # rows not sampled: finite and equal across the two kernel paths within
     # tolerance (for NF4 the paths' readings differ by one bf16 rounding per
     # weight, far inside it on these N(0, 0.02) weights)

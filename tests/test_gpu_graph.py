@@ -9,9 +9,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from oracle import int4b32 as q4
 from bit_grouped_moe_e4b_b200 import e4b, synth
-from gpu_util import assert_close, small_layer
+from gpu_util import LAYER_MIN_RMS, assert_close, small_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -22,7 +23,9 @@ def _inputs(rng, T, k, E, H):
     return x, torch.from_numpy(ids).cuda(), torch.from_numpy(gates).cuda()
 
 
-def _graph_vs_eager(layer, T, k, flags, seed):
+def _graph_vs_eager(layer, T, k, flags, seed, ref=None):
+    """ref: the oracle's packed stacks; each replay is then also checked
+    against the oracle's layer in the reading of the path that ran."""
     rng = np.random.default_rng(seed)
     x, ids, gates = _inputs(rng, T, k, layer.E, layer.H)
     ws = e4b.workspace(layer, T, k)
@@ -48,14 +51,19 @@ def _graph_vs_eager(layer, T, k, flags, seed):
         torch.cuda.synchronize()
         assert_close(got, want.float().cpu().numpy(), f"graph replay {rep}", tol=2e-2)
         assert e4b.e4b_read_device_status(ws) == 0
+        if ref is not None:
+            mode = "level" if path == e4b.E4B_PATH_GEMV else "product"
+            y_ref = oracle.moe_forward_ref(layer.fmt, x.float().cpu().numpy(), ids.cpu().numpy(),
+                                           gates.cpu().numpy(), *ref, layer.E, layer.H, layer.I, nf4_decode=mode)
+            assert_close(got, y_ref, f"graph replay {rep} vs oracle", min_rms=LAYER_MIN_RMS)
     del g
     return path
 
 
 @pytest.mark.parametrize("flags,path", [(0, e4b.E4B_PATH_GEMV), (e4b.FLAG_FORCE_TCGEN05, e4b.E4B_PATH_TCGEN05)])
 def test_nf4_layer_in_a_graph(flags, path):
-    layer, _ = small_layer("nf4", 8, 256, 512, seed=31)
-    assert _graph_vs_eager(layer, 16, 2, flags, seed=32) == path
+    layer, ref = small_layer("nf4", 8, 256, 512, seed=31)
+    assert _graph_vs_eager(layer, 16, 2, flags, seed=32, ref=ref) == path
 
 
 def test_int4_layer_in_a_graph():

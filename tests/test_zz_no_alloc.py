@@ -18,7 +18,7 @@ import torch
 
 from bit_grouped_moe_e4b_b200 import e4b, synth
 from bit_grouped_moe_e4b_b200.configs import DECODE, TINY
-from gpu_util import assert_close
+from gpu_util import assert_close, small_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -85,3 +85,42 @@ def test_noalloc_decode_layer_and_size_limit():
     with pytest.raises(e4b.E4BError) as exc:
         e4b.e4b_moe_forward_noalloc(layer, x, ids, gates, y)
     assert exc.value.status == 8
+
+
+@pytest.mark.parametrize("flags", [0, e4b.FLAG_FORCE_TCGEN05])
+def test_noalloc_mxfp4_layer_twice(flags):
+    layer, _ = small_layer("mxfp4", 8, 256, 512, seed=81)
+    rng = np.random.default_rng(82)
+    for T in (64, 7):
+        x = torch.from_numpy(rng.standard_normal((T, 256)).astype(np.float32)).to(torch.bfloat16).cuda()
+        ids_h, gates_h = synth.random_ids(rng, T, 2, 8)
+        ids = torch.from_numpy(ids_h).cuda()
+        gates = torch.from_numpy(gates_h).cuda()
+        ref = e4b.moe_forward(layer, x, ids, gates, flags=flags).float().cpu().numpy()
+        for _ in range(2):
+            y = torch.full((T, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
+            e4b.e4b_moe_forward_noalloc(layer, x, ids, gates, y, flags=flags)
+            torch.cuda.synchronize()
+            assert_close(y.float().cpu().numpy(), ref, f"noalloc mxfp4 T={T} flags={flags}", min_rms=0.5)
+
+
+def test_noalloc_int4_layer_beyond_the_nf4_token_limit():
+    # int4-b32 stacks need only the status words and h [top_k, I] whatever T,
+    # so T = 256 (more than the 227 tokens an NF4 layer of this shape fits in
+    # the static scratch) is accepted
+    wl = DECODE
+    gc, gs = e4b.quantize_int4_b32(synth.layer_weights(wl, "gate_up", "cuda"))
+    dc, ds = e4b.quantize_int4_b32(synth.layer_weights(wl, "down", "cuda"))
+    layer = e4b.PackedLayer("int4b32", wl.E, wl.H, wl.I, gc, gs, dc, ds)
+    T = 256
+    x = synth.tokens_bf16(wl, T).cuda()
+    ids_h, gates_h = synth.routing(wl, T)
+    ids = torch.from_numpy(ids_h).cuda()
+    gates = torch.from_numpy(gates_h).cuda()
+    ref = e4b.moe_forward(layer, x, ids, gates).float().cpu().numpy()
+    for _ in range(2):
+        y = torch.full((T, wl.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        e4b.e4b_moe_forward_noalloc(layer, x, ids, gates, y)
+        torch.cuda.synchronize()
+        assert e4b.e4b_last_path() == e4b.E4B_PATH_INT4_GEMV
+        assert_close(y.float().cpu().numpy(), ref, f"noalloc int4 T={T}", min_rms=0.5)
