@@ -1,15 +1,19 @@
 #!/usr/bin/env python
 """Benchmark of the packed-4-bit MoE layer forward on B200.
 
-Default workload: the small-M decode layer, NF4, E=8 experts, H=4096,
-I=14336, top-2, T=16 tokens (weights N(0, 0.02) fp32 drawn on the GPU and
-packed by the library's quantiser; x N(0, 1) in bf16; N(0, 1) router logits,
-top-2 and a softmax over the chosen two). One step = one layer forward:
-routing pass, gate_up grouped GEMM with SwiGLU, down grouped GEMM with the
-weighted combine, bf16 output.
+Default line: the prefill layer, NF4, E=8 experts, H=4096, I=14336, top-2,
+T=4096 tokens (the largest single-GPU workload; weights N(0, 0.02) fp32 drawn
+on the GPU and packed by the library's quantiser; x N(0, 1) in bf16; U[0, 1)
+router logits, top-2 and a softmax over the chosen two). One step = one layer
+forward: routing pass, gate_up grouped GEMM with SwiGLU, down grouped GEMM
+with the weighted combine, bf16 output. The same line carries `per_config`:
+every workload and token count, each timed as the median of 50 single-call
+repetitions with the L2 flushed before each, launched on a stream and
+replayed from a CUDA graph, with the spread between two independent medians
+of the same call (self-pair).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl e4b|reference]
-                    [--workload NAME] [--T T] [--sweep]
+                    [--workload NAME] [--T T] [--sweep] [--no-per-config]
 
 Prints one JSON line (rank 0). Under torchrun (N > 1) every rank runs its own
 batch of T tokens on its own GPU with replicated weights and no collective on
@@ -35,8 +39,9 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s and packed-weight HBM GB/s (% roofline) on 1 B200"
-DEFAULT_WORKLOAD = "decode_nf4_E8_H4096_I14336_top2"
-DEFAULT_T = 16
+DEFAULT_WORKLOAD = "prefill_nf4_E8_H4096_I14336_top2"
+DEFAULT_T = 4096
+PER_CONFIG_REPS = 50
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -51,6 +56,10 @@ def _args():
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per workload and token count (no cpu baseline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload table of the default line")
+    ap.add_argument("--reps", type=int, default=PER_CONFIG_REPS,
+                    help="repetitions per median in the per-workload table")
     ap.add_argument("--op", choices=["forward", "dgrad", "int4"], default="forward",
                     help="dgrad: time e4b_grouped_dgrad, the input gradients of both projections "
                          "(one JSON line, TFLOP/s); int4: the int4-b32 decode GEMVs of one token "
@@ -208,12 +217,13 @@ def kernel_bytes(wl, T, ids):
             "layer": active * 3 * wl.H * wl.I * bpw + 4 * T * wl.H + 8 * R}
 
 
-def run_gpu(wl, T, steps, warmup, rank, world, dist):
+def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
     import torch
     from bit_grouped_moe_e4b_b200 import e4b, synth
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    layer = build_layer(wl, dev)
+    if layer is None:
+        layer = build_layer(wl, dev)
     x_h = synth.tokens_bf16(wl, T)
     ids_h, gates_h = synth.routing(wl, T)
     x = x_h.to(dev)
@@ -316,31 +326,177 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist):
     }
 
 
-# ------------------------------------------------------------ CPU oracle
-def oracle_sample(wl, T, ids, gates, x_h, slots):
-    """Times the CPU oracle on routed slots of the same workload: per slot,
-    the expert's decode + fp64 matmuls + bf16(h) (oracle.fast.expert_term).
-    The experts are packed by the oracle before timing. Returns seconds."""
+# ------------------------------------------------------- per-config table
+def _bound_label(t_bytes, t_flops):
+    r = t_bytes / t_flops
+    return "ridge" if 0.5 <= r <= 2.0 else ("hbm" if r > 1 else "tensor")
+
+
+def _median_ms(fn, flush, reps, stream):
+    """Median over `reps` single calls of fn, each timed alone with CUDA events
+    on `stream`, with the L2 flushed (a write of 4x its size) before each."""
+    import torch
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def per_config_entry(wl, T, layer, reps, flush, hbm, bf16, peak_src, flags=0, variant=""):
+    """One workload and token count: the layer call (stream-launched and
+    replayed from a CUDA graph), each the median of `reps` calls with the L2
+    flushed before each; a second independent stream median for the
+    self-pair spread; per-kernel medians from the library's timing events
+    (a separate loop: events between launches stop their overlap)."""
+    import torch
+    from bit_grouped_moe_e4b_b200 import e4b, synth
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    x = synth.tokens_bf16(wl, T).to(dev)
+    ids_h, gates_h = synth.routing(wl, T)
+    ids = torch.from_numpy(ids_h).to(dev)
+    gates = torch.from_numpy(gates_h).to(dev)
+    ws = e4b.workspace(layer, T, wl.top_k, dev)
+    y = torch.empty((T, wl.H), dtype=torch.bfloat16, device=dev)
+
+    def call():
+        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws, flags)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    if e4b.e4b_read_device_status(ws) != 0:
+        raise RuntimeError(f"device status set: {wl.name} T={T}")
+    path = e4b.e4b_last_path()
+    launches = e4b.e4b_last_launch_count()
+    ms_a = _median_ms(call, flush, reps, stream)
+    ms_b = _median_ms(call, flush, reps, stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    g.replay()
+    torch.cuda.synchronize()
+    ms_g = _median_ms(g.replay, flush, reps, stream)
+    del g
+    # per-kernel medians
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+    for row in evs:
+        flush.zero_()
+        e4b.e4b_set_timing_events(row)
+        call()
+    e4b.e4b_set_timing_events(None)
+    torch.cuda.synchronize()
+    if e4b.e4b_read_device_status(ws) != 0:
+        raise RuntimeError(f"device status set in the timed loops: {wl.name} T={T}")
+    if path == e4b.E4B_PATH_GEMV:
+        spans = (("route", 0, 1), ("smallm_layer", 1, 3))
+    else:
+        spans = (("route+stage" if launches == 5 else "route", 0, 1), ("gate_up", 1, 2), ("down", 2, 3),
+                 ("finalize", 3, 4))
+    phases = {n: float(np.median([r[a].elapsed_time(r[b]) for r in evs])) for n, a, b in spans}
+    kb = kernel_bytes(wl, T, ids_h)
+    R = ids_h.size
+    flops = 2.0 * R * 3 * wl.H * wl.I
+    kflops = {"gate_up": 2.0 * R * 2 * wl.I * wl.H, "down": 2.0 * R * wl.H * wl.I, "smallm_layer": flops}
+    ms = ms_a
+    t_bytes = kb["layer"] / (hbm * 1e9)
+    t_flops = flops / (bf16 * 1e12)
+    dom = max((n for n in phases if n in kflops), key=lambda n: phases[n])
+    k_bytes = kb[dom] / (hbm * 1e9)
+    k_flops = kflops[dom] / (bf16 * 1e12)
+    entry = {
+        "workload": wl.name, "T": T, "format": wl.fmt, "path": ["none", "gemv", "tcgen05"][path] + variant,
+        "active_experts": kb["active_experts"], "reps": reps,
+        "ms": ms, "ms_graph": ms_g, "self_pair_ms": [ms_a, ms_b],
+        "self_pair_spread": abs(ms_a - ms_b) / min(ms_a, ms_b),
+        "tokens_s": T / (ms * 1e-3), "tokens_s_graph": T / (ms_g * 1e-3),
+        "tflops": flops / (ms * 1e-3) / 1e12, "packed_gbs": kb["packed_bytes"] / (ms * 1e-3) / 1e9,
+        "bound": _bound_label(t_bytes, t_flops),
+        "roofline_frac": max(t_bytes, t_flops) / (ms * 1e-3),
+        "roofline_frac_graph": max(t_bytes, t_flops) / (ms_g * 1e-3),
+        "dominant_kernel": dom, "dominant_ms": phases[dom],
+        "dominant_bound": _bound_label(k_bytes, k_flops),
+        "dominant_frac": max(k_bytes, k_flops) / (phases[dom] * 1e-3),
+        "phases_ms": phases, "launches_per_call": launches,
+    }
+    return entry
+
+
+def per_config_table(args, hbm, bf16, peak_src, layers, dev):
+    """Every workload and token count of the build's configs, one entry each."""
+    import torch
+    from bit_grouped_moe_e4b_b200.configs import WORKLOADS
+
+    flush = torch.empty(4 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    out = []
+    for wl in WORKLOADS.values():
+        layer = layers.get(wl.layer)
+        if layer is None:
+            layers.clear()
+            torch.cuda.empty_cache()
+            layer = layers[wl.layer] = build_layer(wl, dev)
+        for T in wl.T:
+            out.append(per_config_entry(wl, T, layer, args.reps, flush, hbm, bf16, peak_src))
+    del flush
+    torch.cuda.empty_cache()
+    return {"peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": peak_src + " (burst)"},
+            "timing": f"median of {args.reps} single calls, L2 flushed before each (a {4 * L2_BYTES >> 20} MiB "
+                      "write); stream-launched and CUDA-graph replayed; self-pair = two independent stream "
+                      "medians; roofline_frac = max(algorithmic bytes / HBM, FLOP / bf16 peak) / time",
+            "rows": out}
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_tokens_sample(wl, T, ids, gates, x_h, tokens, packed=None):
+    """Times the CPU oracle's layer (oracle.fast.moe_forward_sampled: per
+    expert decode, fp64 matmuls, bf16 h, fp64 weighted sum) on `tokens` of the
+    batch, with one thread per expert those tokens use, up to the host's cores.
+    The experts are packed by the oracle before timing (pass `packed` to reuse
+    them). Returns (seconds, threads, packed)."""
     import torch
     from oracle import fast
     from bit_grouped_moe_e4b_b200 import synth
 
     fast.build()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    need = sorted({int(ids.reshape(-1)[s]) for s in slots})
-    packed = {}
+    need = sorted({int(ids[t, j]) for t in tokens for j in range(wl.top_k)})
+    packed = dict(packed or {})
     for e in need:
         for which in ("gate_up", "down"):
-            packed[(which, e)] = fast.quantize(wl.fmt, synth.expert_weight(wl, which, e, dev).cpu().numpy())
-    x = x_h.float().numpy().astype(np.float64)
+            if (which, e) not in packed:
+                packed[(which, e)] = fast.quantize(wl.fmt, synth.expert_weight(wl, which, e, dev).cpu().numpy())
+    threads = min(len(need), host_cores())
+    xf = x_h.float().numpy()
     t = time.perf_counter()
-    for s in slots:
-        e = int(ids.reshape(-1)[s])
-        fast.expert_term(wl.fmt, x[s // wl.top_k][None], packed[("gate_up", e)], packed[("down", e)],
-                         wl.H, wl.I)
-    return time.perf_counter() - t
+    fast.moe_forward_sampled(wl.fmt, xf, ids, gates, None, wl.E, wl.H, wl.I, list(tokens),
+                             packed_fn=lambda which, e: packed[(which, e)], workers=threads)
+    return time.perf_counter() - t, threads, packed
 
 
+# ------------------------------------------------------------ CPU oracle
 def run_dgrad(wl, T, steps, warmup, bf16, bf16_sus, peak_src):
     """Times the input gradients through the packed weights of both
     projections of the workload's layer on its routed rows (expert order):
@@ -571,17 +727,36 @@ def run_int4(wl, steps, warmup, hbm, peak_src, cpu_baseline=True):
 
 
 def run_reference(args, wl, T):
+    """The oracle as it stands, on the host cores: each step runs the layer on
+    a sample of the batch's tokens (oracle_tokens_sample), the experts packed
+    once before timing."""
     from bit_grouped_moe_e4b_b200 import synth
 
     x_h = synth.tokens_bf16(wl, T)
     ids, gates = synth.routing(wl, T)
-    R = ids.size
-    # one routed slot per step (a bounded sample: one expert term of one token)
-    if args.warmup:
-        oracle_sample(wl, T, ids, gates, x_h, [i % R for i in range(min(args.warmup, 2))])
-    slots = [(args.warmup + i) % R for i in range(args.steps)]
-    secs = oracle_sample(wl, T, ids, gates, x_h, slots)
-    tokens = len(slots) / wl.top_k
+    n = REF_TOKENS_PER_STEP.get(wl.name, 4)
+    sample = lambda i: [(i * n + j) % T for j in range(n)]
+    packed = None
+    for i in range(args.warmup):
+        _, threads, packed = oracle_tokens_sample(wl, T, ids, gates, x_h, sample(i), packed)
+    # pack every expert before the timed steps
+    all_tokens = sorted({t for i in range(args.warmup, args.warmup + args.steps) for t in sample(i)})
+    need = sorted({int(ids[t, j]) for t in all_tokens for j in range(wl.top_k)})
+    from oracle import fast
+    import torch
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    packed = dict(packed or {})
+    for e in need:
+        for which in ("gate_up", "down"):
+            if (which, e) not in packed:
+                packed[(which, e)] = fast.quantize(wl.fmt, synth.expert_weight(wl, which, e, dev).cpu().numpy())
+    secs, thr = 0.0, 1
+    for i in range(args.warmup, args.warmup + args.steps):
+        dt, t_used, packed = oracle_tokens_sample(wl, T, ids, gates, x_h, sample(i), packed)
+        secs += dt
+        thr = max(thr, t_used)
+    tokens = n * args.steps
     value = tokens / secs
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -590,13 +765,23 @@ def run_reference(args, wl, T):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": T, "format": wl.fmt, "E": wl.E, "H": wl.H, "I": wl.I,
                    "top_k": wl.top_k},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{args.steps} routed slots (one expert term of one token each: "
-                                   "decode gate_up and down, fp64 matmuls, bf16 h), weights packed "
-                                   "before timing"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "host_cores": host_cores(), "cpu": cpu_model(),
+                         "sample": f"{n} tokens of the batch a step (every routed slot of each: decode of the "
+                                   "experts they use, fp64 matmuls, bf16 h, fp64 weighted sum), one thread per "
+                                   "expert (C core, no BLAS), weights packed before timing"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# tokens per reference step: a bounded sample (each step decodes every expert
+# its tokens use, seconds of host work at the large shapes)
+REF_TOKENS_PER_STEP = {"tiny_nf4_E8_H256_I512_top2": 64, "prefill_nf4_E8_H4096_I14336_top2": 4,
+                       "decode_nf4_E8_H4096_I14336_top2": 4, "skewed_nf4_E128_H2048_I768_top8": 8,
+                       "mxfp4_E32_H2880_I2880_top4": 8}
+# tokens in the cpu_baseline sample of the default line
+CPU_BASELINE_TOKENS = 32
 
 
 def main():
@@ -643,8 +828,14 @@ def main():
     cases = [(wl, T)]
     if args.sweep:
         cases = [(w, t) for w in WORKLOADS.values() for t in w.T]
+    layers = {}
+    dev = torch.device("cuda", local)
     for wl_i, T_i in cases:
-        r = run_gpu(wl_i, T_i, args.steps, args.warmup, rank, world, dist)
+        if wl_i.layer not in layers:
+            layers.clear()
+            torch.cuda.empty_cache()
+            layers[wl_i.layer] = build_layer(wl_i, dev)
+        r = run_gpu(wl_i, T_i, args.steps, args.warmup, rank, world, dist, layer=layers[wl_i.layer])
         kb = kernel_bytes(wl_i, T_i, r["ids"])
         dominant = max((k for k in r["phases"] if not k.startswith("route") and not k.startswith("_")),
                        key=lambda k: r["phases"][k])
@@ -676,13 +867,17 @@ def main():
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches"],
         }
+        if not args.sweep and not args.no_per_config and world == 1:
+            line["per_config"] = per_config_table(args, hbm, bf16, peak_src, layers, dev)
         if (not args.sweep and rank == 0 and world == 1 and not args.no_cpu_baseline):
-            slots = list(range(wl_i.top_k))  # one token: both of its slots
-            secs = oracle_sample(wl_i, T_i, r["ids"], r["gates"], r["x"], slots)
+            ntok = min(CPU_BASELINE_TOKENS, T_i)
+            secs, threads, _ = oracle_tokens_sample(wl_i, T_i, r["ids"], r["gates"], r["x"], list(range(ntok)))
             line["cpu_baseline"] = {
-                "value": 1.0 / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                "sample": f"token 0 of the batch ({wl_i.top_k} routed slots: decode gate_up and "
-                          "down of each expert, fp64 matmuls, bf16 h); single-threaded C core"}
+                "value": ntok / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "host_cores": host_cores(), "cpu": cpu_model(), "seconds": secs,
+                "sample": f"tokens 0..{ntok - 1} of the batch (all their routed slots: decode of the experts "
+                          "they use, fp64 matmuls, bf16 h, fp64 weighted sum); one thread per expert, "
+                          "C core without BLAS; weights packed before timing"}
         if rank == 0:
             print(json.dumps(line), flush=True)
         del r
