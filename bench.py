@@ -386,6 +386,10 @@ def per_config_entry(wl, T, layer, reps, flush, hbm, bf16, peak_src, flags=0, va
     del g
     # per-kernel medians
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+    for row in evs:  # torch creates the CUDA event on its first record
+        for e_ in row:
+            e_.record(stream)
+    torch.cuda.synchronize()
     for row in evs:
         flush.zero_()
         e4b.e4b_set_timing_events(row)

@@ -26,6 +26,9 @@ Sources (page titles; sections):
     pack calibrated (GPTQ) weights for it?" (grouped-nf4-gemm solutions page):
     the int4-b32 decode GEMV with exact integer accumulation and the GPTQ
     packer (module ``int4b32``).
+  * OCP Microscaling v1.0 MXFP8 (E4M3 elements, e8m0 scale per 32): the
+    activations of the layer on the block-scaled FP4 MMA (module ``mxfp8``,
+    ``moe_forward_ref(..., act_quant="mxfp8")``).
   * "experts4bit-qlora" README: fused ``gate_up_proj [E, 2I, H]`` and
     ``down_proj [E, H, I]`` expert stacks (transformers v5 layout).
 
@@ -53,6 +56,7 @@ from .formats import (
 from .moe import (route_ref, moe_forward_ref, swiglu_ref, expert_tokens, clamped_glu_ref,
                   split_gate_up, activation_ref, grouped_projection_ref, grouped_dgrad_ref)
 from . import int4b32
+from . import mxfp8
 
 __all__ = [
     "NF4_BLOCK", "MXFP4_BLOCK", "E2M1_MAGNITUDES",
@@ -61,5 +65,5 @@ __all__ = [
     "dequant_ref_exact", "dequant_ref_level", "quantize_pack_mxfp4", "unpack_mxfp4_codes",
     "dequant_mxfp4", "packed_bytes_per_weight",
     "route_ref", "moe_forward_ref", "swiglu_ref", "expert_tokens", "clamped_glu_ref", "split_gate_up",
-    "activation_ref", "grouped_projection_ref", "grouped_dgrad_ref", "int4b32",
+    "activation_ref", "grouped_projection_ref", "grouped_dgrad_ref", "int4b32", "mxfp8",
 ]

@@ -58,6 +58,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from .mxfp8 import mxfp8_round_trip
 from .formats import (
     bf16_round,
     dequant_ref,
@@ -152,7 +153,7 @@ def expert_tokens(ids, tokens=None):
 def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales,
                     E, H, I, tokens=None, exact_decode=False, return_h=False,
                     layout="halves", act="swiglu", alpha=1.702, limit=7.0,
-                    gu_bias=None, dn_bias=None, nf4_decode="product"):
+                    gu_bias=None, dn_bias=None, nf4_decode="product", act_quant=None):
     """The MoE layer forward (per-expert dequantise-then-matmul loop).
 
     x: bf16 values as any float array [T, H]; ids int [T, k]; gates fp32
@@ -173,6 +174,11 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
     absmax)), dequant_ref), "level" (bf16_rne(level) * absmax exactly,
     dequant_ref_level) or "exact" (level * absmax, fidelity only; also
     selected by exact_decode=True).
+
+    act_quant: None (bf16 activations), or "mxfp8": the x rows and the bf16
+    intermediate h are replaced by their MXFP8 decode (oracle.mxfp8: E4M3
+    elements, one e8m0 scale per 32 along K) before the matmul that reads
+    them -- the activations a block-scaled FP4 tensor-core MMA multiplies.
     """
     x = np.asarray(x, dtype=np.float64)
     ids = np.asarray(ids)
@@ -189,12 +195,16 @@ def moe_forward_ref(fmt, x, ids, gates, gu_codes, gu_scales, dn_codes, dn_scales
         Wgu = _decode(fmt, gu_codes[e], gu_scales[e], 2 * I, H, mode)
         Wd = _decode(fmt, dn_codes[e], dn_scales[e], H, I, mode)
         X = x[[t for _, t in pairs]]
+        if act_quant == "mxfp8":
+            X = mxfp8_round_trip(X)
+        elif act_quant is not None:
+            raise ValueError(act_quant)
         GU = X @ Wgu.T
         if gu_bias is not None:
             GU = GU + np.asarray(gu_bias[e], np.float64)
         G, U = split_gate_up(GU, layout)
         h = bf16_round(activation_ref(G, U, act, alpha, limit))
-        O = h @ Wd.T
+        O = (mxfp8_round_trip(h) if act_quant == "mxfp8" else h) @ Wd.T
         if dn_bias is not None:
             O = O + np.asarray(dn_bias[e], np.float64)
         for r, (s, _) in enumerate(pairs):

@@ -104,7 +104,10 @@ def test_workload_sampled_tokens(name, T):
                                                      nf4_decode=other_mode)
     for y, ref, what in ((y_auto, y_ref, "auto"), (y_other, y_ref_other, "other path")):
         got = y.float().cpu().numpy()[tokens]
-        assert_close(got, ref, f"{name} T={T} {what}", min_rms=0.1)
+        # the workloads' N(0, 0.02) weights give output rms from ~0.02 (the
+        # tiny layer) to ~2; the tolerance is relative to that scale, and the
+        # guard only rules out a degenerate (all-zero) reference
+        assert_close(got, ref, f"{name} T={T} {what}", min_rms=0.005)
     # rows not sampled: finite and equal across the two kernel paths within
     # tolerance (for NF4 the paths' readings differ by one bf16 rounding per
     # weight, far inside it on these N(0, 0.02) weights)
