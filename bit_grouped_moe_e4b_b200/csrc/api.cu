@@ -35,11 +35,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace of the layer forward. Everything up to total_min is required;
-// xs (the routed rows of x in expert order) is the large-M path's staging
-// copy, used when the workspace reaches total.
+// Workspace of the layer forward. After the routing arrays and h comes one
+// region that the small-M path uses as its fp32 accumulator acc [T, H]
+// (needs up to small_min) and the large-M path as the gate-weighted fp32 rows
+// [T*top_k, H] (needs up to large_min); xs (the routed rows of x in expert
+// order) is the large-M path's staging copy, used when the workspace reaches
+// total.
 struct MoeWs {
-  size_t status, sync, nsync, counts, offsets, perm, inv, h, acc, total_min, xs, total;
+  size_t status, sync, nsync, counts, offsets, perm, inv, h, acc, small_min, rows, large_min, xs, total;
 };
 
 MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
@@ -54,8 +57,11 @@ MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
   w.perm = o;    o = align_up(o + size_t(R) * 4, 256);
   w.inv = o;     o = align_up(o + size_t(R) * 4, 256);
   w.h = o;       o = align_up(o + size_t(R) * size_t(I) * 2, 256);
-  w.acc = o;     o = align_up(o + size_t(T) * size_t(H) * 4, 256);
-  w.total_min = o;
+  w.acc = o;
+  w.rows = o;
+  w.small_min = align_up(o + size_t(T) * size_t(H) * 4, 256);
+  w.large_min = align_up(o + size_t(R) * size_t(H) * 4, 256);
+  o = w.large_min;
   w.xs = o;      o = align_up(o + size_t(R) * size_t(H) * 2, 256);
   w.total = o;
   return w;
@@ -63,8 +69,9 @@ MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
 
 }  // namespace
 
-size_t e4b::moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
-  return moe_ws_layout(E, H, I, T, top_k).total_min;
+size_t e4b::moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k, bool small_m) {
+  const MoeWs w = moe_ws_layout(E, H, I, T, top_k);
+  return small_m ? w.small_min : w.large_min;
 }
 
 namespace {
@@ -103,6 +110,12 @@ bool choose_gemv(int64_t R, int64_t E, uint32_t flags) {
   if (E > 256) return true;
   return R <= 16 * E;
 }
+
+}  // namespace
+
+bool e4b::layer_uses_small_m(int64_t R, int64_t E, uint32_t flags) { return choose_gemv(R, E, flags); }
+
+namespace {
 
 e4b_status run_projection(const GemmProblem& p, bool gemv, cudaStream_t st) {
   const int sms = sm_count();
@@ -508,11 +521,10 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
       !aligned16(w->down_codes) || !aligned16(w->gate_up_scales) || !aligned16(w->down_scales))
     return E4B_ERR_MISALIGNED;
   const MoeWs L = moe_ws_layout(E, H, I, T, top_k);
-  if (ws_bytes < L.total_min) return E4B_ERR_WORKSPACE_TOO_SMALL;
-
   const int64_t R = T * top_k;
   const bool gemv = choose_gemv(R, E, flags);
   if (!gemv && E > 256) return E4B_ERR_UNSUPPORTED;
+  if (ws_bytes < (gemv ? L.small_min : L.large_min)) return E4B_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* base = static_cast<uint8_t*>(ws);
   int32_t* status = reinterpret_cast<int32_t*>(base + L.status);
   int32_t* counts = reinterpret_cast<int32_t*>(base + L.counts);
@@ -595,8 +607,6 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   g.offsets = offsets;
   g.out = h;
   g.ldo = I;
-  g.zero_buf = acc;
-  g.zero_count = T * H;
   g.status = status;
   g.flags = flags;
   g.layout = w->gate_up_layout;
@@ -608,8 +618,11 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   st = run_projection(g, gemv, s);
   if (st != E4B_OK) return st;
 
+  // down: every routed row's gate-weighted output into its own fp32 row, then
+  // each token's rows summed in slot order (deterministic, no atomics)
+  float* rows = reinterpret_cast<float*>(base + L.rows);
   GemmProblem d = g;
-  d.epilogue = E4B_EPI_COMBINE;
+  d.epilogue = kEpiGatedRows;
   d.N = H;
   d.K = I;
   d.codes = w->down_codes;
@@ -619,17 +632,15 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   d.row_slot = nullptr;
   d.out_slot = perm;
   d.gates = gates;
-  d.out = acc;
+  d.out = rows;
   d.ldo = H;
-  d.zero_buf = nullptr;
-  d.zero_count = 0;
   d.bias = w->down_bias;
   mark(2, s);
   st = run_projection(d, gemv, s);
   if (st != E4B_OK) return st;
 
   mark(3, s);
-  ce = launch_finalize(acc, T * H, y, s, sm_count());
+  ce = launch_combine_rows(rows, inv, T, top_k, H, y, s, sm_count());
   if (ce != cudaSuccess) return E4B_ERR_CUDA;
   mark(4, s);
   g_last_path = gemv ? E4B_PATH_GEMV : E4B_PATH_TCGEN05;

@@ -250,6 +250,40 @@ __global__ void finalize_kernel(const float* __restrict__ acc, int64_t n4, uint1
   }
 }
 
+// One thread per 4 consecutive outputs of a token: the token's k rows are
+// read in slot order and summed in fp32, so the result does not depend on the
+// order in which the rows were produced.
+__global__ void combine_rows_kernel(const float* __restrict__ rows, const int32_t* __restrict__ inv,
+                                    int64_t T, int32_t k, int64_t H4, uint16_t* __restrict__ y) {
+  const int64_t total = T * H4;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = i / H4;
+    const int64_t c = i - t * H4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const int32_t p = __ldg(inv + t * k + j);
+      if (p < 0) continue;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(rows + int64_t(p) * (H4 * 4)) + c);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    reinterpret_cast<uint2*>(y)[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  }
+}
+
+cudaError_t launch_combine_rows(const float* rows, const int32_t* inv, int64_t T, int32_t k, int64_t H,
+                                uint16_t* y, cudaStream_t st, int sms) {
+  const int64_t total = T * (H / 4);
+  int64_t grid = (total + 255) / 256;
+  if (grid > int64_t(sms) * 16) grid = int64_t(sms) * 16;
+  if (grid < 1) grid = 1;
+  combine_rows_kernel<<<int(grid), 256, 0, st>>>(rows, inv, T, k, H / 4, y);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_finalize(const float* acc, int64_t n, uint16_t* y, cudaStream_t st, int sms) {
   const int64_t n4 = n / 4;  // callers guarantee n % 4 == 0
   int64_t grid = (n4 + 255) / 256;

@@ -27,11 +27,28 @@ cudaError_t launch_gather_rows(const uint16_t* x, int64_t H, const int32_t* perm
                                cudaStream_t st, int sms);
 // Smallest workspace e4b_moe_forward accepts (without the staging copy of the
 // routed rows that e4b_moe_workspace_size includes).
-size_t moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k);
+// The path the layer takes for these sizes and flags: true = small-M.
+bool layer_uses_small_m(int64_t R, int64_t E, uint32_t flags);
+// Smallest workspace e4b_moe_forward accepts on that path: the small-M path
+// needs the routing arrays, h and an fp32 [T, H] accumulator; the large-M path
+// the routing arrays, h and the gated rows fp32 [T*top_k, H] (without the
+// staging copy of the routed rows that e4b_moe_workspace_size includes).
+size_t moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k, bool small_m);
 
 // GemmProblem::epilogue for the input gradient through the weights
 // (e4b_grouped_dgrad): out [R, K] bf16, row p = a_p . W_e, a [R, N].
 constexpr int kEpiDgrad = 3;
+// GemmProblem::epilogue of the layer's down projection on the large-M path:
+// out fp32 [R, ldo], row p = gates[s] * (a_p . W_e^T + bias), s = out_slot[p]
+// (p when null); every row is written once (no accumulation), so the
+// token-wise sum that follows (launch_combine_rows) runs in a fixed order.
+constexpr int kEpiGatedRows = 4;
+
+// y[t] = bf16(sum_j rows[inv[t*k + j]]) for j = 0..k-1 in that order, fp32
+// sums; a slot whose inv is -1 adds nothing (rows fp32 [*, H], y bf16 [T, H],
+// H % 4 == 0, both 16-byte aligned).
+cudaError_t launch_combine_rows(const float* rows, const int32_t* inv, int64_t T, int32_t k, int64_t H,
+                                uint16_t* y, cudaStream_t st, int sms);
 
 // Description of one grouped projection as the kernels see it.
 struct GemmProblem {

@@ -23,8 +23,10 @@
 //               (M = 128 weight rows, N = 256 routed rows, K = 16 per MMA).
 //   warps 12-15 epilogue: tcgen05.ld of the fp32 accumulators, then the
 //               biases and the gated activation (gate and up accumulate in two
-//               TMEM column ranges of the same lanes, so it is thread-local)
-//               or the gate-weighted combine.
+//               TMEM column ranges of the same lanes, so it is thread-local),
+//               the gate-weighted combine (atomics, e4b_grouped_gemm), or the
+//               layer's gate-weighted rows (one fp32 row per routed row,
+//               summed per token afterwards in a fixed order).
 // Interleaved gate/up rows (gate 2n, up 2n+1) reach the same tiles through a
 // 3-D view of the codes, [E*I rows, 2, K/2 bytes]: one box fetches 128 gate
 // (or up) rows at a two-row stride.
@@ -524,6 +526,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(hv);
           } else if constexpr (EPI == E4B_EPI_STORE || DG) {
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(gv);
+          } else if constexpr (EPI == kEpiGatedRows) {
+            const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
+            static_cast<float*>(p.out)[pr * p.ldo + n] = p.gates[slot] * gv;
           } else {
             const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
             const int64_t tok = slot / p.top_k;
@@ -649,6 +654,9 @@ cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms) {
     return p.fmt == E4B_FMT_NF4 ? launch_t<E4B_FMT_NF4, kEpiDgrad>(p, st, sms)
                                 : launch_t<E4B_FMT_MXFP4, kEpiDgrad>(p, st, sms);
   }
+  if (p.epilogue == kEpiGatedRows)
+    return p.fmt == E4B_FMT_NF4 ? launch_t<E4B_FMT_NF4, kEpiGatedRows>(p, st, sms)
+                                : launch_t<E4B_FMT_MXFP4, kEpiGatedRows>(p, st, sms);
   if (p.fmt == E4B_FMT_NF4) {
     if (p.epilogue == E4B_EPI_SWIGLU) return launch_t<E4B_FMT_NF4, E4B_EPI_SWIGLU>(p, st, sms);
     if (p.epilogue == E4B_EPI_COMBINE) return launch_t<E4B_FMT_NF4, E4B_EPI_COMBINE>(p, st, sms);

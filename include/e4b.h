@@ -411,11 +411,13 @@ e4b_status e4b_ep_combine(const uint16_t* ys, int64_t H, const int32_t* inv_perm
 /* ---------------------------------------------------------- whole layer */
 
 /* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots.
- * The size includes a staging copy of the routed rows of x in expert order
- * ([T*top_k, H] bf16) that the large-M path uses; a smaller workspace that
- * still holds the routing arrays, h, the accumulator and the status word is
- * accepted, and the large-M path then gathers the rows inside its kernel
- * (same results, slower). */
+ * The workspace holds the status word, the routing arrays, h, one fp32 region
+ * (the small-M path's accumulator [T, H], or the large-M path's gate-weighted
+ * rows [T*top_k, H]) and last a staging copy of the routed rows of x in expert
+ * order ([T*top_k, H] bf16) that the large-M path uses. A smaller workspace
+ * that holds everything the chosen path needs but the staging copy is
+ * accepted; the large-M path then gathers the rows inside its kernel (same
+ * results, slower). */
 e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t top_k,
                                   size_t* bytes);
 
@@ -466,11 +468,12 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
  * that loads the library keeps until the process exits. A call whose
  * required scratch exceeds 16 MiB returns E4B_ERR_EXCEEDS_STATIC_SCRATCH and
  * enqueues nothing. The required scratch is, for NF4 and MXFP4 stacks,
- * e4b_moe_workspace_size without the optional staging copy (a layer with
- * H=4096, I=14336 and top-2 routing fits up to 227 tokens; the staging copy
- * is used while it also fits), and for int4-b32 stacks
- * e4b_moe_workspace_size itself, which does not grow with T. Nothing is
- * allocated or freed.
+ * the part of e4b_moe_workspace_size the chosen path needs (without the
+ * optional staging copy; a layer with E=8, H=4096, I=14336 and top-2 routing
+ * fits up to 186 tokens on the large-M path it takes from 65 tokens on, and up
+ * to 227 with E4B_FLAG_FORCE_GEMV; the staging copy is used while it also
+ * fits), and for int4-b32 stacks e4b_moe_workspace_size itself, which does
+ * not grow with T. Nothing is allocated or freed.
  *   - The first call on each device looks up that device's copy of the
  *     array (set-up, once per device); make that first call before any stream
  *     capture begins. The address found belongs to the device's context as it
