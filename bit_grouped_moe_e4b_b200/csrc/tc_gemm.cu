@@ -77,7 +77,10 @@ struct Cfg {
   static constexpr uint32_t kScal = kBars + kNumBars * 8;       // 16 B
   static constexpr uint32_t kAct = kScal + 16;                  // kMaxE x 4
   static constexpr uint32_t kPre = kAct + kMaxE * 4;            // (kMaxE + 1) x 4
-  static constexpr uint32_t kEnd = kPre + (kMaxE + 1) * 4;
+  // per epilogue warp: the gate weight and token of each of a tile's BN rows
+  static constexpr uint32_t kGate = (kPre + (kMaxE + 1) * 4 + 15) / 16 * 16;
+  static constexpr uint32_t kTok = kGate + 4 * BN * 4;
+  static constexpr uint32_t kEnd = kTok + 4 * BN * 4;
   static constexpr uint32_t kSmemBytes = kEnd + 1024;           // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -488,14 +491,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may read
     const int rloc = q * 32 + lane;
+    constexpr bool GATED = EPI == E4B_EPI_COMBINE || EPI == kEpiGatedRows;
+    float* s_g = reinterpret_cast<float*>(smem + C::kGate) + q * BN;
+    int32_t* s_t = reinterpret_cast<int32_t*>(smem + C::kTok) + q * BN;
     for (int j = 0; j < my_tiles; ++j) {
       const int ab = j % NACC;
+      const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
+      if constexpr (GATED) {
+        // Every row's gate weight and token, staged by this warp for itself
+        // while the tile's MMAs run: the loop below reads them from shared
+        // memory instead of two dependent global loads per row.
+        __syncwarp();
+        int32_t sl[BN / 32];
+#pragma unroll
+        for (int u = 0; u < BN / 32; ++u) {
+          const int64_t pr = T.p0 + lane + 32 * u;
+          sl[u] = pr < T.p1 ? (p.out_slot ? p.out_slot[pr] : int32_t(pr)) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < BN / 32; ++u) {
+          s_g[lane + 32 * u] = sl[u] >= 0 ? p.gates[sl[u]] : 0.f;
+          s_t[lane + 32 * u] = sl[u] >= 0 ? sl[u] / p.top_k : 0;
+        }
+        __syncwarp();
+      }
       if (!mbar_wait_bounded(&acc_full[ab], uint32_t(j / NACC) & 1u, limit, s_abort)) {
         give_up();
         break;
       }
       tc_fence_after();
-      const Tile T = sc.tile(int(blockIdx.x) + j * int(gridDim.x));
       const int64_t n = T.mt * BM + rloc;
       const bool nvalid = n < Mdim;
       // bias of this thread's row(s): gate and up, or the single output row
@@ -527,12 +551,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           } else if constexpr (EPI == E4B_EPI_STORE || DG) {
             static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(gv);
           } else if constexpr (EPI == kEpiGatedRows) {
-            const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
-            static_cast<float*>(p.out)[pr * p.ldo + n] = p.gates[slot] * gv;
+            static_cast<float*>(p.out)[pr * p.ldo + n] = s_g[cc * 16 + t] * gv;
           } else {
-            const int32_t slot = p.out_slot ? p.out_slot[pr] : int32_t(pr);
-            const int64_t tok = slot / p.top_k;
-            atomicAdd(static_cast<float*>(p.out) + tok * p.ldo + n, p.gates[slot] * gv);
+            const int64_t tok = s_t[cc * 16 + t];
+            atomicAdd(static_cast<float*>(p.out) + tok * p.ldo + n, s_g[cc * 16 + t] * gv);
           }
         }
       }
