@@ -67,11 +67,43 @@ MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
   return w;
 }
 
+// Workspace regions of the block-scaled MXFP4 path, after the routing
+// arrays, h and the gate-weighted rows (the staging copy's place): the two
+// e4m3 terms of x and of h in padded per-expert rows, their scale chunks, and
+// bf16 h in padded rows.
+struct MxWs {
+  int64_t Rp_max, Hp, Ip;
+  size_t xq, sfx, hp, hq, sfh, total;
+};
+
+MxWs mx_ws_layout(const MoeWs& L, int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
+  MxWs m;
+  m.Rp_max = mx_padded_rows_max(T * top_k, E);
+  m.Hp = (H + 127) / 128 * 128;
+  m.Ip = (I + 127) / 128 * 128;
+  const size_t rp = size_t(m.Rp_max);
+  size_t o = L.large_min;
+  m.xq = o;  o = align_up(o + 2 * rp * size_t(m.Hp), 256);
+  m.sfx = o; o = align_up(o + 2 * (rp / 128) * size_t(m.Hp / 128) * 512, 256);
+  m.hp = o;  o = align_up(o + rp * size_t(I) * 2, 256);
+  m.hq = o;  o = align_up(o + 2 * rp * size_t(m.Ip), 256);
+  m.sfh = o; o = align_up(o + 2 * (rp / 128) * size_t(m.Ip / 128) * 512, 256);
+  m.total = o;
+  return m;
+}
+
+bool has_mx(const e4b_moe_weights* w) {
+  return w->fmt == E4B_FMT_MXFP4 && w->gate_up_mx_codes && w->gate_up_mx_sf && w->down_mx_codes &&
+         w->down_mx_sf;
+}
+
 }  // namespace
 
-size_t e4b::moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k, bool small_m) {
-  const MoeWs w = moe_ws_layout(E, H, I, T, top_k);
-  return small_m ? w.small_min : w.large_min;
+size_t e4b::moe_workspace_min_bytes(const e4b_moe_weights* w, int64_t T, int64_t top_k, uint32_t flags) {
+  const MoeWs L = moe_ws_layout(w->E, w->H, w->I, T, top_k);
+  if (layer_uses_small_m(T * top_k, w->E, flags)) return L.small_min;
+  if (has_mx(w) && !(flags & E4B_FLAG_MX_DECODE)) return mx_ws_layout(L, w->E, w->H, w->I, T, top_k).total;
+  return L.large_min;
 }
 
 namespace {
@@ -420,8 +452,16 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
                                   size_t* bytes) {
   if (!w || !bytes || T < 0 || top_k <= 0 || w->E <= 0 || w->H <= 0 || w->I <= 0)
     return E4B_ERR_INVALID_ARG;
-  *bytes = w->fmt == E4B_FMT_INT4B32 ? int4_layer_ws_bytes(w->I, top_k)
-                                     : moe_ws_layout(w->E, w->H, w->I, T, top_k).total;
+  if (w->fmt == E4B_FMT_INT4B32) {
+    *bytes = int4_layer_ws_bytes(w->I, top_k);
+    return E4B_OK;
+  }
+  const MoeWs L = moe_ws_layout(w->E, w->H, w->I, T, top_k);
+  *bytes = L.total;
+  if (has_mx(w)) {
+    const size_t mx = mx_ws_layout(L, w->E, w->H, w->I, T, top_k).total;
+    if (mx > *bytes) *bytes = mx;
+  }
   return E4B_OK;
 }
 
@@ -496,6 +536,150 @@ static e4b_status moe_forward_int4(const e4b_moe_weights* w, const uint16_t* x, 
   return E4B_OK;
 }
 
+// The large-M layer on the block-scaled FP4 MMA (csrc/mx_native.cu): x split
+// into e4m3 terms in padded per-expert rows, gate_up with the gated
+// activation into bf16 h (padded rows), h split the same way, down with the
+// gate-weighted rows, then each token's rows summed in slot order.
+static e4b_status moe_forward_mx(const e4b_moe_weights* w, const MoeWs& L, const uint16_t* x, int64_t T,
+                                 int32_t top_k, const int32_t* perm, const int64_t* offsets, const int32_t* inv,
+                                 const float* gates, uint16_t* y, uint8_t* base, size_t ws_bytes,
+                                 int32_t* status, uint32_t flags, cudaStream_t s) {
+  const int64_t E = w->E, H = w->H, I = w->I;
+  const MxWs M = mx_ws_layout(L, E, H, I, T, top_k);
+  if (ws_bytes < M.total) return E4B_ERR_WORKSPACE_TOO_SMALL;
+  if (M.Rp_max >= (int64_t(1) << 31)) return E4B_ERR_UNSUPPORTED;
+  const int nt = (flags & E4B_FLAG_MX_ACT_E4M3) ? 1 : 2;
+  const int sms = sm_count();
+  uint8_t* xq = base + M.xq;
+  uint8_t* sfx = base + M.sfx;
+  uint16_t* hp = reinterpret_cast<uint16_t*>(base + M.hp);
+  uint8_t* hq = base + M.hq;
+  uint8_t* sfh = base + M.sfh;
+  float* rows = reinterpret_cast<float*>(base + L.rows);
+
+  MxActArgs qa{};
+  qa.src = x;
+  qa.ld_src = H;
+  qa.perm = perm;
+  qa.top_k = top_k;
+  qa.offsets = offsets;
+  qa.E = int32_t(E);
+  qa.K = H;
+  qa.rows = M.Rp_max;
+  qa.elems = xq;
+  qa.sf = sfx;
+  qa.nterms = nt;
+  if (launch_mx_act_quant(qa, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+
+  MxGemmArgs g{};
+  g.gated_rows = false;
+  g.nterms = nt;
+  g.E = int(E);
+  g.top_k = top_k;
+  g.Nm = I;
+  g.K = H;
+  g.Rp_max = M.Rp_max;
+  g.codes = w->gate_up_mx_codes;
+  g.sfa = w->gate_up_mx_sf;
+  g.act = xq;
+  g.sfb = sfx;
+  g.offsets = offsets;
+  g.perm = perm;
+  g.gates = gates;
+  g.out = hp;
+  g.ldo = I;
+  g.layout = w->gate_up_layout;
+  g.act_fn = w->activation;
+  g.alpha = w->glu_alpha;
+  g.limit = w->glu_limit;
+  g.bias = w->gate_up_bias;
+  g.status = status;
+  g.flags = flags;
+  mark(1, s);
+  if (launch_mx_gemm(g, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+
+  mark(2, s);
+  MxActArgs qh = qa;
+  qh.src = hp;
+  qh.ld_src = I;
+  qh.perm = nullptr;
+  qh.K = I;
+  qh.elems = hq;
+  qh.sf = sfh;
+  if (launch_mx_act_quant(qh, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+
+  MxGemmArgs d = g;
+  d.gated_rows = true;
+  d.Nm = H;
+  d.K = I;
+  d.codes = w->down_mx_codes;
+  d.sfa = w->down_mx_sf;
+  d.act = hq;
+  d.sfb = sfh;
+  d.out = rows;
+  d.ldo = H;
+  d.bias = w->down_bias;
+  if (launch_mx_gemm(d, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+
+  mark(3, s);
+  if (launch_combine_rows(rows, inv, T, top_k, H, y, s, sms) != cudaSuccess) return E4B_ERR_CUDA;
+  mark(4, s);
+  g_last_path = E4B_PATH_TCGEN05_MX;
+  g_last_launches = 6;
+  return E4B_OK;
+}
+
+e4b_status e4b_mxfp4_native_size(int32_t E, int64_t rows_per_mat, int64_t K, int32_t nmat,
+                                 size_t* codes_bytes, size_t* sf_bytes) {
+  if (!codes_bytes || !sf_bytes || E <= 0 || rows_per_mat <= 0 || K <= 0 || (nmat != 1 && nmat != 2))
+    return E4B_ERR_INVALID_ARG;
+  if (K % E4B_MXFP4_BLOCK) return E4B_ERR_UNSUPPORTED;
+  const size_t Np = size_t((rows_per_mat + 127) / 128 * 128);
+  const size_t Kp = size_t((K + 127) / 128 * 128);
+  *codes_bytes = size_t(E) * size_t(nmat) * Np * Kp / 2;
+  *sf_bytes = size_t(E) * size_t(nmat) * (Np / 128) * (Kp / 128) * 512;
+  return E4B_OK;
+}
+
+e4b_status e4b_mxfp4_native_prepare(const uint8_t* blocks, const uint8_t* scales, int32_t E,
+                                    int64_t rows_per_mat, int64_t K, int32_t nmat,
+                                    int32_t gate_up_layout, uint8_t* codes_out, uint8_t* sf_out,
+                                    void* stream) {
+  size_t cb = 0, fb = 0;
+  e4b_status st = e4b_mxfp4_native_size(E, rows_per_mat, K, nmat, &cb, &fb);
+  if (st != E4B_OK) return st;
+  if (!blocks || !scales || !codes_out || !sf_out) return E4B_ERR_INVALID_ARG;
+  if (nmat == 2 && gate_up_layout != E4B_GATE_UP_HALVES && gate_up_layout != E4B_GATE_UP_INTERLEAVED)
+    return E4B_ERR_INVALID_ARG;
+  if (!aligned16(blocks) || (reinterpret_cast<uintptr_t>(codes_out) & 31u) || !aligned16(sf_out))
+    return E4B_ERR_MISALIGNED;
+  g_last_launches = 1;
+  return cuda_status(launch_mx_prepare(blocks, scales, E, rows_per_mat, nmat, K,
+                                       nmat == 2 ? gate_up_layout : E4B_GATE_UP_HALVES, codes_out, sf_out,
+                                       static_cast<cudaStream_t>(stream), sm_count()));
+}
+
+e4b_status e4b_quantize_mxfp8(const uint16_t* x, int64_t R, int64_t K, uint8_t* elems, uint8_t* scales,
+                              void* stream) {
+  if (R < 0 || K <= 0) return E4B_ERR_INVALID_ARG;
+  if (K % 32) return E4B_ERR_UNSUPPORTED;
+  g_last_launches = 0;
+  if (R == 0) return E4B_OK;
+  if (!x || !elems || !scales) return E4B_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(elems) & 7u)) return E4B_ERR_MISALIGNED;
+  MxActArgs a{};
+  a.src = x;
+  a.ld_src = K;
+  a.K = K;
+  a.rows = R;
+  a.elems = elems;
+  a.sf = scales;
+  a.nterms = 1;
+  a.plain = true;
+  g_last_launches = 1;
+  return cuda_status(launch_mx_act_quant(a, static_cast<cudaStream_t>(stream), sm_count()));
+}
+
 e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
                            const int32_t* ids, const float* gates, uint16_t* y, void* ws,
                            size_t ws_bytes, uint32_t flags, void* stream) {
@@ -512,6 +696,15 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   if (E > 1024 || T * int64_t(top_k) >= (int64_t(1) << 31)) return E4B_ERR_UNSUPPORTED;
   st = check_variant(w->gate_up_layout, w->activation, w->glu_limit, w->gate_up_bias, w->down_bias);
   if (st != E4B_OK) return st;
+  {
+    const int nmx = (w->gate_up_mx_codes != nullptr) + (w->gate_up_mx_sf != nullptr) +
+                    (w->down_mx_codes != nullptr) + (w->down_mx_sf != nullptr);
+    if (nmx != 0 && (nmx != 4 || w->fmt != E4B_FMT_MXFP4)) return E4B_ERR_INVALID_ARG;
+    if (nmx == 4 && ((reinterpret_cast<uintptr_t>(w->gate_up_mx_codes) & 31u) ||
+                     (reinterpret_cast<uintptr_t>(w->down_mx_codes) & 31u) || !aligned16(w->gate_up_mx_sf) ||
+                     !aligned16(w->down_mx_sf)))
+      return E4B_ERR_MISALIGNED;
+  }
   g_last_launches = 0;
   if (T == 0) return E4B_OK;
   if (!x || !ids || !gates || !y || !ws || !w->gate_up_codes || !w->gate_up_scales ||
@@ -580,6 +773,9 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
     g_last_launches = 2;
     return E4B_OK;
   }
+
+  if (has_mx(w) && !(flags & E4B_FLAG_MX_DECODE))
+    return moe_forward_mx(w, L, x, T, top_k, perm, offsets, inv, gates, y, base, ws_bytes, status, flags, s);
 
   // Large-M: stage the routed rows of x in expert order when the workspace
   // holds the copy (contiguous TMA row tiles), else gather them in the kernel.

@@ -29,11 +29,12 @@ cudaError_t launch_gather_rows(const uint16_t* x, int64_t H, const int32_t* perm
 // routed rows that e4b_moe_workspace_size includes).
 // The path the layer takes for these sizes and flags: true = small-M.
 bool layer_uses_small_m(int64_t R, int64_t E, uint32_t flags);
-// Smallest workspace e4b_moe_forward accepts on that path: the small-M path
-// needs the routing arrays, h and an fp32 [T, H] accumulator; the large-M path
-// the routing arrays, h and the gated rows fp32 [T*top_k, H] (without the
-// staging copy of the routed rows that e4b_moe_workspace_size includes).
-size_t moe_workspace_min_bytes(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k, bool small_m);
+// Smallest workspace e4b_moe_forward accepts for this call (NF4 / MXFP4): the
+// small-M path needs the routing arrays, h and an fp32 [T, H] accumulator; the
+// large-M path the routing arrays, h and the gated rows fp32 [T*top_k, H]
+// (without the staging copy of the routed rows that e4b_moe_workspace_size
+// includes); the block-scaled MXFP4 path also its e4m3 activation terms.
+size_t moe_workspace_min_bytes(const e4b_moe_weights* w, int64_t T, int64_t top_k, uint32_t flags);
 
 // GemmProblem::epilogue for the input gradient through the weights
 // (e4b_grouped_dgrad): out [R, K] bf16, row p = a_p . W_e, a [R, N].
@@ -144,5 +145,59 @@ cudaError_t launch_quantize_int4(const float* w, int64_t nblocks, uint8_t* codes
                                  cudaStream_t st, int sms);
 cudaError_t launch_gptq_repack(const int32_t* qweight, const uint16_t* gscales, int64_t E, int64_t N, int64_t K,
                                uint8_t* codes, uint16_t* scales, cudaStream_t st);
+
+// ----------------------------------------------- MXFP4 block-scaled path
+// (csrc/mx_native.cu)
+// Upper bound on the rows of the padded activation layout: R routed rows,
+// each active expert's rows rounded up to a multiple of 128.
+int64_t mx_padded_rows_max(int64_t R, int64_t E);
+// Prepared copy of one MXFP4 stack (see e4b_mxfp4_native_prepare).
+cudaError_t launch_mx_prepare(const uint8_t* blocks, const uint8_t* scales, int E, int64_t Nm, int nmat,
+                              int64_t K, int layout, uint8_t* out_codes, uint8_t* out_sf, cudaStream_t st,
+                              int sms);
+// bf16 rows -> e4m3 terms + e8m0 scales. Layer layouts: padded rows (expert
+// e's rows from poff[e], a multiple of 128), elems [nterms][rows][Kp], sf
+// chunks [nterms][rows/128][Kp/128][512]; rows = the padded bound. perm set:
+// padded row -> source row perm[p] / top_k (x); null: source row = padded row
+// (h). plain: rows [rows][K] -> elems [rows][K], sf [rows][K/32], one term.
+struct MxActArgs {
+  const uint16_t* src;
+  int64_t ld_src;
+  const int32_t* perm;
+  int32_t top_k;
+  const int64_t* offsets;
+  int32_t E;
+  int64_t K;
+  int64_t rows;
+  uint8_t* elems;
+  uint8_t* sf;
+  int nterms;  // 1 = OCP MXFP8 rule, 2 = exact two-term split
+  bool plain;
+};
+cudaError_t launch_mx_act_quant(const MxActArgs& a, cudaStream_t st, int sms);
+// One projection on the block-scaled tensor cores: gate_up (two matrices,
+// gated activation into bf16 h in padded rows) or down (one matrix, the
+// gate-weighted fp32 row of every routed row).
+struct MxGemmArgs {
+  bool gated_rows;
+  int nterms;
+  int E, top_k;
+  int64_t Nm, K, Rp_max;
+  const uint8_t* codes;
+  const uint8_t* sfa;
+  const uint8_t* act;
+  const uint8_t* sfb;
+  const int64_t* offsets;
+  const int32_t* perm;
+  const float* gates;
+  void* out;
+  int64_t ldo;
+  int layout, act_fn;
+  float alpha, limit;
+  const float* bias;
+  int32_t* status;
+  uint32_t flags;
+};
+cudaError_t launch_mx_gemm(const MxGemmArgs& a, cudaStream_t st, int sms);
 
 }  // namespace e4b

@@ -50,11 +50,7 @@ extern "C" e4b_status e4b_moe_forward_noalloc(const e4b_moe_weights* w, const ui
   // int4-b32 stacks need only the status words and h [top_k, I], whatever T.
   // For NF4 / MXFP4 the staging copy of the routed rows is optional: without
   // room for it the large-M path gathers the rows inside its kernel.
-  const size_t need =
-      w->fmt == E4B_FMT_INT4B32
-          ? full
-          : e4b::moe_workspace_min_bytes(w->E, w->H, w->I, T, top_k,
-                                         e4b::layer_uses_small_m(T * int64_t(top_k), w->E, flags));
+  const size_t need = w->fmt == E4B_FMT_INT4B32 ? full : e4b::moe_workspace_min_bytes(w, T, top_k, flags);
   if (need > kNoallocScratchBytes) return E4B_ERR_EXCEEDS_STATIC_SCRATCH;
   if (T == 0) return e4b_moe_forward(w, x, T, top_k, ids, gates, y, nullptr, 0, flags, stream);
   void* scratch = nullptr;

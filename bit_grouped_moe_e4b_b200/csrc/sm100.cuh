@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -246,6 +247,66 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                   // B format: bf16
          | (uint32_t(N >> 3) << 17)     // N / 8
          | (uint32_t(M >> 4) << 24);    // M / 16
+}
+
+// ------------------------------------------------ block-scaled MMA (MX)
+// D[tmem] (+)= (A * 2^sfa) * (B * 2^sfb)^T, kind::mxf8f6f4 with one e8m0 scale
+// per 32 elements of K for every row of A and B (scale_vec 1X, K = 32 per
+// instruction). The scales are read from TMEM at sfa_tmem / sfb_tmem; which
+// byte of their 32-bit words is in the instruction descriptor.
+E4B_DEV void mma_mxf8f6f4_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with e8m0 scales, both operands
+// K-major, shape M x N; a_fmt / b_fmt: 0 = E4M3, 5 = E2M1. sf_ids: the byte of
+// the scale words (k-block of 32 within a 128-wide K chunk) for A and B.
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, uint32_t a_fmt, uint32_t b_fmt) {
+  return (a_fmt << 7) | (b_fmt << 10) | (uint32_t(N >> 3) << 17) | (1u << 23)  // scale type e8m0
+         | (uint32_t(M >> 4) << 24);
+}
+E4B_DEV uint32_t idesc_mx_ids(uint32_t idesc, uint32_t sfa_id, uint32_t sfb_id) {
+  return idesc | (sfa_id << 29) | (sfb_id << 4);
+}
+
+// Copies 32 rows x 16 bytes of shared memory (rows 16 bytes apart, one
+// 512-byte chunk) into TMEM columns [taddr, taddr + 4) of lanes 0-31, and the
+// same data into each of the other three lane quarters.
+E4B_DEV void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a 512-byte chunk of 32 rows x 16 bytes without
+// swizzle (core matrices of 8 rows x 16 bytes, 128 bytes apart).
+E4B_DEV uint64_t chunk512_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t(128 >> 4) << 32;  // stride byte offset between 8-row core matrices
+  d |= uint64_t(1) << 46;         // descriptor version for sm_100
+  return d;                       // layout type 0: no swizzle
+}
+
+// ----------------------------------------------------------------- e4m3
+// Two fp32 values -> two OCP E4M3 bytes, round to nearest even, magnitudes
+// beyond 448 saturated to 448: the low byte holds lo, the high byte hi.
+E4B_DEV uint32_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two E4M3 bytes (low byte first) -> their exact values.
+E4B_DEV float2 f32x2_from_e4m3x2(uint32_t b) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(uint16_t(b)));
+  const __half2 v = *reinterpret_cast<const __half2*>(&h);
+  return __half22float2(v);
 }
 
 }  // namespace sm100

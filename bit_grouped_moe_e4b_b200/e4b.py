@@ -21,11 +21,13 @@ LIB_PATH = os.path.join(_PKG, "libe4b.so")
 E4B_OK = 0
 E4B_FMT_NF4, E4B_FMT_MXFP4, E4B_FMT_INT4B32 = 0, 1, 2
 E4B_EPI_STORE, E4B_EPI_SWIGLU, E4B_EPI_COMBINE = 0, 1, 2
-E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05, E4B_PATH_INT4_GEMV = 0, 1, 2, 3
+E4B_PATH_NONE, E4B_PATH_GEMV, E4B_PATH_TCGEN05, E4B_PATH_INT4_GEMV, E4B_PATH_TCGEN05_MX = 0, 1, 2, 3, 4
 FLAG_FORCE_GEMV = 0x1
 FLAG_FORCE_TCGEN05 = 0x2
 FLAG_TEST_TIMEOUT = 0x4
 FLAG_IDS_READY = 0x10  # e4b_gemv_int4_b32: ids and gates not written by the preceding work on the stream
+FLAG_MX_ACT_E4M3 = 0x20  # native MXFP4 path: one e4m3 term per activation (OCP MXFP8 rule)
+FLAG_MX_DECODE = 0x40  # MXFP4 with prepared stacks: the decode-to-bf16 tcgen05 path anyway
 FLAG_NF4_PRODUCT_DECODE = 0x8  # small-M NF4: bf16(level * absmax) operands (the default is bf16(level), absmax after the block MMA)
 STATUS_NAMES = {
     0: "E4B_OK", 1: "E4B_ERR_INVALID_ARG", 2: "E4B_ERR_UNSUPPORTED",
@@ -43,6 +45,7 @@ EXPORTED = [
     "e4b_status_string", "e4b_version",
     "e4b_quantize_int4_b32", "e4b_gptq_pack_int4_b32", "e4b_gemv_int4_b32",
     "e4b_ep_dest", "e4b_ep_pack", "e4b_ep_combine",
+    "e4b_mxfp4_native_size", "e4b_mxfp4_native_prepare", "e4b_quantize_mxfp8",
 ]
 EPI = {"store": E4B_EPI_STORE, "swiglu": E4B_EPI_SWIGLU, "combine": E4B_EPI_COMBINE}
 
@@ -61,6 +64,8 @@ class MoeWeights(ctypes.Structure):
         ("gate_up_layout", ctypes.c_int32), ("activation", ctypes.c_int32),
         ("glu_alpha", ctypes.c_float), ("glu_limit", ctypes.c_float),
         ("gate_up_bias", ctypes.c_void_p), ("down_bias", ctypes.c_void_p),
+        ("gate_up_mx_codes", ctypes.c_void_p), ("gate_up_mx_sf", ctypes.c_void_p),
+        ("down_mx_codes", ctypes.c_void_p), ("down_mx_sf", ctypes.c_void_p),
     ]
 
 
@@ -139,6 +144,9 @@ def lib() -> ctypes.CDLL:
         "e4b_ep_dest": [vp, i64, i32, i32, vp, vp],
         "e4b_ep_pack": [vp, i64, vp, vp, i32, vp, vp, i32, i64, i32, vp, vp, vp, vp],
         "e4b_ep_combine": [vp, i64, vp, i64, i32, vp, vp],
+        "e4b_mxfp4_native_size": [i32, i64, i64, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)],
+        "e4b_mxfp4_native_prepare": [vp, vp, i32, i64, i64, i32, i32, vp, vp, vp],
+        "e4b_quantize_mxfp8": [vp, i64, i64, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -219,6 +227,36 @@ def dequantize(fmt: str, codes, scales, E, N, K):
     out = torch.empty((E, N, K), dtype=torch.bfloat16, device=codes.device)
     e4b_dequantize(fmt, codes, scales, E, N, K, out)
     return out
+
+
+def e4b_mxfp4_native_size(E, rows_per_mat, K, nmat):
+    c, f = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib().e4b_mxfp4_native_size(E, rows_per_mat, K, nmat, ctypes.byref(c), ctypes.byref(f)),
+           "e4b_mxfp4_native_size")
+    return c.value, f.value
+
+
+def mxfp4_native_prepare(blocks, scales, E, rows_per_mat, K, nmat, layout="halves", stream=None):
+    """The prepared copy of an MXFP4 stack for the block-scaled FP4 MMA (see
+    e4b.h); returns (codes uint8, scale chunks uint8), flat."""
+    _dev(blocks, scales)
+    cb, fb = e4b_mxfp4_native_size(E, rows_per_mat, K, nmat)
+    codes = torch.empty(cb, dtype=torch.uint8, device=blocks.device)
+    sf = torch.empty(fb, dtype=torch.uint8, device=blocks.device)
+    _check(lib().e4b_mxfp4_native_prepare(_ptr(blocks), _ptr(scales), E, rows_per_mat, K, nmat, LAYOUT[layout],
+                                          _ptr(codes), _ptr(sf), _stream(stream)), "e4b_mxfp4_native_prepare")
+    return codes, sf
+
+
+def quantize_mxfp8(x: torch.Tensor, stream=None):
+    """bf16 [R, K] -> (E4M3 bytes uint8 [R, K], e8m0 scale bytes uint8 [R, K/32])."""
+    _dev(x)
+    R, K = x.shape
+    elems = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((R, K // 32), dtype=torch.uint8, device=x.device)
+    _check(lib().e4b_quantize_mxfp8(_ptr(x), R, K, _ptr(elems), _ptr(scales), _stream(stream)),
+           "e4b_quantize_mxfp8")
+    return elems, scales
 
 
 # ------------------------------------------------------------------ routing
@@ -365,14 +403,33 @@ class PackedLayer:
     limit: float = 7.0
     gate_up_bias: torch.Tensor | None = None  # fp32 [E, 2I]
     down_bias: torch.Tensor | None = None     # fp32 [E, H]
+    # MXFP4 stacks prepared for the block-scaled FP4 MMA (prepare_mx())
+    gate_up_mx_codes: torch.Tensor | None = None
+    gate_up_mx_sf: torch.Tensor | None = None
+    down_mx_codes: torch.Tensor | None = None
+    down_mx_sf: torch.Tensor | None = None
 
     def c_struct(self) -> MoeWeights:
         _dev(self.gate_up_codes, self.gate_up_scales, self.down_codes, self.down_scales,
-             self.gate_up_bias, self.down_bias)
+             self.gate_up_bias, self.down_bias, self.gate_up_mx_codes, self.gate_up_mx_sf,
+             self.down_mx_codes, self.down_mx_sf)
         return MoeWeights(FMT[self.fmt], self.E, self.H, self.I, self.gate_up_codes.data_ptr(),
                           self.gate_up_scales.data_ptr(), self.down_codes.data_ptr(),
                           self.down_scales.data_ptr(), LAYOUT[self.layout], ACT[self.act],
-                          self.alpha, self.limit, _ptr(self.gate_up_bias), _ptr(self.down_bias))
+                          self.alpha, self.limit, _ptr(self.gate_up_bias), _ptr(self.down_bias),
+                          _ptr(self.gate_up_mx_codes), _ptr(self.gate_up_mx_sf), _ptr(self.down_mx_codes),
+                          _ptr(self.down_mx_sf))
+
+    def prepare_mx(self) -> "PackedLayer":
+        """A copy of this MXFP4 layer with its stacks also prepared for the
+        block-scaled FP4 MMA (e4b_mxfp4_native_prepare)."""
+        import dataclasses
+        if self.fmt != "mxfp4":
+            raise ValueError("only MXFP4 stacks have a block-scaled MMA form")
+        gc, gs = mxfp4_native_prepare(self.gate_up_codes, self.gate_up_scales, self.E, self.I, self.H, 2,
+                                      self.layout)
+        dc, ds = mxfp4_native_prepare(self.down_codes, self.down_scales, self.E, self.H, self.I, 1)
+        return dataclasses.replace(self, gate_up_mx_codes=gc, gate_up_mx_sf=gs, down_mx_codes=dc, down_mx_sf=ds)
 
     def packed_bytes_per_expert(self) -> int:
         return (self.gate_up_codes[0].numel() + self.gate_up_scales[0].numel() * self.gate_up_scales.element_size()

@@ -74,7 +74,8 @@ typedef enum {
   E4B_PATH_NONE = 0,
   E4B_PATH_GEMV = 1,   /* small-M: register-fed mma.sync streaming the packed bytes */
   E4B_PATH_TCGEN05 = 2, /* large-M: TMA + on-the-fly decode + tcgen05 MMA into TMEM */
-  E4B_PATH_INT4_GEMV = 3 /* the int4-b32 decode GEMV (dp4a, exact integer block sums) */
+  E4B_PATH_INT4_GEMV = 3, /* the int4-b32 decode GEMV (dp4a, exact integer block sums) */
+  E4B_PATH_TCGEN05_MX = 4 /* large-M MXFP4: e2m1 codes straight into the block-scaled MMA */
 } e4b_path;
 
 /* Flags for e4b_moe_forward / e4b_grouped_gemm. */
@@ -95,6 +96,19 @@ typedef enum {
  * enqueued), so the kernel may start streaming the routed experts' weights
  * before that work completes. It still waits for it before reading x. */
 #define E4B_FLAG_IDS_READY 0x10u
+/* MXFP4 layers with prepared stacks (e4b_moe_weights.*_mx_*), large-M path:
+ * each activation row enters the block-scaled MMA as ONE e4m3 term per value
+ * with an e8m0 scale per 32 (the OCP MXFP8 rule: shared exponent
+ * floor(log2 amax) - 8, round to nearest even, saturating at 448), at half the
+ * MMA count. The results are those of the layer on MXFP8-rounded x and h, not
+ * of the bf16 layer. Without the flag every bf16 activation value is split
+ * into two e4m3 terms x1 + x2 (exponents floor(log2 amax) - 7 of the block
+ * and of its residual), which reproduces it exactly except for values below
+ * ~2^-13 of their block's largest magnitude. */
+#define E4B_FLAG_MX_ACT_E4M3 0x20u
+/* MXFP4 layers with prepared stacks: take the decode-to-bf16 tcgen05 path
+ * anyway on large-M shapes (for comparisons). */
+#define E4B_FLAG_MX_DECODE 0x40u
 
 /* NF4 block size (weights per absmax) and MXFP4 block size (weights per scale). */
 #define E4B_NF4_BLOCK 64
@@ -145,6 +159,15 @@ typedef struct {
   float glu_alpha, glu_limit;
   const float* gate_up_bias;
   const float* down_bias;
+  /* MXFP4 only, optional: the stacks prepared for the block-scaled FP4 MMA
+   * by e4b_mxfp4_native_prepare (gate_up with nmat = 2, down with nmat = 1);
+   * all four set, or all null. With them the large-M path multiplies the
+   * e2m1 codes directly (E4B_PATH_TCGEN05_MX); without them it decodes to
+   * bf16. Codes 32-byte aligned, scale chunks 16-byte aligned. */
+  const uint8_t* gate_up_mx_codes;
+  const uint8_t* gate_up_mx_sf;
+  const uint8_t* down_mx_codes;
+  const uint8_t* down_mx_sf;
 } e4b_moe_weights;
 
 /* ---------------------------------------------------------------- formats */
@@ -182,6 +205,45 @@ e4b_status e4b_quantize_mxfp4(const float* w, int64_t E, int64_t N, int64_t K,
  */
 e4b_status e4b_dequantize(int32_t fmt, const uint8_t* codes, const void* scales, int64_t E,
                           int64_t N, int64_t K, uint16_t* out, void* stream);
+
+/*
+ * MXFP4 stacks for the block-scaled FP4 MMA ([G] intro: MXFP4 as OCP e2m1 +
+ * e8m0 on the released bytes; Blackwell's tcgen05.mma kind::mxf8f6f4 reads
+ * e2m1 codes with one e8m0 scale per 32 elements of K). The tensor memory
+ * access that feeds those codes to the MMA needs rows padded to a multiple of
+ * 128 elements, and the MMA takes its scales as 512-byte chunks of 128 rows x
+ * 4 blocks, so a stack is prepared once into a second copy of its bytes:
+ *   codes uint8 [E][nmat][Np][Kp/2]      the same nibbles (earlier weight low),
+ *                                        rows past rows_per_mat and K zero
+ *   sf    uint8 [E][nmat][Np/128][Kp/128][512]  row r of a 128-row block =
+ *                                        32 m1 + m0, 32-block b of a 128-wide
+ *                                        K chunk: byte 16 m0 + 4 m1 + b; pads 0
+ * with Np, Kp = rows_per_mat and K rounded up to multiples of 128. gate_up
+ * stacks are prepared with nmat = 2 (matrix 0 = the gate rows, matrix 1 = the
+ * up rows, de-interleaved according to gate_up_layout), down stacks with
+ * nmat = 1 (gate_up_layout ignored). The source stack is [E, nmat *
+ * rows_per_mat, K/32, 16] codes + [E, nmat * rows_per_mat, K/32] scales as in
+ * e4b_moe_weights; K % 32 == 0; blocks 16-byte aligned; codes_out 32-byte
+ * aligned; sf_out 16-byte aligned. The prepared copy is read-only afterwards.
+ */
+e4b_status e4b_mxfp4_native_size(int32_t E, int64_t rows_per_mat, int64_t K, int32_t nmat,
+                                 size_t* codes_bytes, size_t* sf_bytes);
+e4b_status e4b_mxfp4_native_prepare(const uint8_t* blocks, const uint8_t* scales, int32_t E,
+                                    int64_t rows_per_mat, int64_t K, int32_t nmat,
+                                    int32_t gate_up_layout, uint8_t* codes_out, uint8_t* sf_out,
+                                    void* stream);
+
+/*
+ * e4b_quantize_mxfp8 -- OCP Microscaling v1.0 MXFP8 with E4M3 elements (the
+ * activations of the block-scaled MMA under E4B_FLAG_MX_ACT_E4M3; the pages do
+ * not name an activation precision). x: bf16 [R, K] (16-byte aligned, K % 32
+ * == 0). Per 32 values along K: amax = max|x|, X = floor(log2 amax) - 8
+ * clamped to [-127, 127], scales[r, b] = X + 127 (0 for an all-zero block),
+ * elems[r, k] = E4M3 bits of x / 2^X rounded to nearest even, saturating at
+ * +-448. elems uint8 [R, K] (8-byte aligned), scales uint8 [R, K/32].
+ */
+e4b_status e4b_quantize_mxfp8(const uint16_t* x, int64_t R, int64_t K, uint8_t* elems, uint8_t* scales,
+                              void* stream);
 
 /* Host: copies the library's 16 NF4 levels (fp32, ascending) into out[16]. */
 e4b_status e4b_nf4_codebook(float* out_host);
@@ -447,6 +509,12 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
  * there). The expert variant must be the plain one (halves, SwiGLU, no
  * biases), top_k <= 64, H % 32 == 0 and I % 32 == 0; flags: 0 or
  * E4B_FLAG_TEST_TIMEOUT. Otherwise E4B_ERR_UNSUPPORTED.
+ * MXFP4 weights with prepared stacks (gate_up_mx_codes ...) take, on the
+ * large-M path, the block-scaled FP4 MMA: x and h are split into e4m3 terms
+ * (see E4B_FLAG_MX_ACT_E4M3) in padded per-expert row blocks inside ws
+ * (e4b_moe_workspace_size then includes them), 6 launches. On the large-M
+ * paths every routed row's gate-weighted output is written once and each
+ * token's rows are summed in slot order, so repeated calls give the same bits.
  */
 e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
                            const int32_t* ids, const float* gates, uint16_t* y, void* ws,

@@ -157,3 +157,73 @@ def route_loops(ids, E):
     for p, s in enumerate(perm):
         inv[s] = p
     return counts, offsets, perm, inv
+
+
+def e4m3_finite_values():
+    """(value, code) for every finite E4M3 pattern, decoded from the bit fields
+    (sign, 4 exponent bits with bias 7, 3 mantissa bits; S.1111.111 is NaN)."""
+    out = []
+    for b in range(256):
+        e, m = (b >> 3) & 15, b & 7
+        if e == 15 and m == 7:
+            continue
+        mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+        out.append((-mag if b & 0x80 else mag, b))
+    return out
+
+
+def e4m3_nearest(v: float) -> float:
+    """Nearest finite E4M3 value by search, ties to the even code, magnitudes
+    beyond 448 saturated to 448."""
+    if abs(v) >= 448.0:
+        return math.copysign(448.0, v)
+    best, best_code, best_d = 0.0, 0, None
+    for val, code in e4m3_finite_values():
+        if code & 0x80:
+            continue  # search magnitudes, then restore the sign
+        d = abs(abs(v) - val)
+        if best_d is None or d < best_d or (d == best_d and code % 2 == 0 and best_code % 2 == 1):
+            best, best_code, best_d = val, code, d
+    return math.copysign(best, v)
+
+
+def mxfp8_row_loops(row):
+    """One row (length % 32 == 0) through MXFP8 and back, block by block."""
+    out = []
+    for b0 in range(0, len(row), 32):
+        blk = [float(v) for v in row[b0:b0 + 32]]
+        amax = max(abs(v) for v in blk)
+        if amax == 0:
+            out.extend([0.0] * 32)
+            continue
+        e = math.floor(math.log2(amax))
+        while 2.0 ** e > amax:
+            e -= 1
+        while 2.0 ** (e + 1) <= amax:
+            e += 1
+        X = max(-127, min(127, e - 8))
+        out.extend(e4m3_nearest(v / 2.0 ** X) * 2.0 ** X for v in blk)
+    return out
+
+
+def moe_loops_mxfp8(x, ids, gates, Wgu, Wd, I):
+    """moe_loops with the x rows and the bf16 h rows replaced by their MXFP8
+    decode before the matmuls that read them."""
+    T = len(x)
+    k = len(ids[0])
+    H = len(x[0])
+    y = [[0.0] * H for _ in range(T)]
+    for t in range(T):
+        xq = mxfp8_row_loops(x[t])
+        for j in range(k):
+            e = ids[t][j]
+            g = [sum(xq[c] * Wgu[e][r][c] for c in range(H)) for r in range(2 * I)]
+            h = []
+            for i in range(I):
+                G, U = g[i], g[I + i]
+                h.append(bf16_nearest(G / (1.0 + math.exp(-G)) * U))
+            hq = mxfp8_row_loops(h)
+            for n in range(H):
+                o = sum(hq[i] * Wd[e][n][i] for i in range(I))
+                y[t][n] += float(np.float32(gates[t][j])) * o
+    return y

@@ -19,6 +19,7 @@ import numpy as np
 
 from .formats import bf16_round, nf4_codebook
 from .moe import activation_ref, expert_tokens, split_gate_up
+from .mxfp8 import mxfp8_round_trip
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(_HERE, "oracle_core.c")
@@ -111,16 +112,23 @@ def matvec(W: np.ndarray, X: np.ndarray) -> np.ndarray:
     return Y
 
 
-def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=None, nf4_decode="product"):
+def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=None, nf4_decode="product",
+                act_quant=None):
     """One expert's contribution for the rows X (bf16 values, [n, H]):
     decode gate_up -> fp64 matmul (+ bias) -> bf16(activation(gate, up)) ->
     decode down -> fp64 matmul (+ bias). ``variant``: dict of moe_forward_ref's
     expert-variant arguments (layout, act, alpha, limit, gu_bias, dn_bias),
     the biases indexed by expert ``e``. ``nf4_decode`` as in moe_forward_ref
-    ("product" or "level"). Returns (O fp64 [n, len(cols)], h)."""
+    ("product" or "level"); ``act_quant`` as in moe_forward_ref (None or
+    "mxfp8"). Returns (O fp64 [n, len(cols)], h)."""
     v = variant or {}
     Wgu = decode(fmt, *packed_gu, 2 * I, H, nf4_decode)
-    GU = matvec(Wgu, np.asarray(X, np.float64))
+    X = np.asarray(X, np.float64)
+    if act_quant == "mxfp8":
+        X = mxfp8_round_trip(X)
+    elif act_quant is not None:
+        raise ValueError(act_quant)
+    GU = matvec(Wgu, X)
     del Wgu
     if v.get("gu_bias") is not None:
         GU = GU + np.asarray(v["gu_bias"][e], np.float64)
@@ -129,7 +137,7 @@ def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=N
     Wd = decode(fmt, *packed_dn, H, I, nf4_decode)
     if cols is not None:
         Wd = np.ascontiguousarray(Wd[cols])
-    O = matvec(Wd, h)
+    O = matvec(Wd, mxfp8_round_trip(h) if act_quant == "mxfp8" else h)
     if v.get("dn_bias") is not None:
         b = np.asarray(v["dn_bias"][e], np.float64)
         O = O + (b if cols is None else b[cols])
@@ -137,7 +145,7 @@ def expert_term(fmt, X, packed_gu, packed_dn, H, I, cols=None, variant=None, e=N
 
 
 def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_rows=None,
-                        packed_fn=None, variant=None, nf4_decode="product", workers=None):
+                        packed_fn=None, variant=None, nf4_decode="product", workers=None, act_quant=None):
     """Outputs y[t, n] for the given tokens (and optionally only the given
     output columns n) of the layer whose fp32 expert weights weight_fn(which,
     e) returns ("gate_up" [2I, H], "down" [H, I]); with packed_fn(which, e)
@@ -175,7 +183,7 @@ def moe_forward_sampled(fmt, x, ids, gates, weight_fn, E, H, I, tokens, down_row
             del src
         X = x[[t for _, t in pairs]]
         O, _ = expert_term(fmt, X, mine["gate_up"], mine["down"], H, I,
-                           None if down_rows is None else cols, variant, e, nf4_decode)
+                           None if down_rows is None else cols, variant, e, nf4_decode, act_quant)
         return e, pairs, mine, O
 
     n = workers or min(len(work), os.cpu_count() or 1)
