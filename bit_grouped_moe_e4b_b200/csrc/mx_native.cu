@@ -249,7 +249,10 @@ __global__ void __launch_bounds__(256) mx_act_quant_kernel(ActQuant q) {
 // ------------------------------------------------------------ the GEMM
 template <int NMAT, int NT>
 struct MxCfg {
-  static constexpr uint32_t kStage = (NMAT + NT) * kTile + 1024;  // tiles + the scale-factor chunks
+  // the tiles, then one 512-byte scale-factor chunk per tile, rounded up to
+  // 1 KB so that the next stage's tiles stay 1024-byte aligned
+  static constexpr uint32_t kSfBytes = ((NMAT + NT) * kChunk + 1023) / 1024 * 1024;
+  static constexpr uint32_t kStage = (NMAT + NT) * kTile + kSfBytes;
   static constexpr int S = NMAT + NT == 4 ? 3 : (NMAT + NT == 3 ? 4 : 6);
   static constexpr int NACC = NMAT == 2 ? 1 : 2;
   static constexpr uint32_t kBars = S * kStage;
@@ -265,6 +268,7 @@ struct MxCfg {
   static constexpr uint32_t kSfCol = 256;  // scale-factor slots after the accumulators
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert((NMAT + NT) * kChunk <= kSfBytes && kStage % 1024 == 0, "stage layout");
   static_assert(kSfCol + S * (NMAT + NT) * 4 <= kTmemCols, "TMEM budget");
   static_assert(NMAT * MBN * NACC <= int(kSfCol), "accumulators");
 };
