@@ -211,7 +211,7 @@ def kernel_bytes(wl, T, ids):
     R = ids.size
     gu = active * 2 * wl.I * wl.H * bpw + 2 * T * wl.H + 4 * R
     dn = active * wl.H * wl.I * bpw + 2 * T * wl.H + 4 * R
-    return {"gate_up": gu, "down": dn, "smallm_layer": gu + dn, "finalize": 6 * T * wl.H,
+    return {"gate_up": gu, "down": dn, "smallm_layer": gu + dn, "combine": 4 * ids.size * wl.H + 2 * T * wl.H,
             "active_experts": active,
             "packed_bytes": active * 3 * wl.H * wl.I * bpw,
             "layer": active * 3 * wl.H * wl.I * bpw + 4 * T * wl.H + 8 * R}
@@ -281,7 +281,7 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
         # routing (+ the staging copy of the routed rows when the workspace
         # holds it), the two tcgen05 projections, the bf16 conversion
         first = "route+stage" if launches_per_step == 5 else "route"
-        spans = ((first, 0, 1), ("gate_up", 1, 2), ("down", 2, 3), ("finalize", 3, 4))
+        spans = ((first, 0, 1), ("gate_up", 1, 2), ("down", 2, 3), ("combine", 3, 4))
     phases = {name: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(steps)]))
               for name, a, b in spans}
     phases["_note"] = "each launch alone (events between launches); the timed steps overlap them"
@@ -400,22 +400,32 @@ def per_config_entry(wl, T, layer, reps, flush, hbm, bf16, peak_src, flags=0, va
         raise RuntimeError(f"device status set in the timed loops: {wl.name} T={T}")
     if path == e4b.E4B_PATH_GEMV:
         spans = (("route", 0, 1), ("smallm_layer", 1, 3))
+    elif path == e4b.E4B_PATH_TCGEN05_MX:
+        # routing + x split into e4m3 terms, gate_up, h split + down, combine
+        spans = (("route+quant_x", 0, 1), ("gate_up", 1, 2), ("quant_h+down", 2, 3), ("combine", 3, 4))
     else:
         spans = (("route+stage" if launches == 5 else "route", 0, 1), ("gate_up", 1, 2), ("down", 2, 3),
-                 ("finalize", 3, 4))
+                 ("combine", 3, 4))
     phases = {n: float(np.median([r[a].elapsed_time(r[b]) for r in evs])) for n, a, b in spans}
     kb = kernel_bytes(wl, T, ids_h)
+    kb["quant_h+down"] = kb["down"]
     R = ids_h.size
     flops = 2.0 * R * 3 * wl.H * wl.I
     kflops = {"gate_up": 2.0 * R * 2 * wl.I * wl.H, "down": 2.0 * R * wl.H * wl.I, "smallm_layer": flops}
+    kflops["quant_h+down"] = kflops["down"]
     ms = ms_a
+    # the block-scaled path runs at the f8f6f4 rate: the measured bf16 peak x 2
+    # (the nominal ratio of the dense fp8 and bf16 peaks)
+    peak = bf16 * (2.0 if path == e4b.E4B_PATH_TCGEN05_MX else 1.0)
     t_bytes = kb["layer"] / (hbm * 1e9)
-    t_flops = flops / (bf16 * 1e12)
+    t_flops = flops / (peak * 1e12)
     dom = max((n for n in phases if n in kflops), key=lambda n: phases[n])
     k_bytes = kb[dom] / (hbm * 1e9)
-    k_flops = kflops[dom] / (bf16 * 1e12)
+    k_flops = kflops[dom] / (peak * 1e12)
     entry = {
-        "workload": wl.name, "T": T, "format": wl.fmt, "path": ["none", "gemv", "tcgen05"][path] + variant,
+        "workload": wl.name, "T": T, "format": wl.fmt,
+        "path": ["none", "gemv", "tcgen05", "int4", "tcgen05_mx"][path] + variant,
+        "tensor_peak_tflops": peak,
         "active_experts": kb["active_experts"], "reps": reps,
         "ms": ms, "ms_graph": ms_g, "self_pair_ms": [ms_a, ms_b],
         "self_pair_spread": abs(ms_a - ms_b) / min(ms_a, ms_b),
@@ -447,6 +457,21 @@ def per_config_table(args, hbm, bf16, peak_src, layers, dev):
             layer = layers[wl.layer] = build_layer(wl, dev)
         for T in wl.T:
             out.append(per_config_entry(wl, T, layer, args.reps, flush, hbm, bf16, peak_src))
+        if wl.fmt == "mxfp4":
+            # the same layer on the block-scaled FP4 MMA, at the token counts
+            # that take the large-M path: two-term (bf16-exact) and one-term
+            # (OCP MXFP8) activations
+            from bit_grouped_moe_e4b_b200 import e4b
+
+            mxl = layer.prepare_mx()
+            plain = {r["T"]: r["path"] for r in out if r["workload"] == wl.name}
+            for T in wl.T:
+                if plain[T] != "tcgen05":
+                    continue
+                out.append(per_config_entry(wl, T, mxl, args.reps, flush, hbm, bf16, peak_src, 0, ""))
+                out.append(per_config_entry(wl, T, mxl, args.reps, flush, hbm, bf16, peak_src,
+                                            e4b.FLAG_MX_ACT_E4M3, "_e4m3"))
+            del mxl
     del flush
     torch.cuda.empty_cache()
     return {"peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": peak_src + " (burst)"},
