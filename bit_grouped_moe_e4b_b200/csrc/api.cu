@@ -84,10 +84,10 @@ MxWs mx_ws_layout(const MoeWs& L, int64_t E, int64_t H, int64_t I, int64_t T, in
   const size_t rp = size_t(m.Rp_max);
   size_t o = L.large_min;
   m.xq = o;  o = align_up(o + 2 * rp * size_t(m.Hp), 256);
-  m.sfx = o; o = align_up(o + 2 * (rp / 128) * size_t(m.Hp / 128) * 512, 256);
+  m.sfx = o; o = align_up(o + 2 * (rp / kMxRowBlock) * size_t(m.Hp / 128) * 512, 256);
   m.hp = o;  o = align_up(o + rp * size_t(I) * 2, 256);
   m.hq = o;  o = align_up(o + 2 * rp * size_t(m.Ip), 256);
-  m.sfh = o; o = align_up(o + 2 * (rp / 128) * size_t(m.Ip / 128) * 512, 256);
+  m.sfh = o; o = align_up(o + 2 * (rp / kMxRowBlock) * size_t(m.Ip / 128) * 512, 256);
   m.total = o;
   return m;
 }

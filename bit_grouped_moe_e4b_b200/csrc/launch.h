@@ -148,16 +148,19 @@ cudaError_t launch_gptq_repack(const int32_t* qweight, const uint16_t* gscales, 
 
 // ----------------------------------------------- MXFP4 block-scaled path
 // (csrc/mx_native.cu)
+// Routed rows per tile of the block-scaled GEMM, and the unit the activation
+// rows of each expert are padded to.
+constexpr int kMxRowBlock = 112;
 // Upper bound on the rows of the padded activation layout: R routed rows,
-// each active expert's rows rounded up to a multiple of 128.
+// each active expert's rows rounded up to a multiple of kMxRowBlock.
 int64_t mx_padded_rows_max(int64_t R, int64_t E);
 // Prepared copy of one MXFP4 stack (see e4b_mxfp4_native_prepare).
 cudaError_t launch_mx_prepare(const uint8_t* blocks, const uint8_t* scales, int E, int64_t Nm, int nmat,
                               int64_t K, int layout, uint8_t* out_codes, uint8_t* out_sf, cudaStream_t st,
                               int sms);
 // bf16 rows -> e4m3 terms + e8m0 scales. Layer layouts: padded rows (expert
-// e's rows from poff[e], a multiple of 128), elems [nterms][rows][Kp], sf
-// chunks [nterms][rows/128][Kp/128][512]; rows = the padded bound. perm set:
+// e's rows from poff[e], a multiple of kMxRowBlock), elems [nterms][rows][Kp],
+// sf chunks [nterms][rows/kMxRowBlock][Kp/128][512]; rows = the padded bound. perm set:
 // padded row -> source row perm[p] / top_k (x); null: source row = padded row
 // (h). plain: rows [rows][K] -> elems [rows][K], sf [rows][K/32], one term.
 struct MxActArgs {

@@ -16,8 +16,8 @@
 //
 //  * mx_act_quant_kernel (per layer call, twice): bf16 activation rows -> e4m3
 //    elements with one e8m0 scale per 32, into rows padded per expert to a
-//    multiple of 128 (x rows gathered through the routing permutation; h rows
-//    already in that order). Two readings (flags):
+//    multiple of 112, one scale-factor chunk per 112 rows (x rows gathered
+//    through the routing permutation; h rows already in that order). Two readings (flags):
 //      - one term: the OCP MXFP8 rule, shared exponent floor(log2 amax) - 8,
 //        e4m3 round to nearest even, saturating at 448;
 //      - two terms (default): x = x1 + x2 with x1 = e4m3(x / 2^X1),
@@ -30,12 +30,13 @@
 //  * mx_gemm_kernel: one persistent CTA per SM, warp-specialised:
 //      warp 0      TMA producer: per 128-wide K chunk, the A tile(s) (128
 //                  weight rows, e2m1 unpacked by TMA to one byte per element,
-//                  128B-swizzled), the B tile(s) (128 routed rows of each term),
+//                  128B-swizzled), the B tile(s) (112 routed rows of each term),
 //                  and the scale-factor chunks by bulk copies;
 //      warp 1      TMEM owner and single-thread MMA issuer: the chunk's scale
 //                  factors go to TMEM with tcgen05.cp (one TMEM slot per ring
 //                  stage), then 4 MMAs of K = 32 per matrix and term;
-//      warps 2-5   epilogue from TMEM: the gated activation into bf16 h
+//      warps 2-5   epilogue from TMEM (two accumulator buffers, so it
+//                  overlaps the next tile's MMAs): the gated activation into bf16 h
 //                  (gate_up), or the gate-weighted fp32 row of every routed row
 //                  (down), summed per token afterwards in a fixed order.
 //    Every wait is bounded; a wait that gives up records E4B_ERR_DEVICE_TIMEOUT,
@@ -52,22 +53,28 @@ namespace {
 using namespace sm100;
 
 constexpr int MBM = 128;  // weight rows per tile (MMA M)
-constexpr int MBN = 128;  // routed rows per tile (MMA N)
+// routed rows per tile (MMA N) and the unit of the per-expert row padding:
+// 112 leaves TMEM room for two accumulator buffers of gate and up (448
+// columns) plus the scale-factor slots, so every epilogue overlaps the next
+// tile's MMAs
+constexpr int MBN = kMxRowBlock;
 constexpr int MBK = 128;  // K per stage
 constexpr int kMxMaxE = 256;
 constexpr int kMxThreads = 192;
-constexpr uint32_t kTile = MBM * MBK;         // 16 KB: a 128 x 128 tile at one byte per element
+constexpr uint32_t kTile = MBM * MBK;         // 16 KB: a 128 x 128 A tile at one byte per element
+constexpr uint32_t kBTile = MBN * MBK;        // 14 KB: a B tile (e4m3)
 constexpr uint32_t kATx = MBM * MBK / 2;      // TMA counts the packed 4-bit bytes of an A tile
-constexpr uint32_t kChunk = 512;              // scale-factor chunk: 128 rows x 4 k-blocks
+constexpr uint32_t kChunk = 512;              // scale-factor chunk: up to 128 rows x 4 k-blocks
+static_assert(MBN % 16 == 0 && MBN <= 128 && kBTile % 1024 == 0, "routed-row tile");
 
-// s_poff[e] = sum over e' < e of the expert's rows rounded up to 128, for
+// s_poff[e] = sum over e' < e of the expert's rows rounded up to MBN, for
 // e = 0..E (one warp).
 E4B_DEV void warp_padded_offsets(const int64_t* offsets, int E, int32_t* s_poff, int lane) {
   int run = 0;
   for (int base = 0; base < E; base += 32) {
     const int e = base + lane;
     int v = 0;
-    if (e < E) v = int((offsets[e + 1] - offsets[e] + 127) / 128) * 128;
+    if (e < E) v = int((offsets[e + 1] - offsets[e] + kMxRowBlock - 1) / kMxRowBlock) * kMxRowBlock;
     int incl = v;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -184,7 +191,7 @@ struct ActQuant {
   int64_t K, Kp;         // row length and padded row length (elements)
   int64_t rows;          // plain: rows; otherwise the padded row bound Rp_max
   uint8_t* elems;        // [NT][rows][Kp] e4m3 (plain: [rows][K])
-  uint8_t* sf;           // [NT][rows/128][Kp/128][512] (plain: [rows][K/32])
+  uint8_t* sf;           // [NT][rows/MBN][Kp/128][512] (plain: [rows][K/32])
   int shift;
 };
 
@@ -236,8 +243,8 @@ __global__ void __launch_bounds__(256) mx_act_quant_kernel(ActQuant q) {
         } else {
           *reinterpret_cast<uint2*>(q.elems + (int64_t(t) * q.rows + pp) * q.Kp + k0) = out[t];
           if ((lane & 3) == 0) {
-            const int64_t chunk = (int64_t(t) * (q.rows / 128) + pp / 128) * kbp + blk / 4;
-            const int r = int(pp % 128);
+            const int64_t chunk = (int64_t(t) * (q.rows / MBN) + pp / MBN) * kbp + blk / 4;
+            const int r = int(pp % MBN);
             q.sf[chunk * kChunk + (r % 32) * 16 + (r / 32) * 4 + (blk % 4)] = uint8_t(sb[t]);
           }
         }
@@ -252,9 +259,9 @@ struct MxCfg {
   // the tiles, then one 512-byte scale-factor chunk per tile, rounded up to
   // 1 KB so that the next stage's tiles stay 1024-byte aligned
   static constexpr uint32_t kSfBytes = ((NMAT + NT) * kChunk + 1023) / 1024 * 1024;
-  static constexpr uint32_t kStage = (NMAT + NT) * kTile + kSfBytes;
+  static constexpr uint32_t kStage = NMAT * kTile + NT * kBTile + kSfBytes;
   static constexpr int S = NMAT + NT == 4 ? 3 : (NMAT + NT == 3 ? 4 : 6);
-  static constexpr int NACC = NMAT == 2 ? 1 : 2;
+  static constexpr int NACC = 2;
   static constexpr uint32_t kBars = S * kStage;
   static constexpr int kNumBars = 2 * S + 4;
   static constexpr uint32_t kScal = kBars + kNumBars * 8;  // tmem base, abort, n active
@@ -265,12 +272,12 @@ struct MxCfg {
   static constexpr uint32_t kRow = kGate + 4 * MBN * 4;
   static constexpr uint32_t kEnd = kRow + 4 * MBN * 4;
   static constexpr uint32_t kSmemBytes = kEnd + 1024;
-  static constexpr uint32_t kSfCol = 256;  // scale-factor slots after the accumulators
+  static constexpr uint32_t kSfCol = NMAT * MBN * NACC;  // scale-factor slots after the accumulators
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert((NMAT + NT) * kChunk <= kSfBytes && kStage % 1024 == 0, "stage layout");
   static_assert(kSfCol + S * (NMAT + NT) * 4 <= kTmemCols, "TMEM budget");
-  static_assert(NMAT * MBN * NACC <= int(kSfCol), "accumulators");
+  static_assert(kSfCol % 4 == 0, "scale-factor slots");
 };
 
 struct MxGemm {
@@ -282,7 +289,7 @@ struct MxGemm {
   const uint8_t* codes;    // prepared [E][nmat][Np][Kp/2]
   const uint8_t* sfa;      // prepared [E][nmat][Np/128][Kp/128][512]
   const uint8_t* act;      // [nt][Rp_max][Kp] e4m3
-  const uint8_t* sfb;      // [nt][Rp_max/128][Kp/128][512]
+  const uint8_t* sfb;      // [nt][Rp_max/MBN][Kp/128][512]
   const int64_t* offsets;  // [E+1]
   const int32_t* perm;     // [R] slot of each routed row
   const float* gates;      // [T*top_k]
@@ -409,8 +416,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   const int my_tiles = (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x);
   auto stage = [&](int s) { return smem + uint32_t(s) * C::kStage; };
   auto a_tile = [&](int s, int m) { return stage(s) + uint32_t(m) * kTile; };
-  auto b_tile = [&](int s, int t) { return stage(s) + uint32_t(NMAT + t) * kTile; };
-  auto sf_chunk = [&](int s, int i) { return stage(s) + uint32_t(NMAT + NT) * kTile + uint32_t(i) * kChunk; };
+  auto b_tile = [&](int s, int t) { return stage(s) + uint32_t(NMAT) * kTile + uint32_t(t) * kBTile; };
+  auto sf_chunk = [&](int s, int i) {
+    return stage(s) + uint32_t(NMAT) * kTile + uint32_t(NT) * kBTile + uint32_t(i) * kChunk;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
@@ -427,7 +436,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
             aborted = true;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], NMAT * kATx + NT * kTile + (NMAT + NT) * kChunk);
+          mbar_arrive_expect_tx(&full[s], NMAT * kATx + NT * kBTile + (NMAT + NT) * kChunk);
 #pragma unroll
           for (int m = 0; m < NMAT; ++m) {
             tma_load_2d(a_tile(s, m), &tmap_a, &full[s], kb * MBK,
@@ -461,7 +470,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
           break;
         }
         tc_fence_after();
-        const uint32_t dcol = tmem + uint32_t(NMAT == 2 ? 0 : ab * MBN);
+        const uint32_t dcol = tmem + uint32_t(ab * NMAT * MBN);
         for (int kb = 0; kb < KB; ++kb, ++i) {
           const int s = int(i % S);
           if (!mbar_wait_bounded(&full[s], uint32_t(i / S) & 1u, limit, s_abort)) {
@@ -513,8 +522,9 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         // itself while the tile's MMAs run
         __syncwarp();
 #pragma unroll
-        for (int u = 0; u < MBN / 32; ++u) {
+        for (int u = 0; u < (MBN + 31) / 32; ++u) {
           const int ii = lane + 32 * u;
+          if (ii >= MBN) break;
           const bool ok = ii < T.rows;
           const int32_t slot = ok ? p.perm[T.p0 + ii] : 0;
           s_p[ii] = ok ? int32_t(T.p0 + ii) : -1;
@@ -535,7 +545,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         b0 = b[NMAT == 2 ? gate_up_row(p.layout, p.Nm, 0, n) : n];
         if constexpr (NMAT == 2) b1 = b[gate_up_row(p.layout, p.Nm, 1, n)];
       }
-      const uint32_t lane_base = tmem + (uint32_t(q * 32) << 16) + uint32_t(NMAT == 2 ? 0 : ab * MBN);
+      const uint32_t lane_base = tmem + (uint32_t(q * 32) << 16) + uint32_t(ab * NMAT * MBN);
       for (int cc = 0; cc < MBN / 16; ++cc) {
         if (cc * 16 >= T.rows) break;  // uniform: the rest of the tile is padding
         uint32_t g[16];
@@ -636,7 +646,7 @@ cudaError_t launch_mx_t(const MxGemm& p, cudaStream_t st, int sms) {
 
 int64_t mx_padded_rows_max(int64_t R, int64_t E) {
   const int64_t active = R < E ? R : E;
-  return (R + 127) / 128 * 128 + 128 * active;
+  return (R + kMxRowBlock - 1) / kMxRowBlock * kMxRowBlock + int64_t(kMxRowBlock) * active;
 }
 
 cudaError_t launch_mx_prepare(const uint8_t* blocks, const uint8_t* scales, int E, int64_t Nm, int nmat,
