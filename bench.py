@@ -275,8 +275,8 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
     barrier()
     ms = t0.elapsed_time(t1)
     path = e4b.e4b_last_path()
-    if path == e4b.E4B_PATH_GEMV:  # routing + one fused small-M layer kernel
-        spans = (("route", 0, 1), ("smallm_layer", 1, 3))
+    if path == e4b.E4B_PATH_GEMV:  # routing, the fused small-M layer kernel, the combine
+        spans = (("route", 0, 1), ("smallm_layer", 1, 3), ("combine", 3, 4))
     else:
         # routing (+ the staging copy of the routed rows when the workspace
         # holds it), the two tcgen05 projections, the bf16 conversion
@@ -399,7 +399,7 @@ def per_config_entry(wl, T, layer, reps, flush, hbm, bf16, peak_src, flags=0, va
     if e4b.e4b_read_device_status(ws) != 0:
         raise RuntimeError(f"device status set in the timed loops: {wl.name} T={T}")
     if path == e4b.E4B_PATH_GEMV:
-        spans = (("route", 0, 1), ("smallm_layer", 1, 3))
+        spans = (("route", 0, 1), ("smallm_layer", 1, 3), ("combine", 3, 4))
     elif path == e4b.E4B_PATH_TCGEN05_MX:
         # routing + x split into e4m3 terms, gate_up, h split + down, combine
         spans = (("route+quant_x", 0, 1), ("gate_up", 1, 2), ("quant_h+down", 2, 3), ("combine", 3, 4))

@@ -36,11 +36,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace of the layer forward. After the routing arrays and h comes one
-// region that the small-M path uses as its fp32 accumulator acc [T, H]
-// (needs up to small_min) and the large-M path as the gate-weighted fp32 rows
-// [T*top_k, H] (needs up to large_min); xs (the routed rows of x in expert
-// order) is the large-M path's staging copy, used when the workspace reaches
-// total.
+// fp32 region that the small-M path uses for the partial sums of its down
+// passes, [K slices][T*top_k][H] (needs up to small_min), and the large-M path
+// for the gate-weighted rows [T*top_k, H] (needs up to large_min); xs (the
+// routed rows of x in expert order) is the large-M path's staging copy, after
+// the larger of the two, used when the workspace reaches total.
 struct MoeWs {
   size_t status, sync, nsync, counts, offsets, perm, inv, h, acc, small_min, rows, large_min, xs, total;
 };
@@ -59,9 +59,9 @@ MoeWs moe_ws_layout(int64_t E, int64_t H, int64_t I, int64_t T, int64_t top_k) {
   w.h = o;       o = align_up(o + size_t(R) * size_t(I) * 2, 256);
   w.acc = o;
   w.rows = o;
-  w.small_min = align_up(o + size_t(T) * size_t(H) * 4, 256);
+  w.small_min = align_up(o + size_t(smallm_k_slices(int(I))) * size_t(R) * size_t(H) * 4, 256);
   w.large_min = align_up(o + size_t(R) * size_t(H) * 4, 256);
-  o = w.large_min;
+  o = w.small_min > w.large_min ? w.small_min : w.large_min;
   w.xs = o;      o = align_up(o + size_t(R) * size_t(H) * 2, 256);
   w.total = o;
   return w;
@@ -735,7 +735,8 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   if (ce != cudaSuccess) return E4B_ERR_CUDA;
 
   if (gemv) {
-    // small-M: both projections, SwiGLU, combine and bf16 output in one launch
+    // small-M: both projections and the SwiGLU in one launch, then the
+    // fixed-order combine into bf16 y
     SmallMLayer sl{};
     sl.fmt = w->fmt;
     sl.E = int(E);
@@ -752,7 +753,8 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
     sl.offsets = offsets;
     sl.gates = gates;
     sl.h = h;
-    sl.acc = acc;
+    sl.part = acc;
+    sl.inv = inv;
     sl.y = y;
     sl.sync = sync;
     sl.status = status;
@@ -768,9 +770,11 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
     ce = launch_smallm_layer(sl, s, sm_count());
     if (ce != cudaSuccess) return E4B_ERR_CUDA;
     mark(3, s);
+    ce = launch_smallm_combine(sl, s, sm_count());
+    if (ce != cudaSuccess) return E4B_ERR_CUDA;
     mark(4, s);
     g_last_path = E4B_PATH_GEMV;
-    g_last_launches = 2;
+    g_last_launches = 3;
     return E4B_OK;
   }
 

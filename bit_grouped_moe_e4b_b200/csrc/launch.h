@@ -94,7 +94,8 @@ struct SmallMLayer {
   const int64_t* offsets;
   const float* gates;
   uint16_t* h;
-  float* acc;
+  float* part;     // [smallm_k_slices(I), T*top_k, H] fp32 partial sums of the down passes
+  const int32_t* inv;  // [T*top_k] routed row of each slot (-1: dropped)
   uint16_t* y;
   int32_t* sync;   // smallm_sync_ints(E, H) ints, zero on entry
   int32_t* status;
@@ -105,7 +106,12 @@ struct SmallMLayer {
   const float* dn_bias;  // fp32 [E, H] or null
 };
 size_t smallm_sync_ints(int E, int H);
+// K slices of the small-M down passes (the partial sums kept per slice).
+int smallm_k_slices(int I);
 cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms);
+// The fixed-order sum of the partial sums into bf16 y (a programmatic
+// dependent of launch_smallm_layer).
+cudaError_t launch_smallm_combine(const SmallMLayer& L, cudaStream_t st, int sms);
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms);
 cudaError_t launch_finalize(const float* acc, int64_t n, uint16_t* y, cudaStream_t st, int sms);
 

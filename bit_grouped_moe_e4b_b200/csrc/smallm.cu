@@ -22,9 +22,12 @@
 //  * gate_up items (one expert, 128 gate rows and the matching 128 up rows,
 //    all of K) end in the SwiGLU and store bf16 h; down items (one expert,
 //    256 output rows, a 2048-wide K slice) wait, bounded, until every gate_up
-//    item of their expert has stored h, and end in gate-weighted fp32 atomics
-//    into the accumulator; the last warp to finish a 256-row output slice
-//    converts it to bf16.
+//    item of their expert has stored h, and store their fp32 partial sums,
+//    one per K slice and routed row, with no atomics;
+//  * a second, small kernel (launched as a programmatic dependent) sums each
+//    token's slots and K slices in a fixed order, weights them by the gates
+//    and writes bf16 y, so the result does not depend on the order in which
+//    the passes ran.
 // Every wait is bounded; a wait that gives up records E4B_ERR_DEVICE_TIMEOUT
 // and all warps stop.
 #include "common.cuh"
@@ -51,14 +54,11 @@ constexpr uint64_t kStageWaitNs = 100000000;  // 100 ms for a stage; 16x that fo
 constexpr uint64_t kDrainNs = 1000000000;     // the copies still landing at exit
 constexpr int kKSplit = 2048;                    // K slice of a down item
 
-// sync words (int32) at the start of the layer's sync area:
-//   work item counter, zeroing-chunk counter, zeroed-chunk count, then
-//   done_A[E] (finished gate_up passes per active expert, one count per
-//   consumer warp) and arrive[] (finished down passes per 256-row output
-//   slice, one count per consumer warp). Cleared by the routing kernel before
-//   every layer call.
-enum : int { kWork = 0, kZeroWork = 1, kZeroDone = 2, kDoneA = 3 };
-constexpr int64_t kZeroChunk = 16384;  // floats per zeroing chunk
+// sync words (int32) at the start of the layer's sync area: the work item
+// counter, then done_A[E] (finished gate_up passes per active expert, one
+// count per consumer warp). Cleared by the routing kernel before every layer
+// call.
+enum : int { kWork = 0, kDoneA = 1 };
 
 E4B_DEV void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                       uint32_t b1) {
@@ -159,8 +159,7 @@ struct Params {
   const int64_t* offsets;
   const float* gates;
   uint16_t* h;       // [R, I] bf16, expert-ordered rows
-  float* acc;        // [T, H] fp32
-  uint16_t* y;       // [T, H] bf16
+  float* part;       // [NKS, R, H] fp32: down partial sums per K slice and routed row
   int32_t* sync;     // see the sync words above
   int32_t* status;
   uint32_t flags;
@@ -313,7 +312,7 @@ struct Work {
 // bounded wait gives up.
 template <int FMT>
 E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int32_t* s_act, uint8_t* stages,
-                     uint64_t* full, uint64_t* empty, StageInfo* info, volatile int* s_abort, int nzero,
+                     uint64_t* full, uint64_t* empty, StageInfo* info, volatile int* s_abort,
                      uint64_t limit) {
   constexpr int kStages = Geo<FMT>::kStages;
   constexpr int kSlot = Geo<FMT>::kSlot;
@@ -362,14 +361,11 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
     const int ngroups = int((p1 - p0 + kMaxTok - 1) / kMaxTok);
     if (down) {
       // h of this expert complete (every gate_up pass of it, one count per
-      // consumer warp) and the accumulator cleared
+      // consumer warp)
       int ok = 1;
-      if (lane == 0)
-      {
+      if (lane == 0) {
         ok = wait_geq(p.sync + kDoneA + ai, W.MTA * ngroups * kConsumers, 16 * limit, s_abort);
         if (!ok) record_wait_site(p.status, 2, i);
-        ok = ok && wait_geq(p.sync + kZeroDone, nzero, 16 * limit, s_abort);
-        if (!ok) record_wait_site(p.status, 3, i);
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         give_up();
@@ -571,8 +567,7 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
 // and up rows of an output are neighbours, four lanes apart in the fragment.
 template <int FMT, bool SA>
 E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
-                     const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, int arrive_target,
-                     uint64_t limit) {
+                     const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, uint64_t limit) {
   constexpr int kStages = Geo<FMT>::kStages;
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;  // 0 .. kConsumers-1
@@ -580,7 +575,6 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
   const int c = lane & 3;
   const int H = p.H, I = p.I;
   int32_t* done_A = p.sync + kDoneA;
-  int32_t* arrive = p.sync + kDoneA + p.E;
   float acc[2][4];
 #pragma unroll
   for (int j = 0; j < 2; ++j)
@@ -687,40 +681,20 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
       __syncwarp();
       if (lane == 0) atomicAdd(done_A + f.ai, 1);
     } else {
-      // the down bias joins the first K slice's partial sum only
-      const float* db = p.dn_bias && f.kc < kKSplit ? p.dn_bias + int64_t(f.e) * H : nullptr;
+      // the partial sum of this K slice for every routed row of the pass; the
+      // down bias joins the first K slice only
+      const int ks = f.kc / kKSplit;
+      const int64_t R = p.T * p.top_k;
+      const float* db = p.dn_bias && ks == 0 ? p.dn_bias + int64_t(f.e) * H : nullptr;
+      float* part = p.part + int64_t(ks) * R * H;
       for (int j = 0; j < nt; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int tok = 8 * j + 2 * c + (q & 1);
           const int n = f.mt * 256 + 16 * w + g + ((q & 2) ? 8 : 0);
           if (tok >= f.ntok || n >= H) continue;
-          const int slot = p.perm[f.p0 + tok];
-          const float v = acc[j][q] + (db ? db[n] : 0.f);
-          atomicAdd(p.acc + int64_t(slot / p.top_k) * H + n, p.gates[slot] * v);
+          part[int64_t(f.p0 + tok) * H + n] = acc[j][q] + (db ? db[n] : 0.f);
         }
-      // the last warp to finish a pass over this 256-row output slice
-      // converts the slice to bf16
-      __threadfence();
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) last = atomicAdd(arrive + f.mt, 1) == arrive_target - 1;
-      if (__shfl_sync(0xffffffffu, last, 0)) {
-        __threadfence();
-        const int n0 = f.mt * 256;
-        const int width = min(256, H - n0);  // a multiple of 32
-        for (int64_t q = lane; q < p.T * (width / 4); q += 32) {
-          const int64_t t = q / (width / 4);
-          const int part = int(q % (width / 4));
-          const float* src = p.acc + t * H + n0 + part * 4;
-          float4 v;
-          asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
-                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                       : "l"(src));
-          *reinterpret_cast<uint2*>(p.y + t * H + n0 + part * 4) =
-              make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-        }
-      }
     }
 #pragma unroll
     for (int j = 0; j < 2; ++j)
@@ -737,8 +711,6 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   __shared__ int32_t s_act[1024];
   __shared__ int32_t s_n;
   __shared__ int32_t s_wscr[kThreads / 32 + 1];
-  __shared__ int s_zc;
-  __shared__ int s_arrive_target;
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int H = p.H, I = p.I;
@@ -766,30 +738,10 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   // output or the counters it clears
   grid_dependency_wait();
 
-  // Clear the fp32 accumulator in chunks handed out by a counter, so that
-  // waiting on the cleared count only depends on CTAs that are running.
-  const int64_t nacc = p.T * int64_t(H);
-  const int nzero = int((nacc + kZeroChunk - 1) / kZeroChunk);
-  while (true) {
-    if (threadIdx.x == 0) s_zc = atomicAdd(p.sync + kZeroWork, 1);
-    __syncthreads();
-    const int zc = s_zc;
-    __syncthreads();
-    if (zc >= nzero) break;
-    const int64_t b0 = int64_t(zc) * kZeroChunk;
-    const int64_t b1 = min(nacc, b0 + kZeroChunk);
-    for (int64_t i = b0 + threadIdx.x; i < b1; i += kThreads) p.acc[i] = 0.f;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      atomicAdd(p.sync + kZeroDone, 1);
-    }
-  }
   block_active_experts(p.offsets, p.E, s_act, &s_n, s_wscr);  // ends with __syncthreads
   const int nact = s_n;
-  if (nact == 0) {  // no routed slot at all: the output is zero
-    for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < nacc; i += int64_t(gridDim.x) * kThreads)
-      p.y[i] = 0;
+  if (nact == 0) {  // no routed slot: nothing to compute (the combine writes zeros)
+    grid_launch_dependents();
     return;
   }
   Work W;
@@ -798,31 +750,73 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   W.NKS = (I + kKSplit - 1) / kKSplit;
   W.nA = nact * W.MTA;
   W.nB = nact * W.MTB * W.NKS;
-  // passes over each 256-row output slice: every K slice of every routed-row
-  // group of every active expert, one count per consumer warp
-  if (wid == 0) {
-    int groups = 0;
-    for (int a = lane; a < nact; a += 32) {
-      const int e = s_act[a];
-      groups += int((p.offsets[e + 1] - p.offsets[e] + kMaxTok - 1) / kMaxTok);
-    }
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) groups += __shfl_xor_sync(0xffffffffu, groups, d);
-    if (lane == 0) s_arrive_target = groups * W.NKS * kConsumers;
-  }
-  __syncthreads();
-
   if (wid == kConsumers) {
-    produce<FMT>(maps, p, W, s_act, stages, full, empty, info, s_abort, nzero, limit);
+    produce<FMT>(maps, p, W, s_act, stages, full, empty, info, s_abort, limit);
+    // no more work items for this CTA: the combine kernel may start launching
+    // (it waits for this whole grid before reading the partial sums)
+    grid_launch_dependents();
   } else {
     const uint32_t lut_lane = smem_u32(smem) + uint32_t(!SA ? 8 * (lane & 15) : 4 * lane);
-    consume<FMT, SA>(p, stages, full, empty, info, s_abort, lut_lane, s_arrive_target, limit);
+    consume<FMT, SA>(p, stages, full, empty, info, s_abort, lut_lane, limit);
   }
 }
 
 }  // namespace
 
-size_t smallm_sync_ints(int E, int H) { return size_t(kDoneA) + E + H / 16; }
+size_t smallm_sync_ints(int E, int H) {
+  (void)H;
+  return size_t(kDoneA) + E;
+}
+
+// y[t, n] = bf16( sum_j gates[s] * sum_ks part[ks][inv[s]][n] ), s = t*k + j,
+// in that order (fp32); slots whose inv is -1 add nothing. One thread per 4
+// consecutive outputs of a token.
+__global__ void __launch_bounds__(256) smallm_combine_kernel(const float* __restrict__ part,
+                                                              const int32_t* __restrict__ inv,
+                                                              const float* __restrict__ gates, int64_t T,
+                                                              int32_t k, int64_t H4, int32_t nks, int64_t R,
+                                                              uint16_t* __restrict__ y) {
+  grid_dependency_wait();  // the layer kernel's partial sums
+  const int64_t total = T * H4;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = i / H4;
+    const int64_t c = i - t * H4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const int64_t s = t * k + j;
+      const int32_t p = __ldg(inv + s);
+      if (p < 0) continue;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int ks = 0; ks < nks; ++ks) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(part + (int64_t(ks) * R + p) * (H4 * 4)) + c);
+        o.x += v.x;
+        o.y += v.y;
+        o.z += v.z;
+        o.w += v.w;
+      }
+      const float gw = __ldg(gates + s);
+      acc.x += gw * o.x;
+      acc.y += gw * o.y;
+      acc.z += gw * o.z;
+      acc.w += gw * o.w;
+    }
+    reinterpret_cast<uint2*>(y)[i] = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  }
+}
+
+int smallm_k_slices(int I) { return (I + kKSplit - 1) / kKSplit; }
+
+cudaError_t launch_smallm_combine(const SmallMLayer& L, cudaStream_t st, int sms) {
+  const int64_t total = L.T * (L.H / 4);
+  int64_t grid = (total + 255) / 256;
+  if (grid > int64_t(sms) * 8) grid = int64_t(sms) * 8;
+  if (grid < 1) grid = 1;
+  return launch_dependent(smallm_combine_kernel, dim3(unsigned(grid)), dim3(256), 0, st,
+                          static_cast<const float*>(L.part), static_cast<const int32_t*>(L.inv), L.gates, L.T,
+                          int32_t(L.top_k), int64_t(L.H / 4), int32_t(smallm_k_slices(L.I)),
+                          int64_t(L.T * L.top_k), L.y);
+}
 
 cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) {
   Params p;
@@ -840,8 +834,7 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms) 
   p.offsets = L.offsets;
   p.gates = L.gates;
   p.h = L.h;
-  p.acc = L.acc;
-  p.y = L.y;
+  p.part = L.part;
   p.sync = L.sync;
   p.status = L.status;
   p.flags = L.flags;

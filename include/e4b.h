@@ -474,9 +474,10 @@ e4b_status e4b_ep_combine(const uint16_t* ys, int64_t H, const int32_t* inv_perm
 
 /* Host: workspace bytes for e4b_moe_forward with T tokens and top_k slots.
  * The workspace holds the status word, the routing arrays, h, one fp32 region
- * (the small-M path's accumulator [T, H], or the large-M path's gate-weighted
- * rows [T*top_k, H]) and last a staging copy of the routed rows of x in expert
- * order ([T*top_k, H] bf16) that the large-M path uses. A smaller workspace
+ * (the small-M path's partial sums [ceil(I/2048)][T*top_k][H] of its down
+ * passes, or the large-M path's gate-weighted rows [T*top_k, H]) and last a
+ * staging copy of the routed rows of x in expert order ([T*top_k, H] bf16)
+ * that the large-M path uses. A smaller workspace
  * that holds everything the chosen path needs but the staging copy is
  * accepted; the large-M path then gathers the rows inside its kernel (same
  * results, slower). */
@@ -512,9 +513,11 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
  * MXFP4 weights with prepared stacks (gate_up_mx_codes ...) take, on the
  * large-M path, the block-scaled FP4 MMA: x and h are split into e4m3 terms
  * (see E4B_FLAG_MX_ACT_E4M3) in padded per-expert row blocks inside ws
- * (e4b_moe_workspace_size then includes them), 6 launches. On the large-M
- * paths every routed row's gate-weighted output is written once and each
- * token's rows are summed in slot order, so repeated calls give the same bits.
+ * (e4b_moe_workspace_size then includes them), 6 launches. On every path each
+ * routed row's output (small-M: each 2048-wide K slice's partial sum) is
+ * written once and each token's rows are summed in a fixed order, so repeated
+ * calls give the same bits. Launches: small-M 3 (routing, the layer kernel,
+ * the combine), large-M 5 (4 without the staging copy).
  */
 e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
                            const int32_t* ids, const float* gates, uint16_t* y, void* ws,
@@ -538,10 +541,11 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
  * enqueues nothing. The required scratch is, for NF4 and MXFP4 stacks,
  * the part of e4b_moe_workspace_size the chosen path needs (without the
  * optional staging copy; a layer with E=8, H=4096, I=14336 and top-2 routing
- * fits up to 186 tokens on the large-M path it takes from 65 tokens on, and up
- * to 227 with E4B_FLAG_FORCE_GEMV; the staging copy is used while it also
- * fits), and for int4-b32 stacks e4b_moe_workspace_size itself, which does
- * not grow with T. Nothing is allocated or freed.
+ * fits up to 58 tokens on the small-M path it takes up to 64 tokens, and up to
+ * 186 tokens on the large-M path it takes from 65 tokens on; the staging copy
+ * is used while it also fits), and for int4-b32 stacks
+ * e4b_moe_workspace_size itself, which does not grow with T. Nothing is
+ * allocated or freed.
  *   - The first call on each device looks up that device's copy of the
  *     array (set-up, once per device); make that first call before any stream
  *     capture begins. The address found belongs to the device's context as it

@@ -51,9 +51,9 @@ def test_tiny_workload(path):
     assert_close(y, y_ref, f"tiny workload, {path}")
     if path != "auto":
         assert e4b.e4b_last_path() == (e4b.E4B_PATH_GEMV if path == "gemv" else e4b.E4B_PATH_TCGEN05)
-    # small-M: routing + one fused layer kernel; tcgen05: routing, staging of
-    # the routed rows, two GEMMs, conversion
-    assert e4b.e4b_last_launch_count() == (2 if e4b.e4b_last_path() == e4b.E4B_PATH_GEMV else 5)
+    # small-M: routing, the fused layer kernel, the fixed-order combine;
+    # tcgen05: routing, staging of the routed rows, two GEMMs, the combine
+    assert e4b.e4b_last_launch_count() == (3 if e4b.e4b_last_path() == e4b.E4B_PATH_GEMV else 5)
 
 
 # shapes that span several tiles of both kernels and leave ragged tails:
@@ -211,10 +211,11 @@ def test_grouped_gemm_store_epilogue():
         assert_close(out.float().cpu().numpy(), want, f"store flags={flags}")
 
 
-@pytest.mark.parametrize("path", ["tcgen05", "tcgen05_gather"])
-def test_large_m_combine_is_deterministic(path):
-    # the large-M path writes each routed row's gate-weighted output once and
-    # sums every token's rows in slot order: repeated calls give the same bits
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+def test_combine_is_deterministic(path):
+    # every path writes each routed row's output (small-M: each K slice's
+    # partial sum) once and sums every token's rows in a fixed order:
+    # repeated calls give the same bits
     fmt, E, H, I, T, k = "nf4", 16, 256, 384, 300, 8
     layer, ref = small_layer(fmt, E, H, I, seed=91)
     x = _x(T, H, seed=92)

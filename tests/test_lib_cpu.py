@@ -66,14 +66,12 @@ def test_host_argument_checks_return_before_launch():
     # misaligned
     assert fwd(ctypes.byref(w), ctypes.c_void_p(4098), 4, 2, p, p, p, p, need, 0, None) == 7
     # workspace too small: below the required part of the path taken. The size
-    # query ends with one fp32 region (the small-M path's accumulator [T, H],
-    # or the large-M path's gate-weighted rows [T*k, H]) and an optional
-    # [T*k, H] bf16 staging copy, each 256-byte aligned; the small-M path
-    # (T*k = 128 <= 16 E here) needs the accumulator part of the region only.
+    # query ends with one fp32 region (the small-M path's partial sums
+    # [K slices][T*k][H], or the large-M path's gate-weighted rows [T*k, H];
+    # one K slice here, I = 512) and an optional [T*k, H] bf16 staging copy,
+    # each 256-byte aligned; both paths need everything but the staging copy.
     staging = (64 * 2 * 256 * 2 + 255) // 256 * 256
-    rows = (64 * 2 * 256 * 4 + 255) // 256 * 256
-    acc = (64 * 256 * 4 + 255) // 256 * 256
-    assert fwd(ctypes.byref(w), p, 64, 2, p, p, p, p, need - staging - rows + acc - 1, 0, None) == 3
+    assert fwd(ctypes.byref(w), p, 64, 2, p, p, p, p, need - staging - 1, 0, None) == 3
     assert fwd(ctypes.byref(w), p, 64, 2, p, p, p, p, need - staging - 1, e4b.FLAG_FORCE_TCGEN05, None) == 3
     # bad format
     assert fwd(ctypes.byref(_w(fmt=5)), p, 4, 2, p, p, p, p, need, 0, None) == 1
