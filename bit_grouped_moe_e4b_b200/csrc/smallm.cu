@@ -501,7 +501,7 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
 // hence inside one scale block of each row.
 template <int FMT, int NT, bool SA>
 E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, int rB, uint64_t mxA,
-                           uint64_t mxB, uint32_t lut_lane, const Lut& lreg, float (&acc)[2][4]) {
+                           uint64_t mxB, uint32_t lut_lane, float (&acc)[2][4]) {
   static_assert(SA || FMT == E4B_FMT_NF4, "MXFP4 scales always apply after the block's MMA");
   constexpr int kSlot = Geo<FMT>::kSlot;
   constexpr int BLK = FMT == E4B_FMT_NF4 ? 64 : 32;  // weights per scale block
@@ -538,15 +538,7 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
       const uint32_t sw = uint32_t((ch ^ g) << 4);  // the 128B swizzle of chunk ch in row g (mod 8)
       uint32_t dA[4], dB[4];
       lut_lookup8<SA>(lut_lane, lds32(cA + sw), sA2, dA);
-      if constexpr (SA) {
-        // the operand does not depend on the block's scale: row B decodes
-        // through the 16 values held in registers (byte permutes on the
-        // integer pipe), row A through the shared-memory byte table, so the
-        // two rows share the load of two otherwise separate pipes
-        lut_decode8<FMT>(lreg, lds32(cB + sw), dB);
-      } else {
-        lut_lookup8<SA>(lut_lane, lds32(cB + sw), sB2, dB);
-      }
+      lut_lookup8<SA>(lut_lane, lds32(cB + sw), sB2, dB);
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         float(&D)[4] = SA ? P[j] : acc[j];
@@ -590,9 +582,6 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
     for (int q = 0; q < 4; ++q) acc[j][q] = 0.f;
   uint32_t pfA[3] = {0, 0, 0}, pfB[3] = {0, 0, 0};  // MXFP4: prefetched scale words
   int64_t pf_o = -1;                                // ... of the chunk at row-A offset pf_o
-  // the unscaled operand values in registers: bf16(level) (NF4) or e2m1 (MXFP4)
-  Lut lreg;
-  lut_build<FMT>(lreg, 1.0f, 127u);
 
   for (int64_t i = 0;; ++i) {
     const int s = int(i % kStages);
@@ -646,8 +635,8 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
         mx_words(scales, n, oB + 8, pfB);
       }
     }
-    if (f.ntok > 8) consume_stage<FMT, 2, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, lreg, acc);
-    else consume_stage<FMT, 1, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, lreg, acc);
+    if (f.ntok > 8) consume_stage<FMT, 2, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
+    else consume_stage<FMT, 1, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
     mbar_arrive(&empty[s]);  // this lane's reads of the stage are done
     if (!f.last) continue;
 
