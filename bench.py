@@ -58,6 +58,9 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload table of the default line")
+    ap.add_argument("--mx", choices=["off", "exact", "e4m3"], default="off",
+                    help="MXFP4 workloads: run the block-scaled FP4 MMA path on the prepared stacks, with the "
+                         "bf16-exact two-term activations or one e4m3 term (OCP MXFP8)")
     ap.add_argument("--reps", type=int, default=PER_CONFIG_REPS,
                     help="repetitions per median in the per-workload table")
     ap.add_argument("--op", choices=["forward", "dgrad", "int4"], default="forward",
@@ -188,14 +191,18 @@ def _roofline(path, kernel, kb, dur_s, wl, ids, key, hbm, bf16, bf16_sus, peak_s
     """Roofline of the dominant kernel: HBM bytes for the small-M layer kernel,
     dense bf16 FLOPs for a tcgen05 projection (burst peak: the kernel runs for
     milliseconds, not the seconds the sustained figure needs)."""
-    if path == 2 and kernel in ("gate_up", "down"):
+    if path in (2, 4) and kernel in ("gate_up", "down", "quant_h+down"):
         R = ids.size
         flops = 2.0 * R * (2 * wl.I * wl.H if kernel == "gate_up" else wl.H * wl.I)
         achieved = flops / dur_s / 1e12
-        return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": bf16,
-                "unit": "TFLOP/s", "frac": achieved / bf16, "peak_source": peak_src + " (burst)",
-                "peak_sustained": bf16_sus, "traffic": _traffic(key, kernel),
-                "algorithmic_flops": flops}
+        # the block-scaled FP4 MMA runs at the f8f6f4 rate: the measured bf16
+        # peak times 2, the nominal ratio of the dense fp8 and bf16 peaks
+        peak = bf16 * (2.0 if path == 4 else 1.0)
+        return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": peak_src + (" bf16 burst x 2 (f8f6f4)" if path == 4 else " (burst)"),
+                "peak_sustained": bf16_sus * (2.0 if path == 4 else 1.0),
+                "traffic": _traffic(key, kernel) if path == 2 else None, "algorithmic_flops": flops}
     achieved = kb[kernel] / dur_s / 1e9
     return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "peak_source": peak_src, "traffic": _traffic(key, kernel),
@@ -217,7 +224,7 @@ def kernel_bytes(wl, T, ids):
             "layer": active * 3 * wl.H * wl.I * bpw + 4 * T * wl.H + 8 * R}
 
 
-def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
+def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None, flags=0):
     import torch
     from bit_grouped_moe_e4b_b200 import e4b, synth
 
@@ -238,7 +245,7 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
             dist.barrier()
 
     for _ in range(warmup):
-        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws)
+        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws, flags)
     torch.cuda.synchronize()
     status = e4b.e4b_read_device_status(ws)
     if status != 0:
@@ -263,12 +270,12 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
     # from a second loop with the library's events between its launches
     t0.record(stream)
     for i in range(steps):
-        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws)
+        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws, flags)
     t1.record(stream)
     torch.cuda.synchronize()
     for i in range(steps):
         e4b.e4b_set_timing_events(ev[i])
-        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws)
+        e4b.e4b_moe_forward(layer, x, ids, gates, y, ws, flags)
     torch.cuda.synchronize()
     e4b.e4b_set_timing_events(None)
     clk = clocks.stop()
@@ -277,6 +284,8 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
     path = e4b.e4b_last_path()
     if path == e4b.E4B_PATH_GEMV:  # routing, the fused small-M layer kernel, the combine
         spans = (("route", 0, 1), ("smallm_layer", 1, 3), ("combine", 3, 4))
+    elif path == e4b.E4B_PATH_TCGEN05_MX:  # routing + x terms, gate_up, h terms + down, combine
+        spans = (("route+quant_x", 0, 1), ("gate_up", 1, 2), ("quant_h+down", 2, 3), ("combine", 3, 4))
     else:
         # routing (+ the staging copy of the routed rows when the workspace
         # holds it), the two tcgen05 projections, the bf16 conversion
@@ -298,7 +307,7 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
     for _ in range(warmup):
         x_d.copy_(x_pin, non_blocking=True)
         e4b.e4b_moe_forward(layer, x_d, ids_d.copy_(ids_pin, non_blocking=True),
-                            g_d.copy_(g_pin, non_blocking=True), y, ws)
+                            g_d.copy_(g_pin, non_blocking=True), y, ws, flags)
         y_pin.copy_(y, non_blocking=True)
     barrier()
     torch.cuda.synchronize()
@@ -309,7 +318,7 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None):
         x_d.copy_(x_pin, non_blocking=True)
         ids_d.copy_(ids_pin, non_blocking=True)
         g_d.copy_(g_pin, non_blocking=True)
-        e4b.e4b_moe_forward(layer, x_d, ids_d, g_d, y, ws)
+        e4b.e4b_moe_forward(layer, x_d, ids_d, g_d, y, ws, flags)
         y_pin.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -864,7 +873,14 @@ def main():
             layers.clear()
             torch.cuda.empty_cache()
             layers[wl_i.layer] = build_layer(wl_i, dev)
-        r = run_gpu(wl_i, T_i, args.steps, args.warmup, rank, world, dist, layer=layers[wl_i.layer])
+        flags = 0
+        lay = layers[wl_i.layer]
+        if args.mx != "off" and wl_i.fmt == "mxfp4":
+            from bit_grouped_moe_e4b_b200 import e4b as _e4b
+
+            lay = lay.prepare_mx()
+            flags = _e4b.FLAG_FORCE_TCGEN05 | (_e4b.FLAG_MX_ACT_E4M3 if args.mx == "e4m3" else 0)
+        r = run_gpu(wl_i, T_i, args.steps, args.warmup, rank, world, dist, layer=lay, flags=flags)
         kb = kernel_bytes(wl_i, T_i, r["ids"])
         dominant = max((k for k in r["phases"] if not k.startswith("route") and not k.startswith("_")),
                        key=lambda k: r["phases"][k])
@@ -880,7 +896,9 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl_i.name, "T": T_i, "format": wl_i.fmt, "E": wl_i.E,
                        "H": wl_i.H, "I": wl_i.I, "top_k": wl_i.top_k,
-                       "active_experts": kb["active_experts"], "path": ["none", "gemv", "tcgen05"][r["path"]],
+                       "active_experts": kb["active_experts"],
+                       "path": ["none", "gemv", "tcgen05", "int4", "tcgen05_mx"][r["path"]]
+                       + ("_e4m3" if args.mx == "e4m3" and r["path"] == 4 else ""),
                        "weights": "N(0,0.02) fp32 packed on the GPU by e4b_quantize_*",
                        "l2": "no flush: packed weights of the active experts "
                              f"({kb['packed_bytes'] / 2 ** 20:.0f} MiB) exceed the 126 MB L2",
