@@ -113,6 +113,11 @@ cudaError_t launch_smallm_layer(const SmallMLayer& L, cudaStream_t st, int sms);
 // dependent of launch_smallm_layer).
 cudaError_t launch_smallm_combine(const SmallMLayer& L, cudaStream_t st, int sms);
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms);
+// The SM-pair (cta_group::2) form of the large-M projection (csrc/tc_pair.cu):
+// forward epilogues on contiguous activation rows; launch_tc_gemm takes it
+// whenever tc_pair_supported says so.
+bool tc_pair_supported(const GemmProblem& p);
+cudaError_t launch_tc_pair(const GemmProblem& p, cudaStream_t st, int sms);
 cudaError_t launch_finalize(const float* acc, int64_t n, uint16_t* y, cudaStream_t st, int sms);
 
 // The int4-b32 decode GEMV (csrc/int4.cu): one token against n_slots routed

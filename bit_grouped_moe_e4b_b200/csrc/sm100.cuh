@@ -293,6 +293,98 @@ E4B_DEV uint64_t chunk512_desc(uint32_t saddr) {
   return d;                       // layout type 0: no swizzle
 }
 
+// ------------------------------------------------- CTA pairs (cta_group::2)
+// A cluster of two CTAs on two SMs issues one MMA of M = 256: each CTA holds
+// 128 rows of A and half of B's N rows in its own shared memory (same
+// offsets), and each CTA's TMEM receives its 128 rows of D over all N.
+// Every tcgen05 instruction of a kernel that uses pairs names cta_group::2.
+E4B_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs; orders the shared-memory writes before it
+// (barrier initialisation included) with the reads after it, cluster-wide.
+E4B_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The shared::cluster address of the same shared-memory offset in CTA `rank`.
+E4B_DEV uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier given by its cluster address (possibly the other
+// CTA's). Default semantics (release at CTA scope): a release at cluster scope
+// costs a fence of ~1000 clocks per arrival, and what the arrival publishes
+// here is shared memory the pair MMA reads through the async proxy, which the
+// writer has already made visible with fence.proxy.async.
+E4B_DEV void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// try_wait with acquire at cluster scope: for barriers completed by the other
+// CTA of the pair (remote arrivals, or the pair MMA's commits).
+E4B_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+E4B_DEV bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, uint32_t limit,
+                                       const volatile int* abort) {
+  uint32_t polls = 0;
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (polls >= limit) return false;
+    if (abort && *abort) return false;
+    ++polls;
+    if (polls > 64) __nanosleep(64);
+  }
+}
+
+E4B_DEV void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+E4B_DEV void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+E4B_DEV void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A * B^T over the pair, kind::f16: issued by the even CTA only.
+E4B_DEV void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// One arrival on the mbarrier at this offset in both CTAs of the pair once
+// the pair MMAs issued so far by this thread have completed.
+E4B_DEV void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(uint16_t(3))
+      : "memory");
+}
+
 // ----------------------------------------------------------------- e4m3
 // Two fp32 values -> two OCP E4M3 bytes, round to nearest even, magnitudes
 // beyond 448 saturated to 448: the low byte holds lo, the high byte hi.

@@ -671,6 +671,7 @@ cudaError_t launch_t(const GemmProblem& p, cudaStream_t st, int sms) {
 
 cudaError_t launch_tc_gemm(const GemmProblem& p, cudaStream_t st, int sms) {
   if (p.E > kMaxE) return cudaErrorInvalidValue;
+  if (tc_pair_supported(p)) return launch_tc_pair(p, st, sms);
   if (p.epilogue == kEpiDgrad) {
     if (p.row_slot) return cudaErrorInvalidValue;  // dy rows are expert-ordered
     return p.fmt == E4B_FMT_NF4 ? launch_t<E4B_FMT_NF4, kEpiDgrad>(p, st, sms)

@@ -28,6 +28,7 @@ FLAG_TEST_TIMEOUT = 0x4
 FLAG_IDS_READY = 0x10  # e4b_gemv_int4_b32: ids and gates not written by the preceding work on the stream
 FLAG_MX_ACT_E4M3 = 0x20  # native MXFP4 path: one e4m3 term per activation (OCP MXFP8 rule)
 FLAG_MX_DECODE = 0x40  # MXFP4 with prepared stacks: the decode-to-bf16 tcgen05 path anyway
+FLAG_TC_SINGLE_SM = 0x80  # large-M projections on the one-SM tcgen05 kernel instead of SM pairs
 FLAG_NF4_PRODUCT_DECODE = 0x8  # small-M NF4: bf16(level * absmax) operands (the default is bf16(level), absmax after the block MMA)
 STATUS_NAMES = {
     0: "E4B_OK", 1: "E4B_ERR_INVALID_ARG", 2: "E4B_ERR_UNSUPPORTED",

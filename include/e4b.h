@@ -109,6 +109,11 @@ typedef enum {
 /* MXFP4 layers with prepared stacks: take the decode-to-bf16 tcgen05 path
  * anyway on large-M shapes (for comparisons). */
 #define E4B_FLAG_MX_DECODE 0x40u
+/* Large-M tcgen05 projections: run on the one-SM kernel (M = 128 weight rows
+ * per MMA) instead of SM pairs (tcgen05.mma.cta_group::2, M = 256 over two
+ * SMs of a cluster); for comparisons. Gathered activation rows and the input
+ * gradients always take the one-SM kernel. */
+#define E4B_FLAG_TC_SINGLE_SM 0x80u
 
 /* NF4 block size (weights per absmax) and MXFP4 block size (weights per scale). */
 #define E4B_NF4_BLOCK 64

@@ -15,6 +15,8 @@ pytestmark = pytest.mark.gpu
 
 PATHS = {"gemv": e4b.FLAG_FORCE_GEMV, "tcgen05": e4b.FLAG_FORCE_TCGEN05,
          "tcgen05_gather": e4b.FLAG_FORCE_TCGEN05,
+         # the one-SM tcgen05 kernel on staged rows ("tcgen05" runs on SM pairs)
+         "tcgen05_1sm": e4b.FLAG_FORCE_TCGEN05 | e4b.FLAG_TC_SINGLE_SM,
          # small-M with the NF4 product decode (the tcgen05 path's operands)
          "gemv_product": e4b.FLAG_FORCE_GEMV | e4b.FLAG_NF4_PRODUCT_DECODE}
 
@@ -67,7 +69,7 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather", "tcgen05_1sm"])
 @pytest.mark.parametrize("fmt,E,H,I,T,k", SHAPES)
 def test_ragged_shapes(fmt, E, H, I, T, k, path):
     layer, ref = small_layer(fmt, E, H, I, seed=E * 100 + H)
@@ -83,7 +85,7 @@ def test_ragged_shapes(fmt, E, H, I, T, k, path):
 _many = {}
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather", "tcgen05_1sm"])
 def test_many_tiles_per_cta(path):
     # 64 experts x 4 weight-row tiles per projection = 256 tcgen05 tiles, more
     # than one per SM, with 8 k-blocks each: the persistent kernels walk
@@ -104,7 +106,7 @@ def test_many_tiles_per_cta(path):
     assert_close(y, _many[key], f"{fmt} {E}x{H}x{I} T={T} {path}", min_rms=LAYER_MIN_RMS)
 
 
-@pytest.mark.parametrize("path", ["gemv", "gemv_product", "tcgen05"])
+@pytest.mark.parametrize("path", ["gemv", "gemv_product", "tcgen05", "tcgen05_1sm"])
 @pytest.mark.parametrize("fmt,E,H,I,T,k", [("nf4", 3, 256, 320, 40, 2), ("mxfp4", 3, 288, 224, 40, 2),
                                            ("mxfp4", 2, 96, 160, 9, 1)])
 def test_block_scales_and_large_outputs(fmt, E, H, I, T, k, path):
@@ -137,7 +139,7 @@ EDGE = {
 }
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather", "tcgen05_1sm"])
 @pytest.mark.parametrize("case", list(EDGE))
 def test_degenerate_routing(case, path):
     E, H, I = 4, 128, 256
@@ -153,7 +155,7 @@ def test_degenerate_routing(case, path):
     assert_close(y, oracle_layer("nf4", x, ids, gates, ref, E, H, I), f"{case} {path}", min_rms=LAYER_MIN_RMS)
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather", "tcgen05_1sm"])
 def test_bad_expert_ids_drop_only_their_slots(path):
     E, H, I, T = 4, 128, 128, 6
     layer, ref = small_layer("nf4", E, H, I, seed=11)
@@ -170,7 +172,7 @@ def test_bad_expert_ids_drop_only_their_slots(path):
     assert_close(y, oracle_layer("nf4", x, ids2, g2, ref, E, H, I), "bad ids", min_rms=LAYER_MIN_RMS)
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_1sm"])
 def test_bounded_wait_reports_timeout_and_returns(path):
     # the test flag makes the kernels' bounded waits give up at once: the
     # kernel must record E4B_ERR_DEVICE_TIMEOUT and return (no hang, no trap)
@@ -211,7 +213,7 @@ def test_grouped_gemm_store_epilogue():
         assert_close(out.float().cpu().numpy(), want, f"store flags={flags}")
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather", "tcgen05_1sm"])
 def test_combine_is_deterministic(path):
     # every path writes each routed row's output (small-M: each K slice's
     # partial sum) once and sums every token's rows in a fixed order:

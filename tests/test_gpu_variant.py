@@ -19,7 +19,8 @@ from gpu_util import assert_close, last_nf4_decode, run_layer, small_layer
 pytestmark = pytest.mark.gpu
 
 PATHS = {"gemv": e4b.FLAG_FORCE_GEMV, "tcgen05": e4b.FLAG_FORCE_TCGEN05,
-         "tcgen05_gather": e4b.FLAG_FORCE_TCGEN05}
+         "tcgen05_gather": e4b.FLAG_FORCE_TCGEN05,
+         "tcgen05_1sm": e4b.FLAG_FORCE_TCGEN05 | e4b.FLAG_TC_SINGLE_SM}
 ALPHA, LIMIT = 1.702, 7.0
 
 
@@ -50,7 +51,7 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_gather", "tcgen05_1sm"])
 @pytest.mark.parametrize("layout", ["halves", "interleaved"])
 @pytest.mark.parametrize("fmt,E,H,I,T,k", SHAPES)
 def test_clamped_glu_with_biases(fmt, E, H, I, T, k, layout, path):
@@ -68,7 +69,7 @@ def test_clamped_glu_with_biases(fmt, E, H, I, T, k, layout, path):
     assert_close(y, y_ref, f"{fmt} {layout} {path}")
 
 
-@pytest.mark.parametrize("path", ["gemv", "tcgen05"])
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_1sm"])
 @pytest.mark.parametrize("which", ["interleaved_swiglu", "halves_biases_only", "down_bias_only"])
 def test_variant_parts(which, path):
     # each part of the variant alone: the interleaved rows with the plain
@@ -123,7 +124,8 @@ def test_invalid_variant_arguments():
         run_layer(vl, x, ids, gates)
 
 
-@pytest.mark.parametrize("flags", [e4b.FLAG_FORCE_GEMV, e4b.FLAG_FORCE_TCGEN05])
+@pytest.mark.parametrize("flags", [e4b.FLAG_FORCE_GEMV, e4b.FLAG_FORCE_TCGEN05,
+                                   e4b.FLAG_FORCE_TCGEN05 | e4b.FLAG_TC_SINGLE_SM])
 @pytest.mark.parametrize("layout", ["halves", "interleaved"])
 def test_grouped_gemm_gated_epilogue(layout, flags):
     # e4b_grouped_gemm alone: the gate_up projection with biases and the
@@ -155,7 +157,8 @@ def test_grouped_gemm_gated_epilogue(layout, flags):
     assert_close(out.float().cpu().numpy(), want, f"gated epilogue {layout} flags={flags}")
 
 
-@pytest.mark.parametrize("flags", [e4b.FLAG_FORCE_GEMV, e4b.FLAG_FORCE_TCGEN05])
+@pytest.mark.parametrize("flags", [e4b.FLAG_FORCE_GEMV, e4b.FLAG_FORCE_TCGEN05,
+                                   e4b.FLAG_FORCE_TCGEN05 | e4b.FLAG_TC_SINGLE_SM])
 def test_grouped_gemm_store_and_combine_bias(flags):
     fmt, E, N, K = "nf4", 2, 96, 192
     rng = np.random.default_rng(21)
