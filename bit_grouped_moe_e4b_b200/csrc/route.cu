@@ -17,6 +17,7 @@ namespace e4b {
 
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kBatch = 8;  // 32-slot pieces whose ids are loaded together
 
 __global__ void __launch_bounds__(kRouteThreads, 1)
 route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __restrict__ counts,
@@ -51,17 +52,28 @@ route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __r
   const int32_t end = min(R, beg + chunk);
   int32_t* my = wcnt + warp * E;
 
-  // pass 1: per-warp histogram
-  for (int32_t s0 = beg; s0 < end; s0 += 32) {
-    const int32_t s = s0 + lane;
-    const bool in = s < end;
-    int32_t e = in ? ids[s] : -1;
-    const bool ok = in && e >= 0 && e < E;
-    if (in && !ok) atomicAdd(&s_bad, 1);
-    if (!ok) e = -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    const int leader = __ffs(peers) - 1;
-    if (ok && lane == leader) my[e] += __popc(peers);
+  // pass 1: per-warp histogram (the ids of kBatch pieces are loaded together
+  // so that their latencies overlap)
+  for (int32_t b0 = beg; b0 < end; b0 += 32 * kBatch) {
+    int32_t ev[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int32_t s = b0 + 32 * u + lane;
+      ev[u] = s < end ? __ldg(ids + s) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int32_t s = b0 + 32 * u + lane;
+      if (b0 + 32 * u >= end) break;  // uniform
+      const bool in = s < end;
+      int32_t e = ev[u];
+      const bool ok = in && e >= 0 && e < E;
+      if (in && !ok) atomicAdd(&s_bad, 1);
+      if (!ok) e = -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const int leader = __ffs(peers) - 1;
+      if (ok && lane == leader) my[e] += __popc(peers);
+    }
   }
   __syncthreads();
 
@@ -107,24 +119,34 @@ route_kernel(const int32_t* __restrict__ ids, int32_t R, int32_t E, int32_t* __r
     if (tid == kRouteThreads - 1) active[0] = scan[tid];
   }
 
-  // pass 2: stable scatter
-  for (int32_t s0 = beg; s0 < end; s0 += 32) {
-    const int32_t s = s0 + lane;
-    const bool in = s < end;
-    int32_t e = in ? ids[s] : -1;
-    const bool ok = in && e >= 0 && e < E;
-    if (!ok) e = -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    const int leader = __ffs(peers) - 1;
-    int32_t pos = -1;
-    if (ok) {
-      pos = my[e] + __popc(peers & ((1u << lane) - 1u));
-      perm[pos] = s;
+  // pass 2: stable scatter, pieces in slot order
+  for (int32_t b0 = beg; b0 < end; b0 += 32 * kBatch) {
+    int32_t ev[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int32_t s = b0 + 32 * u + lane;
+      ev[u] = s < end ? __ldg(ids + s) : 0;
     }
-    if (in) inv[s] = pos;
-    __syncwarp();
-    if (ok && lane == leader) my[e] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int32_t s = b0 + 32 * u + lane;
+      if (b0 + 32 * u >= end) break;  // uniform
+      const bool in = s < end;
+      int32_t e = ev[u];
+      const bool ok = in && e >= 0 && e < E;
+      if (!ok) e = -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const int leader = __ffs(peers) - 1;
+      int32_t pos = -1;
+      if (ok) {
+        pos = my[e] + __popc(peers & ((1u << lane) - 1u));
+        perm[pos] = s;
+      }
+      if (in) inv[s] = pos;
+      __syncwarp();
+      if (ok && lane == leader) my[e] += __popc(peers);
+      __syncwarp();
+    }
   }
   __syncthreads();
   if (tid == 0 && s_bad) {
