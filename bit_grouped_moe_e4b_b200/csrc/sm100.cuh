@@ -340,6 +340,19 @@ E4B_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase, acquire at cluster scope.
+E4B_DEV bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 E4B_DEV bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, uint32_t limit,
                                        const volatile int* abort) {
   uint32_t polls = 0;
