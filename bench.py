@@ -297,7 +297,9 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None, flags=0):
     else:
         # routing (+ the staging copy of the routed rows when the workspace
         # holds it), the two tcgen05 projections, the bf16 conversion
-        first = "route+stage" if launches_per_step == 5 else "route"
+        # 5 or 6 launches with the staging copy (routing takes 2 launches from
+        # 16384 routed rows), 4 without
+        first = "route+stage" if launches_per_step >= 5 else "route"
         spans = ((first, 0, 1), ("gate_up", 1, 2), ("down", 2, 3), ("combine", 3, 4))
     phases = {name: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(steps)]))
               for name, a, b in spans}
@@ -421,7 +423,7 @@ def per_config_entry(wl, T, layer, reps, flush, hbm, bf16, peak_src, flags=0, va
         # routing + x split into e4m3 terms, gate_up, h split + down, combine
         spans = (("route+quant_x", 0, 1), ("gate_up", 1, 2), ("quant_h+down", 2, 3), ("combine", 3, 4))
     else:
-        spans = (("route+stage" if launches == 5 else "route", 0, 1), ("gate_up", 1, 2), ("down", 2, 3),
+        spans = (("route+stage" if launches >= 5 else "route", 0, 1), ("gate_up", 1, 2), ("down", 2, 3),
                  ("combine", 3, 4))
     phases = {n: float(np.median([r[a].elapsed_time(r[b]) for r in evs])) for n, a, b in spans}
     kb = kernel_bytes(wl, T, ids_h)

@@ -235,7 +235,8 @@ e4b_status e4b_dequantize(int32_t fmt, const uint8_t* codes, const void* scales,
 
 e4b_status e4b_route_workspace_size(int64_t T, int32_t top_k, int32_t E, size_t* bytes) {
   if (!bytes || T < 0 || top_k <= 0 || E <= 0) return E4B_ERR_INVALID_ARG;
-  *bytes = kStatusBytes;
+  const int64_t R = T * int64_t(top_k);
+  *bytes = kStatusBytes + (E <= 1024 && R < (int64_t(1) << 31) ? route_scratch_bytes(int32_t(R), E) : 0);
   return E4B_OK;
 }
 
@@ -247,10 +248,14 @@ e4b_status e4b_route(const int32_t* ids, int64_t T, int32_t top_k, int32_t E, in
     return E4B_ERR_INVALID_ARG;
   if (E > 1024 || T * int64_t(top_k) >= (int64_t(1) << 31)) return E4B_ERR_UNSUPPORTED;
   if (ws_bytes < size_t(kStatusBytes)) return E4B_ERR_WORKSPACE_TOO_SMALL;
-  g_last_launches = 1;
-  return cuda_status(launch_route(ids, int32_t(T * top_k), E, counts, offsets, perm, inv_perm,
-                                  nullptr, static_cast<int32_t*>(ws),
-                                  static_cast<cudaStream_t>(stream)));
+  int launches = 1;
+  // the status words, then (large batches) the many-CTA pass's scratch
+  const e4b_status st = cuda_status(launch_route(
+      ids, int32_t(T * top_k), E, counts, offsets, perm, inv_perm, nullptr, static_cast<int32_t*>(ws),
+      static_cast<cudaStream_t>(stream), nullptr, 0,
+      reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kStatusBytes), ws_bytes - kStatusBytes, &launches));
+  g_last_launches = launches;
+  return st;
 }
 
 e4b_status e4b_grouped_gemm(const e4b_gemm_args* a, uint32_t flags, void* stream) {
@@ -730,8 +735,12 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
 
   mark(0, s);
   int32_t* sync = reinterpret_cast<int32_t*>(base + L.sync);
+  // the fp32 rows / partial sums region is free until the projections: it
+  // lends the many-CTA routing its scratch
+  int route_launches = 1;
   cudaError_t ce = launch_route(ids, int32_t(R), int32_t(E), counts, offsets, perm, inv, nullptr,
-                                status, s, sync, int32_t(L.nsync));
+                                status, s, sync, int32_t(L.nsync), reinterpret_cast<int32_t*>(acc),
+                                (gemv ? L.small_min : L.large_min) - L.acc, &route_launches);
   if (ce != cudaSuccess) return E4B_ERR_CUDA;
 
   if (gemv) {
@@ -774,12 +783,16 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
     if (ce != cudaSuccess) return E4B_ERR_CUDA;
     mark(4, s);
     g_last_path = E4B_PATH_GEMV;
-    g_last_launches = 3;
+    g_last_launches = 2 + route_launches;
     return E4B_OK;
   }
 
-  if (has_mx(w) && !(flags & E4B_FLAG_MX_DECODE))
-    return moe_forward_mx(w, L, x, T, top_k, perm, offsets, inv, gates, y, base, ws_bytes, status, flags, s);
+  if (has_mx(w) && !(flags & E4B_FLAG_MX_DECODE)) {
+    const e4b_status r =
+        moe_forward_mx(w, L, x, T, top_k, perm, offsets, inv, gates, y, base, ws_bytes, status, flags, s);
+    g_last_launches += route_launches - 1;
+    return r;
+  }
 
   // Large-M: stage the routed rows of x in expert order when the workspace
   // holds the copy (contiguous TMA row tiles), else gather them in the kernel.
@@ -844,7 +857,7 @@ e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t 
   if (ce != cudaSuccess) return E4B_ERR_CUDA;
   mark(4, s);
   g_last_path = gemv ? E4B_PATH_GEMV : E4B_PATH_TCGEN05;
-  g_last_launches = staged ? 5 : 4;
+  g_last_launches = (staged ? 4 : 3) + route_launches;
   return E4B_OK;
 }
 

@@ -18,9 +18,15 @@ cudaError_t launch_dequantize(int fmt, const uint8_t* codes, const void* scales,
 void host_nf4_levels(float* out);
 
 size_t route_smem_bytes(int32_t E);
+// Bytes of scratch the many-CTA routing of R slots over E experts needs (0:
+// R is small enough for the one-CTA pass).
+size_t route_scratch_bytes(int32_t R, int32_t E);
+// The routing pass; with `scratch` (at least route_scratch_bytes) and a large
+// R it runs over many CTAs in two launches (*launches says how many).
 cudaError_t launch_route(const int32_t* ids, int32_t R, int32_t E, int32_t* counts, int64_t* offsets,
                          int32_t* perm, int32_t* inv, int32_t* active, int32_t* status,
-                         cudaStream_t st, int32_t* clear = nullptr, int32_t nclear = 0);
+                         cudaStream_t st, int32_t* clear = nullptr, int32_t nclear = 0,
+                         int32_t* scratch = nullptr, size_t scratch_bytes = 0, int* launches = nullptr);
 // xs[p] = x[perm[p] / top_k] for p < offsets[E] (H % 8 == 0, 16-byte aligned).
 cudaError_t launch_gather_rows(const uint16_t* x, int64_t H, const int32_t* perm, int32_t top_k,
                                const int64_t* offsets, int32_t E, int64_t R_max, uint16_t* xs,

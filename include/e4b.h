@@ -255,7 +255,10 @@ e4b_status e4b_nf4_codebook(float* out_host);
 
 /* ---------------------------------------------------------------- routing */
 
-/* Host: bytes of workspace e4b_route needs for these sizes (always > 0). */
+/* Host: bytes of workspace e4b_route needs for these sizes (always > 0):
+ * the status words, plus, for T*top_k >= 16384 slots, the scratch that lets
+ * the pass run over many CTAs (two launches instead of one; same result). A
+ * workspace of only the status words still routes any size, on one CTA. */
 e4b_status e4b_route_workspace_size(int64_t T, int32_t top_k, int32_t E, size_t* bytes);
 
 /*

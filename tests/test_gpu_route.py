@@ -59,3 +59,53 @@ def test_route_bad_ids_are_dropped_and_reported():
     assert np.all(inv_h[~ok] == -1)
     # after reading, the status word is clear
     assert e4b.e4b_read_device_status(ws) == 0
+
+
+def _route_ws(ids, E, ws_bytes):
+    ids_d = torch.from_numpy(ids).cuda()
+    T, k = ids.shape
+    dev = ids_d.device
+    out = (torch.empty(E, dtype=torch.int32, device=dev), torch.empty(E + 1, dtype=torch.int64, device=dev),
+           torch.empty(T * k, dtype=torch.int32, device=dev), torch.empty(T * k, dtype=torch.int32, device=dev))
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    e4b.e4b_route(ids_d, E, *out, ws)
+    launches = e4b.e4b_last_launch_count()
+    return [o.cpu().numpy() for o in out], e4b.e4b_read_device_status(ws), launches
+
+
+@pytest.mark.parametrize("T,k,E,skew", [(2500, 8, 1024, 0.0), (8192, 8, 128, 0.05), (4097, 4, 32, 0.0),
+                                        (16384, 1, 1, 0.0), (6000, 3, 7, 0.3)])
+def test_route_many_ctas_equals_one_cta_and_oracle(T, k, E, skew):
+    # from 16384 slots a workspace of e4b_route_workspace_size bytes routes
+    # over many CTAs (two launches); a status-only workspace on one CTA
+    rng = np.random.default_rng(T + E)
+    if skew:
+        ids = rng.choice(E, size=(T, k), p=rng.dirichlet(np.full(E, skew))).astype(np.int32)
+    else:
+        ids = rng.integers(0, E, (T, k)).astype(np.int32)
+    full = e4b.e4b_route_workspace_size(T, k, E)
+    assert full > 256
+    many, st_m, l_m = _route_ws(ids, E, full)
+    one, st_o, l_o = _route_ws(ids, E, 256)
+    assert (l_m, l_o) == (2, 1) and st_m == 0 and st_o == 0
+    ref = oracle.route_ref(ids, E)
+    for a, b, r in zip(many, one, ref):
+        assert np.array_equal(a, r) and np.array_equal(b, r)
+
+
+def test_route_many_ctas_bad_ids():
+    rng = np.random.default_rng(17)
+    T, k, E = 9000, 2, 40
+    ids = rng.integers(0, E, (T, k)).astype(np.int32)
+    bad = rng.choice(T * k, 37, replace=False)
+    ids.reshape(-1)[bad[:20]] = -3
+    ids.reshape(-1)[bad[20:]] = E + 5
+    (counts, offsets, perm, inv), status, launches = _route_ws(ids, E, e4b.e4b_route_workspace_size(T, k, E))
+    assert launches == 2 and status == 6   # E4B_ERR_BAD_EXPERT_ID
+    flat = ids.reshape(-1)
+    ok = (flat >= 0) & (flat < E)
+    rc, ro, rp, _ = oracle.route_ref(np.where(ok, flat, 0)[ok].reshape(1, -1), E)
+    assert np.array_equal(counts, rc) and np.array_equal(offsets, ro)
+    assert np.array_equal(perm[:ok.sum()], np.nonzero(ok)[0][rp])
+    assert np.all(inv[~ok] == -1)
+    assert np.array_equal(perm[inv[ok]], np.nonzero(ok)[0])
