@@ -525,7 +525,8 @@ e4b_status e4b_moe_workspace_size(const e4b_moe_weights* w, int64_t T, int32_t t
  * routed row's output (small-M: each 2048-wide K slice's partial sum) is
  * written once and each token's rows are summed in a fixed order, so repeated
  * calls give the same bits. Launches: small-M 3 (routing, the layer kernel,
- * the combine), large-M 5 (4 without the staging copy).
+ * the combine), large-M 5 (4 without the staging copy); from 16384 routed rows
+ * on the large-M paths the routing takes 2 launches instead of 1.
  */
 e4b_status e4b_moe_forward(const e4b_moe_weights* w, const uint16_t* x, int64_t T, int32_t top_k,
                            const int32_t* ids, const float* gates, uint16_t* y, void* ws,
