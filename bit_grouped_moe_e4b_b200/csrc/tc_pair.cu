@@ -45,6 +45,10 @@
 // before TMEM is freed and before either exits, so no remote arrival or MMA
 // read ever targets a CTA that has left.
 //
+// The input gradient (kEpiDgrad, e4b_grouped_dgrad) runs here too: the MMA's
+// M then runs over the weight's columns (each CTA 128 of them, its A tile
+// MN-major as in the one-SM kernel) and its reduction over the weight's rows.
+//
 // gate_up rows in a CTA (SWIGLU): the pair covers features F .. F+127, the
 // CTA of rank r features F + 64r .. F + 64r + 63. Lane quarter q (lanes
 // 32q .. 32q+31) holds features 16q .. 16q+15 of the CTA: gate rows in its
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                const __grid_constant__ CUtensorMap tmap_act, GemmProblem p) {
   constexpr int NMAT = (EPI == E4B_EPI_SWIGLU) ? 2 : 1;
+  constexpr bool DG = EPI == kEpiDgrad;
   using C = PCfg;
   constexpr int CS = C::CS;
   constexpr int S = C::S;
@@ -178,9 +183,13 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   const int64_t N = p.N;
   const int64_t K = p.K;
   const int64_t rows_per_mat = NMAT == 2 ? N / 2 : N;
-  constexpr int64_t TM = NMAT == 2 ? 128 : 256;   // weight rows (features) per pair tile
-  const int64_t MT = (rows_per_mat + TM - 1) / TM;
-  const int KB = int((K + PK - 1) / PK);
+  // dgrad: the MMA's M runs over the weight's columns, its reduction over the
+  // weight's rows
+  const int64_t Mdim = DG ? K : rows_per_mat;
+  const int64_t Kred = DG ? N : K;
+  constexpr int64_t TM = NMAT == 2 ? 128 : 256;   // M rows (features) per pair tile
+  const int64_t MT = (Mdim + TM - 1) / TM;
+  const int KB = int((Kred + PK - 1) / PK);
   const bool il = NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED;
   const uint32_t limit = (p.flags & E4B_FLAG_TEST_TIMEOUT) ? 0u : kWaitPolls;
 
@@ -295,7 +304,11 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           }
           mbar_arrive_expect_tx(&c_full[s], kPCTile);
           uint8_t* dst = smem + C::kC + s * kPCTile;
-          if constexpr (NMAT == 1) {
+          if constexpr (DG) {
+            // 64 weight rows x this CTA's 128 weight columns (64 bytes)
+            tma_load_2d(dst, &tmap_codes, &c_full[s], int32_t((T.mt * TM + int64_t(rank) * 128) / 2),
+                        int32_t(int64_t(T.e) * N + int64_t(kb) * PK));
+          } else if constexpr (NMAT == 1) {
             tma_load_2d(dst, &tmap_codes, &c_full[s], kb * (PK / 2),
                         int32_t(int64_t(T.e) * N + T.mt * TM + int64_t(rank) * 128));
           } else {
@@ -318,7 +331,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   } else if (warp == 1) {
     // ------------------------------------------------------- pair MMA (leader)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_bf16_f32(2 * PM, PN);
+      // dgrad: A is MN-major (bit 15, "transpose A")
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * PM, PN) | (DG ? (1u << 15) : 0u);
       int64_t i = 0;
       bool aborted = false;
       uint64_t* last_bar = nullptr;
@@ -343,9 +357,11 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           const uint32_t abase = smem_u32(smem + C::kA + st * kPATile);
           const uint32_t bbase = smem_u32(smem + C::kB + st * kPBTile);
 #pragma unroll
-          for (int kk = 0; kk < PK / 16; ++kk)
-            mma_bf16_pair(dcol, sw128_kmajor_desc(abase + kk * 32), sw128_kmajor_desc(bbase + kk * 32), idesc,
-                          (kb | kk) ? 1u : 0u);
+          for (int kk = 0; kk < PK / 16; ++kk) {
+            const uint64_t adesc = DG ? sw128_mnmajor_desc(abase + kk * 2048, 8192, 1024)
+                                      : sw128_kmajor_desc(abase + kk * 32);
+            mma_bf16_pair(dcol, adesc, sw128_kmajor_desc(bbase + kk * 32), idesc, (kb | kk) ? 1u : 0u);
+          }
           mma_commit_pair(&empty[st]);
           last_bar = &empty[st];
           last_ph = ph;
@@ -404,6 +420,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const int mat = NMAT == 2 ? ((m >> 4) & 1) : 0;
     const int floc = NMAT == 2 ? ((m >> 5) * 16 + (m & 15)) : m;      // feature within the CTA's 64
     const int crow = NMAT == 2 ? (mat * 64 + floc) : m;                // row of the codes stage
+    // dgrad: weight row dr of the job's 64, columns 64 db .. 64 db + 63 of the CTA's 128
+    const int dr = m & 63, db = m >> 6;
     const uint8_t* scales = static_cast<const uint8_t*>(p.scales);
     const int64_t sstride = FMT == E4B_FMT_NF4 ? (K / 64) * 4 : (K / 32);
 
@@ -413,6 +431,25 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       if (q >= njobs) return 0u;
       const int j = int(q / KB);
       const int kb = int(q % KB);
+      if constexpr (DG) {
+        // the absmax (or the two scale bytes) of weight row kb*64 + dr at the
+        // columns 64 db.. of this CTA; zero past the weight's rows or columns
+        if (j != cached_j) {
+          cached_j = j;
+          const PTile T = sc.tile(pair + j * npairs);
+          const int64_t col0 = T.mt * TM + int64_t(rank) * 128 + 64 * db;
+          srow = col0 < K ? scales + int64_t(T.e) * N * sstride + (FMT == E4B_FMT_NF4 ? (col0 / 64) * 4 : col0 / 32)
+                          : nullptr;
+        }
+        const int64_t wr = int64_t(kb) * PK + dr;
+        if (!srow || wr >= N) return 0u;
+        if constexpr (FMT == E4B_FMT_NF4) {
+          return __float_as_uint(__ldg(reinterpret_cast<const float*>(srow + wr * sstride)));
+        } else {
+          const uint8_t* sb = srow + wr * sstride;
+          return uint32_t(__ldg(sb)) | (uint32_t(__ldg(sb + 1)) << 8);
+        }
+      }
       if (j != cached_j) {
         cached_j = j;
         const PTile T = sc.tile(pair + j * npairs);
@@ -456,7 +493,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           aborted = true;
           break;
         }
-        const uint4* cp = reinterpret_cast<const uint4*>(smem + C::kC + cs * kPCTile + crow * 32);
+        const uint4* cp =
+            reinterpret_cast<const uint4*>(smem + C::kC + cs * kPCTile + (DG ? dr * 64 + db * 32 : crow * 32));
         const uint4 c0 = cp[0];
         const uint4 c1 = cp[1];
         // the slot's next fill is a TMA write (async proxy)
@@ -470,8 +508,12 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           break;
         }
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const int sw = m & 7;
-        uint8_t* arow = smem + C::kA + st * kPATile + m * 128;
+        // K-major: the 128-byte row m of the tile. dgrad, MN-major: the
+        // 128-byte row of K index dr (8-row atoms of 1024 bytes) in the atom
+        // column db (8 KB apart); the same 128B swizzle by row within the atom.
+        const int sw = DG ? (dr & 7) : (m & 7);
+        uint8_t* arow = smem + C::kA + st * kPATile +
+                        (DG ? db * 8192 + (dr >> 3) * 1024 + (dr & 7) * 128 : m * 128);
         Lut L;
         lut_build<FMT>(L, __uint_as_float(cur), cur & 0xFFu);
 #pragma unroll
@@ -559,8 +601,8 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
       } else {
         const int64_t n = T.mt * TM + int64_t(rank) * 128 + q * 32 + lane;
-        const bool nvalid = n < rows_per_mat;
-        const float b0 = (p.bias && nvalid) ? p.bias[int64_t(T.e) * N + n] : 0.f;
+        const bool nvalid = n < Mdim;
+        const float b0 = (!DG && p.bias && nvalid) ? p.bias[int64_t(T.e) * N + n] : 0.f;
         for (int cc = 0; cc < PN / 16; ++cc) {
           const int64_t pbase = T.p0 + cc * 16;
           if (pbase >= T.p1) break;  // uniform
@@ -573,7 +615,7 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
             const int64_t pr = pbase + t;
             if (pr >= T.p1) break;
             const float gv = __uint_as_float(g[t]) + b0;
-            if constexpr (EPI == E4B_EPI_STORE) {
+            if constexpr (EPI == E4B_EPI_STORE || DG) {
               static_cast<uint16_t*>(p.out)[pr * p.ldo + n] = to_bf16_bits(gv);
             } else if constexpr (EPI == kEpiGatedRows) {
               static_cast<float*>(p.out)[pr * p.ldo + n] = s_g[cc * 16 + t] * gv;
@@ -623,6 +665,7 @@ EncodeTiledFn pair_encode_fn() {
 template <int FMT, int EPI>
 cudaError_t launch_pair_t(const GemmProblem& p, cudaStream_t st, int sms) {
   constexpr int NMAT = (EPI == E4B_EPI_SWIGLU) ? 2 : 1;
+  constexpr bool DG = EPI == kEpiDgrad;
   using C = PCfg;
   EncodeTiledFn enc = pair_encode_fn();
   if (!enc) return cudaErrorInitializationError;
@@ -630,7 +673,16 @@ cudaError_t launch_pair_t(const GemmProblem& p, cudaStream_t st, int sms) {
   // or of 64 gate and 64 up rows (interleaved rows: the 3-D view [E*I, 2, K/2]).
   CUtensorMap tmap_codes;
   CUresult cr;
-  if (NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED) {
+  if (DG) {
+    // boxes of 64 weight rows x 128 weight columns (64 bytes)
+    const cuuint64_t gdim[2] = {cuuint64_t(p.K / 2), cuuint64_t(int64_t(p.E) * p.N)};
+    const cuuint64_t gstride[1] = {cuuint64_t(p.K / 2)};
+    const cuuint32_t box[2] = {PM / 2, PK};
+    const cuuint32_t estride[2] = {1, 1};
+    cr = enc(&tmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p.codes), gdim, gstride, box,
+             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else if (NMAT == 2 && p.layout == E4B_GATE_UP_INTERLEAVED) {
     const cuuint64_t gdim[3] = {cuuint64_t(p.K / 2), 2, cuuint64_t(int64_t(p.E) * (p.N / 2))};
     const cuuint64_t gstride[2] = {cuuint64_t(p.K / 2), cuuint64_t(p.K)};
     const cuuint32_t box[3] = {PK / 2, 1, 64};
@@ -648,10 +700,11 @@ cudaError_t launch_pair_t(const GemmProblem& p, cudaStream_t st, int sms) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  // Activations [R_max, K] bf16 (row stride lda), 128-row boxes, 128B swizzle.
+  // Activations [R_max, K] bf16 (row stride lda; dgrad: dy [R_max, N]),
+  // 128-row boxes, 128B swizzle.
   CUtensorMap tmap_act;
   {
-    const cuuint64_t gdim[2] = {cuuint64_t(p.K), cuuint64_t(p.R_max)};
+    const cuuint64_t gdim[2] = {cuuint64_t(DG ? p.N : p.K), cuuint64_t(p.R_max)};
     const cuuint64_t gstride[1] = {cuuint64_t(p.lda) * 2};
     const cuuint32_t box[2] = {PK, PN / 2};
     const cuuint32_t estride[2] = {1, 1};
@@ -692,7 +745,7 @@ cudaError_t launch_pair_t(const GemmProblem& p, cudaStream_t st, int sms) {
   }
   const int64_t rows_per_mat = NMAT == 2 ? p.N / 2 : p.N;
   const int64_t TM = NMAT == 2 ? 128 : 256;
-  const int64_t MT = (rows_per_mat + TM - 1) / TM;
+  const int64_t MT = ((DG ? p.K : rows_per_mat) + TM - 1) / TM;
   const int64_t max_tiles = MT * ((p.R_max + PN - 1) / PN + p.E);
   int np = int(max_tiles < max_pairs ? max_tiles : max_pairs);
   if (np < 1) np = 1;
@@ -703,13 +756,15 @@ cudaError_t launch_pair_t(const GemmProblem& p, cudaStream_t st, int sms) {
 }  // namespace
 
 bool tc_pair_supported(const GemmProblem& p) {
-  // contiguous activation rows (the gathered form stays on the one-SM kernel),
-  // forward epilogues only
-  return p.row_slot == nullptr && p.epilogue != kEpiDgrad && p.E <= kPMaxE && (p.flags & E4B_FLAG_TC_SINGLE_SM) == 0;
+  // contiguous activation rows (the gathered form stays on the one-SM kernel)
+  return p.row_slot == nullptr && p.E <= kPMaxE && (p.flags & E4B_FLAG_TC_SINGLE_SM) == 0;
 }
 
 cudaError_t launch_tc_pair(const GemmProblem& p, cudaStream_t st, int sms) {
   if (!tc_pair_supported(p)) return cudaErrorInvalidValue;
+  if (p.epilogue == kEpiDgrad)
+    return p.fmt == E4B_FMT_NF4 ? launch_pair_t<E4B_FMT_NF4, kEpiDgrad>(p, st, sms)
+                                : launch_pair_t<E4B_FMT_MXFP4, kEpiDgrad>(p, st, sms);
   if (p.epilogue == kEpiGatedRows)
     return p.fmt == E4B_FMT_NF4 ? launch_pair_t<E4B_FMT_NF4, kEpiGatedRows>(p, st, sms)
                                 : launch_pair_t<E4B_FMT_MXFP4, kEpiGatedRows>(p, st, sms);

@@ -109,10 +109,10 @@ typedef enum {
 /* MXFP4 layers with prepared stacks: take the decode-to-bf16 tcgen05 path
  * anyway on large-M shapes (for comparisons). */
 #define E4B_FLAG_MX_DECODE 0x40u
-/* Large-M tcgen05 projections: run on the one-SM kernel (M = 128 weight rows
- * per MMA) instead of SM pairs (tcgen05.mma.cta_group::2, M = 256 over two
- * SMs of a cluster); for comparisons. Gathered activation rows and the input
- * gradients always take the one-SM kernel. */
+/* Large-M tcgen05 projections and e4b_grouped_dgrad: run on the one-SM
+ * kernel (M = 128 weight rows per MMA) instead of SM pairs
+ * (tcgen05.mma.cta_group::2, M = 256 over two SMs of a cluster); for
+ * comparisons. Gathered activation rows always take the one-SM kernel. */
 #define E4B_FLAG_TC_SINGLE_SM 0x80u
 
 /* NF4 block size (weights per absmax) and MXFP4 block size (weights per scale). */
@@ -337,8 +337,9 @@ e4b_status e4b_grouped_gemm(const e4b_gemm_args* args, uint32_t flags, void* str
  * p < offsets[e+1]):  dx[p] = dy[p] . W_e  (the contraction over the weight's
  * rows), fp32 accumulation, bf16 output. W_e is decoded as in e4b_grouped_gemm
  * (NF4 bf16_rne(fp32(level * absmax)), MXFP4 exact); no bf16 weight tensor is
- * stored. Runs on the tcgen05 path (E <= 256); flags: 0 (E4B_FLAG_FORCE_GEMV
- * returns E4B_ERR_UNSUPPORTED). Shapes: K % 64 == 0 (NF4) or K % 32 == 0
+ * stored. Runs on the tcgen05 path (E <= 256), on SM pairs; flags: 0 or
+ * E4B_FLAG_TC_SINGLE_SM (the one-SM kernel; E4B_FLAG_FORCE_GEMV returns
+ * E4B_ERR_UNSUPPORTED). Shapes: K % 64 == 0 (NF4) or K % 32 == 0
  * (MXFP4); N any. dy, codes, dx 16-byte aligned; ld_dy >= N and ld_dx >= K,
  * both multiples of 8. Rows p >= offsets[E] of dx are not written.
  */

@@ -33,8 +33,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("flags", [0, e4b.FLAG_TC_SINGLE_SM], ids=["sm_pairs", "one_sm"])
 @pytest.mark.parametrize("fmt,E,N,K,counts", CASES)
-def test_dgrad_matches_oracle(fmt, E, N, K, counts):
+def test_dgrad_matches_oracle(fmt, E, N, K, counts, flags):
     codes, scales, rc, rs = _stack(fmt, E, N, K, seed=N + K)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
     R = int(offsets[-1])
@@ -42,7 +43,7 @@ def test_dgrad_matches_oracle(fmt, E, N, K, counts):
     dy = torch.from_numpy(rng.standard_normal((R + 3, N)).astype(np.float32)).to(torch.bfloat16)
     dx = torch.full((R + 3, K), 7.0, dtype=torch.bfloat16, device="cuda")
     e4b.e4b_grouped_dgrad(fmt, codes, scales, dy.cuda(), torch.from_numpy(offsets).cuda(), dx, E=E, N=N, K=K,
-                          R_max=R)
+                          R_max=R, flags=flags)
     torch.cuda.synchronize()
     assert e4b.e4b_last_path() == e4b.E4B_PATH_TCGEN05
     want = oracle.grouped_dgrad_ref(fmt, dy.float().numpy()[:R], offsets, rc, rs, N, K)
