@@ -202,7 +202,13 @@ E4B_DEV uint4 ldg_nc_v4(const void* p) {
   return r;
 }
 
-E4B_DEV float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u in fp32 with the hardware exp2 approximation and an approximate
+// reciprocal (__expf, __fdividef): relative error ~2^-20, so the bf16 h the
+// layer keeps is the correctly rounded value or one ulp off in rare elements.
+// The epilogues evaluate it once per gate/up pair; with IEEE expf and division
+// it took issue slots the tcgen05 path's decoder warps (on the same SM
+// sub-partitions) need. g -> -inf: __expf = inf and __fdividef(g, inf) = -0.
+E4B_DEV float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 // The gate_up activation of the expert variant (include/e4b.h): SwiGLU, or
 // the clamped GLU (u' + 1) * g' * sigmoid(alpha * g') with g' = min(g, limit)
@@ -211,7 +217,7 @@ E4B_DEV float glu_act(int act, float g, float u, float alpha, float limit) {
   if (act == E4B_ACT_CLAMPED_GLU) {
     g = g > limit ? limit : g;
     u = u > limit ? limit : (u < -limit ? -limit : u);
-    return (u + 1.0f) * g / (1.0f + expf(-alpha * g));
+    return __fdividef((u + 1.0f) * g, 1.0f + __expf(-alpha * g));
   }
   return silu_mul(g, u);
 }
