@@ -592,11 +592,17 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           }
           if (!fvalid) continue;
           const int64_t r0 = pbase + (isup ? 8 : 0);
+          uint16_t* o = out + r0 * p.ldo + f;
+          if (r0 + 8 <= T.p1) {
+            // all 8 rows valid (every chunk but an expert's last): no per-row check
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const int64_t pr = r0 + t;
-            if (pr < T.p1)
-              out[pr * p.ldo + f] = to_bf16_bits(glu_act(p.act, g[t] + bg, u[t] + bu, p.alpha, p.limit));
+            for (int t = 0; t < 8; ++t)
+              o[t * p.ldo] = to_bf16_bits(glu_act(p.act, g[t] + bg, u[t] + bu, p.alpha, p.limit));
+          } else {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              if (r0 + t < T.p1)
+                o[t * p.ldo] = to_bf16_bits(glu_act(p.act, g[t] + bg, u[t] + bu, p.alpha, p.limit));
           }
         }
       } else {
@@ -610,6 +616,25 @@ tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           tmem_ld_32x32b_x16(lane_base + uint32_t(cc * 16), g);
           tmem_ld_wait();
           if (!nvalid) continue;
+          if constexpr (EPI == kEpiGatedRows) {
+            if (pbase + 16 <= T.p1) {
+              // all 16 rows valid: the gates as four 16-byte shared loads (the
+              // same address for every lane), no per-row check
+              float gw[16];
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float4 q4 = reinterpret_cast<const float4*>(s_g + cc * 16)[v];
+                gw[4 * v] = q4.x;
+                gw[4 * v + 1] = q4.y;
+                gw[4 * v + 2] = q4.z;
+                gw[4 * v + 3] = q4.w;
+              }
+              float* o = static_cast<float*>(p.out) + pbase * p.ldo + n;
+#pragma unroll
+              for (int t = 0; t < 16; ++t) o[t * p.ldo] = gw[t] * (__uint_as_float(g[t]) + b0);
+              continue;
+            }
+          }
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
             const int64_t pr = pbase + t;
