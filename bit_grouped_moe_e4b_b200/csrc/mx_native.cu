@@ -554,6 +554,31 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         if constexpr (NMAT == 2) tmem_ld_32x32b_x16(lane_base + uint32_t(MBN + cc * 16), u);
         tmem_ld_wait();
         if (!nvalid) continue;
+        if (cc * 16 + 16 <= T.rows) {
+          // all 16 rows valid: no per-row check, pointer stepping (the gated
+          // rows' gates as four 16-byte shared loads; row ii is T.p0 + ii)
+          if constexpr (GATED) {
+            float gw[16];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 q4 = reinterpret_cast<const float4*>(s_g + cc * 16)[v];
+              gw[4 * v] = q4.x;
+              gw[4 * v + 1] = q4.y;
+              gw[4 * v + 2] = q4.z;
+              gw[4 * v + 3] = q4.w;
+            }
+            float* o = static_cast<float*>(p.out) + (T.p0 + cc * 16) * p.ldo + n;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) o[t * p.ldo] = gw[t] * (__uint_as_float(g[t]) + b0);
+          } else {
+            uint16_t* o = static_cast<uint16_t*>(p.out) + (T.pp0 + cc * 16) * p.ldo + n;
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              o[t * p.ldo] = to_bf16_bits(
+                  glu_act(p.act_fn, __uint_as_float(g[t]) + b0, __uint_as_float(u[t]) + b1, p.alpha, p.limit));
+          }
+          continue;
+        }
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int ii = cc * 16 + t;
