@@ -268,3 +268,14 @@ def test_expert_parallel_layer_rejects_a_bad_split():
             ExpertParallelLayer(_L(), 8)   # 8 experts on one rank, but the local layer holds 3
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (64, 2, 8), (8191, 2, 128), (8192, 2, 128), (4097, 4, 32),
+                                   (8192, 8, 128), (65536, 1, 1024)])
+def test_route_workspace_size_holds_the_many_cta_scratch(T, k, E):
+    # the status words (256 bytes); from 16384 routed slots also one int32
+    # histogram per 2048-slot chunk and expert, plus the chunk's bad-id count
+    n = e4b.e4b_route_workspace_size(T, k, E)
+    R = T * k
+    chunks = -(-R // 2048)
+    assert n == 256 + (chunks * (E + 1) * 4 if R >= 16384 else 0)
