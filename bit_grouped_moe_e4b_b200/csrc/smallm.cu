@@ -50,6 +50,10 @@ constexpr int kMaxTok = 16;                      // routed rows per pass (two ch
 // copy per half-warp lane (entry v of lane l at v * 128 + 8 * (l % 16)).
 // MXFP4: two bf16 values per entry, one copy per lane (v * 128 + 4 * l).
 constexpr int kLutBytes = 256 * 128;
+// MXFP4 scale table: 2^(s-127) as fp32 for every byte s, 8 copies side by
+// side ([s][g], g = the lane's fragment row modulo 8) so the 8 rows a warp
+// reads at once sit in 8 different banks.
+constexpr int kScaleTabBytes = 256 * 8 * 4;
 constexpr uint64_t kStageWaitNs = 100000000;  // 100 ms for a stage; 16x that for h of an expert
 constexpr uint64_t kDrainNs = 1000000000;     // the copies still landing at exit
 constexpr int kKSplit = 2048;                    // K slice of a down item
@@ -245,15 +249,18 @@ E4B_DEV void lut_lookup8(uint32_t lut_lane, uint32_t w, uint64_t absmax2, uint32
 }
 
 // Scale of block b of a row in a stage. NF4: the absmax staged at `slot`.
-// MXFP4: 2^(s-127) of byte b of `mx` (the row's 8 scale bytes of the chunk),
-// with byte 0 = 2^-127 and byte 255 = NaN.
+// MXFP4: 2^(s-127) for byte b of `mx` (the row's 8 scale bytes of the
+// chunk), looked up in this lane's column `tab_lane` of the scale table
+// (byte 0 = 2^-127, byte 255 = NaN).
 template <int FMT>
-E4B_DEV float stage_scale(uint32_t slot, int b, uint64_t mx) {
+E4B_DEV float stage_scale(uint32_t slot, int b, uint64_t mx, uint32_t tab_lane) {
   if constexpr (FMT == E4B_FMT_NF4) {
     return __uint_as_float(lds32(slot + uint32_t(4 * b)));
   } else {
-    const uint32_t e = uint32_t(mx >> (8 * b)) & 0xFFu;
-    return (e - 1u < 254u) ? __uint_as_float(e << 23) : e8m0_to_f32(e);
+    const uint32_t w = b < 4 ? uint32_t(mx) : uint32_t(mx >> 32);
+    const int sh = 8 * (b & 3);  // the byte's offset in w; the table row is 32 bytes
+    const uint32_t off = sh >= 5 ? (w >> (sh - 5)) & 0x1FE0u : (w << 5) & 0x1FE0u;
+    return __uint_as_float(lds32(tab_lane + off));
   }
 }
 
@@ -261,6 +268,11 @@ E4B_DEV float stage_scale(uint32_t slot, int b, uint64_t mx) {
 // bytes [o, o + 8), read through L1; words past the end read as zero bytes.
 E4B_DEV void mx_words(const uint8_t* scales, int64_t n, int64_t o, uint32_t (&w)[3]) {
   const int64_t a = o & ~int64_t(3);
+  if (a + 12 <= n) {  // every row but the array's last few: three plain loads
+#pragma unroll
+    for (int j = 0; j < 3; ++j) w[j] = __ldg(reinterpret_cast<const uint32_t*>(scales + a + 4 * j));
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
     const int64_t q = a + 4 * j;
@@ -294,7 +306,9 @@ struct Geo {
   static constexpr int kSlot = 16;
   static constexpr int kStageBytes = kSOff + kRows * kSlot;
   static constexpr int kStages = 4;
-  static constexpr int kSmemBytes = 1024 + kLutBytes + kStages * kStageBytes + 256;  // + alignment, barriers, info
+  // MXFP4: + the e8m0 scale table after the barriers and stage info
+  static constexpr int kTabBytes = FMT == E4B_FMT_MXFP4 ? kScaleTabBytes : 0;
+  static constexpr int kSmemBytes = 1024 + kLutBytes + kStages * kStageBytes + 256 + kTabBytes;
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(kSmemBytes + 8192 <= 232448, "shared memory budget");
 };
@@ -501,7 +515,7 @@ E4B_DEV void produce(const Maps& maps, const Params& p, const Work& W, const int
 // hence inside one scale block of each row.
 template <int FMT, int NT, bool SA>
 E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, int rB, uint64_t mxA,
-                           uint64_t mxB, uint32_t lut_lane, float (&acc)[2][4]) {
+                           uint64_t mxB, uint32_t lut_lane, uint32_t tab_lane, float (&acc)[2][4]) {
   static_assert(SA || FMT == E4B_FMT_NF4, "MXFP4 scales always apply after the block's MMA");
   constexpr int kSlot = Geo<FMT>::kSlot;
   constexpr int BLK = FMT == E4B_FMT_NF4 ? 64 : 32;  // weights per scale block
@@ -512,11 +526,18 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
   const int c = lane & 3;
   const uint32_t cA = st + uint32_t(kCodeOff + (rA + g) * 128 + 4 * c);  // both rows are g modulo 8
   const uint32_t cB = st + uint32_t(kCodeOff + (rB + g) * 128 + 4 * c);
+  uint32_t x_lane[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) x_lane[j] = uint32_t(min(8 * j + g, f.ntok - 1) * 64 + 16 * c);
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    const bool live = f.kc + BLK * b < kend;  // blocks past K: codes are zero, scale 0
-    const float sA = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rA + g) * kSlot), b, mxA) : 0.f;
-    const float sB = live ? stage_scale<FMT>(st + uint32_t(kSOff + (rB + g) * kSlot), b, mxB) : 0.f;
+    // blocks past K: codes and activations are zero, scale 0. The scale slot
+    // of every block exists, so it is read either way and then selected.
+    const bool live = f.kc + BLK * b < kend;
+    float sA = stage_scale<FMT>(st + uint32_t(kSOff + (rA + g) * kSlot), b, mxA, tab_lane);
+    float sB = stage_scale<FMT>(st + uint32_t(kSOff + (rB + g) * kSlot), b, mxB, tab_lane);
+    sA = live ? sA : 0.f;
+    sB = live ? sB : 0.f;
     const uint64_t sA2 = (uint64_t(__float_as_uint(sA)) << 32) | __float_as_uint(sA);
     const uint64_t sB2 = (uint64_t(__float_as_uint(sB)) << 32) | __float_as_uint(sB);
     float P[NT][4];
@@ -527,14 +548,13 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
 #pragma unroll
     for (int it = 0; it < CPB; ++it) {
       const int ch = CPB * b + it;  // 32-wide chunk of the stage
-      // activations: 8 values of this lane's token in each chunk of 8 routed rows
+      // activations: 8 values of this lane's token in each chunk of 8 routed
+      // rows. Lanes past the pass's routed rows read the last routed row
+      // instead (no branch; the same addresses as other lanes): those values
+      // reach only MMA columns that no epilogue stores.
       uint4 xv[NT];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        const int tok = 8 * j + g;
-        xv[j] = tok < f.ntok ? lds128(st + uint32_t(kXOff + ch * kMaxTok * 64 + tok * 64 + 16 * c))
-                             : make_uint4(0, 0, 0, 0);
-      }
+      for (int j = 0; j < NT; ++j) xv[j] = lds128(st + uint32_t(kXOff + ch * kMaxTok * 64) + x_lane[j]);
       const uint32_t sw = uint32_t((ch ^ g) << 4);  // the 128B swizzle of chunk ch in row g (mod 8)
       uint32_t dA[4], dB[4];
       lut_lookup8<SA>(lut_lane, lds32(cA + sw), sA2, dA);
@@ -567,7 +587,8 @@ E4B_DEV void consume_stage(uint32_t st, const StageInfo& f, int kend, int rA, in
 // and up rows of an output are neighbours, four lanes apart in the fragment.
 template <int FMT, bool SA>
 E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t* empty,
-                     const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, uint64_t limit) {
+                     const StageInfo* info, volatile int* s_abort, uint32_t lut_lane, uint32_t tab_lane,
+                     uint64_t limit) {
   constexpr int kStages = Geo<FMT>::kStages;
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;  // 0 .. kConsumers-1
@@ -635,8 +656,8 @@ E4B_DEV void consume(const Params& p, uint8_t* stages, uint64_t* full, uint64_t*
         mx_words(scales, n, oB + 8, pfB);
       }
     }
-    if (f.ntok > 8) consume_stage<FMT, 2, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
-    else consume_stage<FMT, 1, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, acc);
+    if (f.ntok > 8) consume_stage<FMT, 2, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, tab_lane, acc);
+    else consume_stage<FMT, 1, SA>(st, f, kend, rA, rB, mxA, mxB, lut_lane, tab_lane, acc);
     mbar_arrive(&empty[s]);  // this lane's reads of the stage are done
     if (!f.last) continue;
 
@@ -721,9 +742,16 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
   uint64_t* empty = full + kStages;
   StageInfo* info = reinterpret_cast<StageInfo*>(empty + kStages);
   volatile int* s_abort = reinterpret_cast<volatile int*>(info + kStages);
+  static_assert(2 * kStages * sizeof(uint64_t) + kStages * sizeof(StageInfo) + sizeof(int) <= 256,
+                "barriers, stage info and the abort flag fit their 256 bytes");
+  float* scale_tab = reinterpret_cast<float*>(stages + kStages * Geo<FMT>::kStageBytes + 256);
 
-  // The byte table (made visible by the barriers of the clearing loop below).
+  // The byte table (and, for MXFP4, the scale table), made visible by the
+  // barrier that ends build_lut.
   __shared__ float s_val[16];
+  if constexpr (FMT == E4B_FMT_MXFP4)
+    for (int i = threadIdx.x; i < kScaleTabBytes / 4; i += blockDim.x)
+      scale_tab[i] = e8m0_to_f32(uint32_t(i >> 3));
   build_lut<FMT, SA>(smem, s_val);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -757,7 +785,9 @@ smallm_layer_kernel(const __grid_constant__ Maps maps, const Params p) {
     grid_launch_dependents();
   } else {
     const uint32_t lut_lane = smem_u32(smem) + uint32_t(!SA ? 8 * (lane & 15) : 4 * lane);
-    consume<FMT, SA>(p, stages, full, empty, info, s_abort, lut_lane, limit);
+    // MXFP4: this lane's column of the scale table
+    const uint32_t tab_lane = smem_u32(scale_tab) + uint32_t(4 * ((lane >> 2) & 7));
+    consume<FMT, SA>(p, stages, full, empty, info, s_abort, lut_lane, tab_lane, limit);
   }
 }
 
