@@ -333,13 +333,61 @@ def run_gpu(wl, T, steps, warmup, rank, world, dist, layer=None, flags=0):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_serial_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+
+    # the same calls pipelined the way a serving loop runs them: step i's
+    # inputs go up on one copy stream while step i-1 computes, and step i's
+    # output comes down on another while step i+1 computes (two device
+    # buffers of each; every step's bytes still cross PCIe inside the timed
+    # region, which opens before the first upload and closes after the last
+    # download)
+    nb = 2
+    xs = [x_d] + [torch.empty_like(x) for _ in range(nb - 1)]
+    idss = [ids_d] + [torch.empty_like(ids) for _ in range(nb - 1)]
+    gs_ = [g_d] + [torch.empty_like(gates) for _ in range(nb - 1)]
+    ys = [y] + [torch.empty_like(y) for _ in range(nb - 1)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    uploaded = [torch.cuda.Event() for _ in range(nb)]
+    computed = [torch.cuda.Event() for _ in range(nb)]
+    downloaded = [torch.cuda.Event() for _ in range(nb)]
+    for e_ in uploaded + computed + downloaded:  # created on first record
+        e_.record(stream)
+
+    def pipelined(n):
+        for i in range(n):
+            b = i % nb
+            up.wait_event(computed[b])  # step i - nb no longer reads buffer b
+            with torch.cuda.stream(up):
+                xs[b].copy_(x_pin, non_blocking=True)
+                idss[b].copy_(ids_pin, non_blocking=True)
+                gs_[b].copy_(g_pin, non_blocking=True)
+            uploaded[b].record(up)
+            stream.wait_event(uploaded[b])
+            stream.wait_event(downloaded[b])  # y of step i - nb has left buffer b
+            e4b.e4b_moe_forward(layer, xs[b], idss[b], gs_[b], ys[b], ws, flags, stream=stream)
+            computed[b].record(stream)
+            down.wait_event(computed[b])
+            with torch.cuda.stream(down):
+                y_pin.copy_(ys[b], non_blocking=True)
+            downloaded[b].record(down)
+        for b in range(nb):
+            stream.wait_event(downloaded[b])
+
+    pipelined(warmup)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    up.wait_event(e0)
+    pipelined(steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     if e4b.e4b_read_device_status(ws) != 0:
         raise RuntimeError("device status set during the timed loops")
     return {
         "ms": ms, "phases": phases, "clocks": clk, "path": path,
-        "launches": launches_per_step * steps, "e2e_ms": e2e_ms,
+        "launches": launches_per_step * steps, "e2e_ms": e2e_ms, "e2e_serial_ms": e2e_serial_ms,
         "h2d": x_h.numel() * 2 + ids_h.nbytes + gates_h.nbytes, "d2h": T * wl.H * 2,
         "ids": ids_h, "layer": layer, "x": x_h, "gates": gates_h,
     }
@@ -922,7 +970,10 @@ def main():
                                   power_capped="sw_power_cap" in r["clocks"].get("reasons", [])),
             "clocks": r["clocks"],
             "e2e": {"value": world * T_i / (r["e2e_ms"] * 1e-3 / args.steps), "unit": "tokens/s",
-                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                    "copies": "pipelined: step i+1's upload and step i-1's download overlap step i "
+                              "(two copy streams, double-buffered device inputs and outputs)",
+                    "serial_value": world * T_i / (r["e2e_serial_ms"] * 1e-3 / args.steps)},
             "gpu_launches": r["launches"],
         }
         if not args.sweep and not args.no_per_config and world == 1:

@@ -130,6 +130,35 @@ def test_block_scales_and_large_outputs(fmt, E, H, I, T, k, path):
         assert scaled_err(y, y_ref) < scaled_err(y, other), (path, mode)
 
 
+@pytest.mark.parametrize("path", ["gemv", "tcgen05", "tcgen05_1sm"])
+def test_mxfp4_special_scale_bytes(path):
+    # e8m0 (OCP MX v1.0): byte 255 is NaN and byte 0 is 2^-127. One NaN block
+    # in a down row makes exactly that output column NaN for the tokens routed
+    # to the expert; one in an up row makes every output of the expert's
+    # tokens NaN (through h). Byte-0 blocks stay finite.
+    E, H, I, T, k = 3, 288, 224, 40, 2
+    layer, (gc, gs, dc, ds) = small_layer("mxfp4", E, H, I, seed=11, std=0.06)
+    gs, ds = gs.copy(), ds.copy()
+    gs[0, 5, 1] = gs[0, 200, 0] = gs[0, 17, 8] = 0  # gate and up blocks of 2^-127
+    ds[0, 100, 6] = 0
+    ds[1, 7, 3] = 255  # output column 7 of expert 1
+    gs[2, I + 76, 4] = 255  # up row 76 of expert 2
+    layer.gate_up_scales.copy_(torch.from_numpy(gs))
+    layer.down_scales.copy_(torch.from_numpy(ds))
+    x = _x(T, H, seed=5)
+    ids, gates = synth.random_ids(np.random.default_rng(6), T, k, E)
+    to1, to2 = np.any(ids == 1, axis=1), np.any(ids == 2, axis=1)
+    assert to1.any() and to2.any() and not (to1 | to2).all()
+    y, status, _ = run_layer(layer, x, ids, gates, PATHS[path])
+    y_ref = oracle_layer("mxfp4", x, ids, gates, (gc, gs, dc, ds), E, H, I)
+    want_nan = to2[:, None] | (to1[:, None] & (np.arange(H) == 7)[None, :])
+    assert status == 0
+    assert np.array_equal(np.isnan(y_ref), want_nan)
+    assert np.array_equal(np.isnan(y), want_nan), path
+    fin = ~want_nan
+    assert_close(y[fin], y_ref[fin], f"mxfp4 special scale bytes {path}")
+
+
 EDGE = {
     "single_slot": (1, 1, lambda T, k, E: np.zeros((1, 1), np.int32)),
     "all_on_one_expert": (300, 2, lambda T, k, E: np.full((T, k), 3, np.int32)),
