@@ -31,8 +31,9 @@
 //     fp32 accumulators in shared memory, which the epilogue (store / SwiGLU
 //     / gate-weighted combine over the routed slots) turns into bf16;
 //   * the kernel is a programmatic dependent of the work before it on the
-//     stream: it waits (griddepcontrol.wait) only before it reads x, the ids
-//     and gates (or, with E4B_FLAG_IDS_READY, after its first copies), and
+//     stream: it waits (griddepcontrol.wait) before it reads the ids and
+//     gates (with E4B_FLAG_IDS_READY only before it reads x, so its set-up
+//     overlaps that work), quantises x before its first weight copies, and
 //     lets the next kernel launch once its copies are all issued.
 #include <cuda_fp16.h>
 
@@ -487,15 +488,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     const uint32_t i0 = streams ? uint32_t(uint64_t(warp) * items / q.warps) : 0;
     const uint32_t i1 = streams ? uint32_t(uint64_t(warp + 1) * items / q.warps) : 0;
     for (uint32_t i = tid; i < 2 * nout; i += blockDim.x) s_acc[i] = 0.f;
-    // the first item (and its scales) is on its way while the activation rows
-    // are quantised; the other stages start at the top of the item loop (a
-    // burst of copies at the start would hold up the quantisation's loads)
+    // the activation rows are quantised before the first weight copies
+    // start: copies issued earlier hold up the quantisation's loads behind
+    // them (one token through the decode layer: quantisation 6-7 -> 4-5 us a
+    // launch, the two-launch step 74.8 -> 70.7 us, timed on one B200)
     Cursor ki{}, kc{};
     if (i0 < i1) {
       cursor_init<EPI>(ki, i0, p, q, r0);
       kc = ki;
     }
     uint32_t issued = i0, waited = i0;
+    if (first) {
+      if (ids_ready) grid_dependency_wait();
+      quantize_rows(p, xs, s_sx, s_red);  // ends with __syncthreads (s_acc cleared too)
+      first = false;
+    } else {
+      __syncthreads();  // s_acc cleared
+    }
     if (issued < i1) {
       issue_item<EPI>(ki, nout, p, q, s_ids, my_desc, my_ring, my_bar, lane);
       cursor_next<EPI>(ki, p, q);
@@ -503,14 +512,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) int4_gemv_kernel(const Int4Ge
     }
     uint32_t hn[kRows][kLaneBlocks];  // scales of the next item (when they are not copied)
     if (!q.sbulk && i0 < i1) load_scales(my_desc[0], lane, hn);
-    if (first) {
-      // with the ids ready the first weight copies are already on their way
-      if (ids_ready) grid_dependency_wait();
-      quantize_rows(p, xs, s_sx, s_red);  // ends with __syncthreads (s_acc cleared too)
-      first = false;
-    } else {
-      __syncthreads();  // s_acc cleared
-    }
     bool ok = true;
     for (uint32_t it = i0; it < i1; ++it) {
       // keep kStages items in flight: the stages of items before `it` are free

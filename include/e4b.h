@@ -93,8 +93,9 @@ typedef enum {
 #define E4B_FLAG_NF4_PRODUCT_DECODE 0x8u
 /* e4b_gemv_int4_b32: the expert ids and gates are not written by the work
  * queued just before the call on the stream (they are ready when the call is
- * enqueued), so the kernel may start streaming the routed experts' weights
- * before that work completes. It still waits for it before reading x. */
+ * enqueued), so the kernel reads them and sets up its work before that work
+ * completes. It still waits for it before reading x (and streams weights only
+ * after quantising x). */
 #define E4B_FLAG_IDS_READY 0x10u
 /* MXFP4 layers with prepared stacks (e4b_moe_weights.*_mx_*), large-M path:
  * each activation row enters the block-scaled MMA as ONE e4m3 term per value
