@@ -271,7 +271,9 @@ def unpack_mxfp4_codes(blocks) -> np.ndarray:
 
 def dequant_mxfp4(blocks, scales) -> np.ndarray:
     """Decode MXFP4 to fp32 [..., N, K]: sign * e2m1 * 2^(scale - 127).
-    The values are exact in fp32 and in bf16."""
+    The values are exact in fp32 and in bf16 where they are in range; the
+    few past fp32's largest value (scale byte 254 with magnitude >= 2, byte
+    253 with magnitude 4 or 6) become +-inf."""
     codes = unpack_mxfp4_codes(blocks)
     mag = E2M1_MAGNITUDES[codes & 7]
     val = np.where(codes & 8, -mag, mag)
@@ -279,7 +281,8 @@ def dequant_mxfp4(blocks, scales) -> np.ndarray:
     out = np.ldexp(val, (s - 127)[..., None])
     out = np.where((s == 255)[..., None], np.nan, out)
     out = out.reshape(*out.shape[:-2], out.shape[-2] * out.shape[-1])
-    return out.astype(np.float32)
+    with np.errstate(over="ignore"):  # the out-of-range values above
+        return out.astype(np.float32)
 
 
 def packed_bytes_per_weight(fmt: str) -> float:
